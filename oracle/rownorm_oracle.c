@@ -1,0 +1,161 @@
+/*
+ * Row-normalization ORACLE: plain, slow, fp64 CPU reference.
+ *
+ * TEST INFRASTRUCTURE ONLY. This file is built and called by the test suite,
+ * by the entry module's smoke check and by the CPU-baseline leg of the
+ * benchmark. The product library never links, loads or calls it, and it
+ * shares no code, header, constant or helper with the CUDA path.
+ *
+ * What it computes (one row at a time, every sum in fp64, plain sequential
+ * order, no blocking or reordering):
+ *
+ *   RMSNorm   -- "Fused transformer kernels on Emily", Part 1 (the composed
+ *                RMSNorm written with Nx primitives) and "Emily.Fast",
+ *                `rms_norm/3`:
+ *                  y_j = x_j / sqrt( (1/D) * sum_i x_i^2 + eps ) * w_j
+ *
+ *   LayerNorm -- "Emily.Fast", `layer_norm/4`:
+ *                  mu      = (1/D) * sum_i x_i
+ *                  var     = (1/D) * sum_i (x_i - mu)^2
+ *                  y_j     = (x_j - mu) / sqrt(var + eps) * w_j + b_j
+ *                The page names the statistic "Welford-style" mean and
+ *                variance; that is a way of computing the same population
+ *                mean and variance, so the oracle writes out the definition.
+ *
+ *   Dual q/k head RMSNorm -- "norm_fusion.rs" (mlx_c_rust compile module),
+ *                `build_dual_head_norm_graph` / `apply_compiled_dual_head_norm`:
+ *                the RMSNorm of the query rows with the query weight, and the
+ *                RMSNorm of the key rows with the key weight, one eps shared,
+ *                returned queries first, keys second.
+ *
+ * Readings where the pages are silent (each is listed in the design doc):
+ *   - the variance divisor is D (population variance);
+ *   - eps travels as a binary32 value (norm_fusion.rs keeps it as f32 bits)
+ *     and is promoted exactly to fp64 here;
+ *   - a null weight means all ones, a null bias all zeros.
+ *
+ * Inputs are [rows, dim] views whose last axis is contiguous and whose rows
+ * start row_stride elements apart. Element type 0 = binary32, 1 = bfloat16
+ * (raw 16-bit patterns). Every input element is decoded exactly to fp64.
+ * Outputs are dense [rows, dim] fp64 arrays.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#define ORACLE_F32 0
+#define ORACLE_BF16 1
+
+/* bfloat16 is, by its definition, the upper 16 bits of an IEEE binary32
+ * value; placing the pattern there and widening is exact. */
+static double decode_element(const void *base, int dtype, int64_t index) {
+    if (dtype == ORACLE_F32) {
+        float f;
+        memcpy(&f, (const char *)base + 4 * index, 4);
+        return (double)f;
+    }
+    uint16_t half;
+    memcpy(&half, (const char *)base + 2 * index, 2);
+    uint32_t bits = (uint32_t)half << 16;
+    float f;
+    memcpy(&f, &bits, 4);
+    return (double)f;
+}
+
+static int check_view(const void *x, int dtype, int64_t rows, int64_t dim,
+                      int64_t row_stride) {
+    if (x == NULL && rows > 0) return 1;
+    if (dtype != ORACLE_F32 && dtype != ORACLE_BF16) return 2;
+    if (rows < 0 || dim < 1 || row_stride < dim) return 3;
+    return 0;
+}
+
+/* One RMSNorm row, exactly in the order the composed formula states. */
+static void rms_norm_row(const void *x, int dtype, int64_t row, int64_t dim,
+                         int64_t row_stride, const void *w, double eps,
+                         double *y_row) {
+    const int64_t first = row * row_stride;
+    double sum_sq = 0.0;
+    for (int64_t i = 0; i < dim; ++i) {
+        double v = decode_element(x, dtype, first + i);
+        sum_sq += v * v;
+    }
+    double mean_sq = sum_sq / (double)dim;
+    double rms = sqrt(mean_sq + eps);
+    for (int64_t j = 0; j < dim; ++j) {
+        double v = decode_element(x, dtype, first + j);
+        double weight = (w != NULL) ? decode_element(w, dtype, j) : 1.0;
+        y_row[j] = v / rms * weight;
+    }
+}
+
+/* One LayerNorm row: population mean, population variance, then affine. */
+static void layer_norm_row(const void *x, int dtype, int64_t row, int64_t dim,
+                           int64_t row_stride, const void *w, const void *b,
+                           double eps, double *y_row) {
+    const int64_t first = row * row_stride;
+    double sum = 0.0;
+    for (int64_t i = 0; i < dim; ++i) sum += decode_element(x, dtype, first + i);
+    double mean = sum / (double)dim;
+    double sum_dev_sq = 0.0;
+    for (int64_t i = 0; i < dim; ++i) {
+        double dev = decode_element(x, dtype, first + i) - mean;
+        sum_dev_sq += dev * dev;
+    }
+    double var = sum_dev_sq / (double)dim;
+    double denom = sqrt(var + eps);
+    for (int64_t j = 0; j < dim; ++j) {
+        double v = decode_element(x, dtype, first + j);
+        double weight = (w != NULL) ? decode_element(w, dtype, j) : 1.0;
+        double bias = (b != NULL) ? decode_element(b, dtype, j) : 0.0;
+        y_row[j] = (v - mean) / denom * weight + bias;
+    }
+}
+
+/* Rows are independent; nthreads > 1 only spreads whole rows over threads
+ * and leaves every row's arithmetic exactly as above. */
+int oracle_rms_norm(const void *x, int dtype, int64_t rows, int64_t dim,
+                    int64_t row_stride, const void *w, float eps, double *y,
+                    int nthreads) {
+    int status = check_view(x, dtype, rows, dim, row_stride);
+    if (status) return status;
+    if (rows > 0 && y == NULL) return 1;
+    const double eps64 = (double)eps;
+    (void)nthreads;
+#pragma omp parallel for schedule(static) num_threads(nthreads > 0 ? nthreads : 1)
+    for (int64_t r = 0; r < rows; ++r)
+        rms_norm_row(x, dtype, r, dim, row_stride, w, eps64, y + r * dim);
+    return 0;
+}
+
+int oracle_layer_norm(const void *x, int dtype, int64_t rows, int64_t dim,
+                      int64_t row_stride, const void *w, const void *b,
+                      float eps, double *y, int nthreads) {
+    int status = check_view(x, dtype, rows, dim, row_stride);
+    if (status) return status;
+    if (rows > 0 && y == NULL) return 1;
+    const double eps64 = (double)eps;
+    (void)nthreads;
+#pragma omp parallel for schedule(static) num_threads(nthreads > 0 ? nthreads : 1)
+    for (int64_t r = 0; r < rows; ++r)
+        layer_norm_row(x, dtype, r, dim, row_stride, w, b, eps64, y + r * dim);
+    return 0;
+}
+
+/* Queries first, keys second; both with the one shared eps. */
+int oracle_dual_head_rms_norm(const void *q, int64_t q_rows, int64_t q_dim,
+                              int64_t q_stride, const void *k, int64_t k_rows,
+                              int64_t k_dim, int64_t k_stride, int dtype,
+                              const void *wq, const void *wk, float eps,
+                              double *yq, double *yk, int nthreads) {
+    int status = oracle_rms_norm(q, dtype, q_rows, q_dim, q_stride, wq, eps, yq,
+                                 nthreads);
+    if (status) return status;
+    return oracle_rms_norm(k, dtype, k_rows, k_dim, k_stride, wk, eps, yk,
+                           nthreads);
+}
+
+/* Exposed so the test suite can pin the element decoding on its own. */
+void oracle_decode(const void *src, int dtype, int64_t n, double *dst) {
+    for (int64_t i = 0; i < n; ++i) dst[i] = decode_element(src, dtype, i);
+}

@@ -1,0 +1,82 @@
+"""Plant plausible mistakes in a COPY of the oracle (on the CPU) and require
+each one to trip at least one pin. This is what shows the pins would catch a
+dropped term, a wrong sign, a wrong divisor, a wrong index or a swapped
+operand in the oracle."""
+import os
+
+import pytest
+
+import oracle
+import oracle_pins
+from oracle import build as oracle_build
+
+with open(oracle_build.SOURCE) as _f:
+    SOURCE = _f.read()
+
+MUTANTS = {
+    "rms divisor D-1": ("double mean_sq = sum_sq / (double)dim;",
+                        "double mean_sq = sum_sq / (double)(dim - 1);"),
+    "rms divisor D+1": ("double mean_sq = sum_sq / (double)dim;",
+                        "double mean_sq = sum_sq / (double)(dim + 1);"),
+    "rms drops eps": ("sqrt(mean_sq + eps)", "sqrt(mean_sq)"),
+    "rms eps outside sqrt": ("sqrt(mean_sq + eps)", "(sqrt(mean_sq) + eps)"),
+    "rms drops weight": ("y_row[j] = v / rms * weight;", "y_row[j] = v / rms;"),
+    "rms squares weight": ("y_row[j] = v / rms * weight;",
+                           "y_row[j] = v / rms * weight * weight;"),
+    "rms multiplies by rms": ("y_row[j] = v / rms * weight;",
+                              "y_row[j] = v * rms * weight;"),
+    "rms sums |x| not x^2": ("sum_sq += v * v;", "sum_sq += fabs(v);"),
+    "rms ignores row offset": (
+        "double v = decode_element(x, dtype, first + j);\n        double weight = (w != NULL) ? decode_element(w, dtype, j) : 1.0;\n        y_row[j] = v / rms",
+        "double v = decode_element(x, dtype, j);\n        double weight = (w != NULL) ? decode_element(w, dtype, j) : 1.0;\n        y_row[j] = v / rms"),
+    "rms weight reversed": (
+        "double weight = (w != NULL) ? decode_element(w, dtype, j) : 1.0;\n        y_row[j] = v / rms",
+        "double weight = (w != NULL) ? decode_element(w, dtype, dim - 1 - j) : 1.0;\n        y_row[j] = v / rms"),
+    "row stride ignored": ("const int64_t first = row * row_stride;\n    double sum_sq",
+                           "const int64_t first = row * dim;\n    double sum_sq"),
+    "ln mean divisor D-1": ("double mean = sum / (double)dim;",
+                            "double mean = sum / (double)(dim - 1);"),
+    "ln sample variance": ("double var = sum_dev_sq / (double)dim;",
+                           "double var = sum_dev_sq / (double)(dim - 1);"),
+    "ln raw second moment": ("double dev = decode_element(x, dtype, first + i) - mean;",
+                             "double dev = decode_element(x, dtype, first + i);"),
+    "ln output misses mean": ("y_row[j] = (v - mean) / denom * weight + bias;",
+                              "y_row[j] = v / denom * weight + bias;"),
+    "ln output adds mean": ("y_row[j] = (v - mean) / denom * weight + bias;",
+                            "y_row[j] = (v + mean) / denom * weight + bias;"),
+    "ln bias sign": ("y_row[j] = (v - mean) / denom * weight + bias;",
+                     "y_row[j] = (v - mean) / denom * weight - bias;"),
+    "ln bias scaled by weight": ("y_row[j] = (v - mean) / denom * weight + bias;",
+                                 "y_row[j] = ((v - mean) / denom + bias) * weight;"),
+    "ln drops eps": ("double denom = sqrt(var + eps);", "double denom = sqrt(var);"),
+    "ln eps outside sqrt": ("double denom = sqrt(var + eps);", "double denom = sqrt(var) + eps;"),
+    "ln weight and bias swapped": (
+        "double weight = (w != NULL) ? decode_element(w, dtype, j) : 1.0;\n        double bias = (b != NULL) ? decode_element(b, dtype, j) : 0.0;",
+        "double weight = (b != NULL) ? decode_element(b, dtype, j) : 1.0;\n        double bias = (w != NULL) ? decode_element(w, dtype, j) : 0.0;"),
+    "dual query uses key weight": (
+        "oracle_rms_norm(q, dtype, q_rows, q_dim, q_stride, wq, eps, yq,",
+        "oracle_rms_norm(q, dtype, q_rows, q_dim, q_stride, wk, eps, yq,"),
+    "bf16 decoded with wrong shift": ("(uint32_t)half << 16", "(uint32_t)half << 15"),
+}
+
+
+def _mutant(tmp_path_factory, name):
+    old, new = MUTANTS[name]
+    assert SOURCE.count(old) == 1, f"mutation site for {name!r} must be unique"
+    d = tmp_path_factory.mktemp("mutant")
+    src = os.path.join(d, "mutant.c")
+    with open(src, "w") as f:
+        f.write(SOURCE.replace(old, new))
+    return oracle.Oracle(oracle_build.compile_source(src, os.path.join(d, "libmutant.so")))
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(tmp_path_factory, name):
+    orc = _mutant(tmp_path_factory, name)
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(orc)
+        except (AssertionError, ValueError, FloatingPointError, ZeroDivisionError) as e:
+            caught.append(pin.__name__)
+    assert caught, f"no pin catches the planted mistake {name!r}"

@@ -1,0 +1,166 @@
+"""Seeded synthetic workloads for row normalization.
+
+This module holds the input recipes shared by the tests and the benchmark:
+shapes, value distributions, seeds. It contains none of the normalization
+arithmetic. Values are drawn in float32 with a seeded ``torch.Generator`` on
+the requested device (CPU: Mersenne Twister; CUDA: Philox) and rounded to
+bfloat16 with round-to-nearest-even where the workload is bfloat16. Parity
+checks always hand the oracle the exact bytes that the GPU reads, so the two
+generators never need to agree with each other.
+
+Workloads (shapes follow the pages' examples):
+  rms_f32_4x128x1024      RMSNorm f32; the batch=4, seq=128, hidden=1024
+                          block of "Fused transformer kernels on Emily",
+                          Part 1, Correctness; values U(-1,1), w U(0.5,1.5).
+  ln_f32_1x1024x768       LayerNorm f32; the (1, 1024, 768) tower shape of
+                          "kernel_micro_ab.rs", section 1 (LayerNorm); x
+                          U(-1,1), w U(0.5,1.5), b U(-0.1,0.1), eps 1e-6.
+  dual_bf16_prefill       q [8192, 32, 128], k [8192, 8, 128] N(0,1),
+                          wq, wk N(1, 0.1) -- the query/key head norms of
+                          "norm_fusion.rs" at a prefill token count.
+  dual_bf16_decode        the same heads at one token (decode).
+  rms_bf16_16x4096x4096   RMSNorm bf16, N(0,1) with 1 % of entries x50.
+  ln_bf16_65536x{D}       LayerNorm bf16, N(0.5, 2), every 64th row constant.
+"""
+from dataclasses import dataclass, field
+from typing import Dict, Optional, Tuple
+
+import torch
+
+LN_WIDTHS = (768, 1000, 4097, 8192, 16384)
+CONSTANT_ROW_PERIOD = 64
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    op: str                      # "rms", "ln" or "dual"
+    dtype: torch.dtype
+    shape: Tuple[int, ...]       # x (or q) shape; last axis is the row
+    eps: float
+    seed: int
+    k_shape: Optional[Tuple[int, ...]] = None
+    meta: Dict[str, float] = field(default_factory=dict)
+
+    @property
+    def dim(self) -> int:
+        return self.shape[-1]
+
+    @property
+    def rows(self) -> int:
+        n = 1
+        for s in self.shape[:-1]:
+            n *= s
+        return n
+
+    @property
+    def k_rows(self) -> int:
+        if self.k_shape is None:
+            return 0
+        n = 1
+        for s in self.k_shape[:-1]:
+            n *= s
+        return n
+
+    @property
+    def total_rows(self) -> int:
+        return self.rows + self.k_rows
+
+    @property
+    def element_size(self) -> int:
+        return torch.empty((), dtype=self.dtype).element_size()
+
+    def algorithmic_bytes(self) -> int:
+        """Read x + write y + read each per-column vector once."""
+        s = self.element_size
+        if self.op == "dual":
+            kd = self.k_shape[-1]
+            return (2 * self.rows * self.dim * s + self.dim * s
+                    + 2 * self.k_rows * kd * s + kd * s)
+        vectors = 2 if self.op == "ln" else 1
+        return 2 * self.rows * self.dim * s + vectors * self.dim * s
+
+
+WORKLOADS: Dict[str, Workload] = {}
+
+
+def _register(w: Workload) -> Workload:
+    WORKLOADS[w.name] = w
+    return w
+
+
+_register(Workload("rms_f32_4x128x1024", "rms", torch.float32, (4, 128, 1024), 1e-6, 1))
+_register(Workload("ln_f32_1x1024x768", "ln", torch.float32, (1, 1024, 768), 1e-6, 2))
+_register(Workload("dual_bf16_prefill", "dual", torch.bfloat16, (8192, 32, 128), 1e-6, 3,
+                   k_shape=(8192, 8, 128)))
+_register(Workload("dual_bf16_decode", "dual", torch.bfloat16, (1, 32, 128), 1e-6, 30,
+                   k_shape=(1, 8, 128)))
+_register(Workload("rms_bf16_16x4096x4096", "rms", torch.bfloat16, (16, 4096, 4096), 1e-5, 4))
+for _k, _d in enumerate(LN_WIDTHS):
+    _register(Workload(f"ln_bf16_65536x{_d}", "ln", torch.bfloat16, (65536, _d), 1e-5, 50 + _k))
+
+# The large bf16 workloads: one pass over each is one benchmark step.
+LARGE_SUITE = ("dual_bf16_prefill", "rms_bf16_16x4096x4096") + tuple(
+    f"ln_bf16_65536x{d}" for d in LN_WIDTHS)
+SMALL_SUITE = ("rms_f32_4x128x1024", "ln_f32_1x1024x768", "dual_bf16_decode")
+
+
+def _gen(device, seed):
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def _uniform(shape, lo, hi, g, device):
+    return torch.rand(shape, generator=g, device=device, dtype=torch.float32) * (hi - lo) + lo
+
+
+def _normal(shape, mean, std, g, device):
+    return torch.randn(shape, generator=g, device=device, dtype=torch.float32) * std + mean
+
+
+def make_inputs(w: Workload, device="cpu") -> Dict[str, torch.Tensor]:
+    """Draw the workload's tensors on ``device`` (a fixed draw order per
+    workload: x, then the per-column vectors, then masks/constants)."""
+    device = torch.device(device)
+    g = _gen(device, w.seed)
+    out: Dict[str, torch.Tensor] = {}
+    if w.name in ("rms_f32_4x128x1024",):
+        out["x"] = _uniform(w.shape, -1.0, 1.0, g, device)
+        out["w"] = _uniform((w.dim,), 0.5, 1.5, g, device)
+    elif w.name == "ln_f32_1x1024x768":
+        out["x"] = _uniform(w.shape, -1.0, 1.0, g, device)
+        out["w"] = _uniform((w.dim,), 0.5, 1.5, g, device)
+        out["b"] = _uniform((w.dim,), -0.1, 0.1, g, device)
+    elif w.op == "dual":
+        out["q"] = _normal(w.shape, 0.0, 1.0, g, device)
+        out["k"] = _normal(w.k_shape, 0.0, 1.0, g, device)
+        out["wq"] = _normal((w.dim,), 1.0, 0.1, g, device)
+        out["wk"] = _normal((w.k_shape[-1],), 1.0, 0.1, g, device)
+    elif w.name == "rms_bf16_16x4096x4096":
+        x = _normal(w.shape, 0.0, 1.0, g, device)
+        out["w"] = _normal((w.dim,), 1.0, 0.1, g, device)
+        outliers = torch.rand(w.shape, generator=g, device=device) < 0.01
+        out["x"] = torch.where(outliers, x * 50.0, x)
+    elif w.name.startswith("ln_bf16_65536x"):
+        x = _normal(w.shape, 0.5, 2.0, g, device)
+        out["w"] = _normal((w.dim,), 1.0, 0.1, g, device)
+        out["b"] = _normal((w.dim,), 0.0, 0.1, g, device)
+        const_rows = torch.arange(0, w.rows, CONSTANT_ROW_PERIOD, device=device)
+        values = _normal((const_rows.numel(), 1), 0.5, 2.0, g, device)
+        x[const_rows] = values.expand(-1, w.dim)
+        out["x"] = x
+    else:
+        raise KeyError(w.name)
+    return {k: v.to(w.dtype) for k, v in out.items()}
+
+
+def random_rows(rows, dim, dtype, seed, device="cpu", mean=0.0, std=1.0):
+    """Generic N(mean, std) rows for edge-case tests, rounded to ``dtype``."""
+    g = _gen(torch.device(device), seed)
+    return _normal((rows, dim), mean, std, g, device).to(dtype)
+
+
+def random_vector(dim, dtype, seed, device="cpu", mean=1.0, std=0.1):
+    g = _gen(torch.device(device), seed)
+    return _normal((dim,), mean, std, g, device).to(dtype)
