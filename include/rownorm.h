@@ -1,0 +1,201 @@
+/*
+ * rownorm.h -- fused last-axis row normalization on NVIDIA B200 (sm_100a).
+ *
+ * C ABI of librownorm.so. Every entry point takes plain pointers and sizes;
+ * no C++ or framework types cross this boundary.
+ *
+ * Operations (what each computes is stated with the function):
+ *   rn_rms_norm            RMSNorm    -- "Emily.Fast", rms_norm/3, and the
+ *                                        composed RMSNorm of "Fused
+ *                                        transformer kernels on Emily",
+ *                                        Part 1.
+ *   rn_layer_norm          LayerNorm  -- "Emily.Fast", layer_norm/4.
+ *   rn_dual_head_rms_norm  query/key head RMSNorm, both outputs from one
+ *                          launch -- "norm_fusion.rs" (mlx_c_rust compile),
+ *                          MlxCompiledDualHeadNorm and
+ *                          apply_compiled_dual_head_norm.
+ *
+ * Common conventions
+ *   Views. A tensor is passed as an rn_view: `rows` rows of `dim` elements,
+ *   the elements of a row contiguous (unit stride), consecutive rows
+ *   `row_stride` elements apart (row_stride >= dim). Any leading dimensions
+ *   of a tensor are folded into `rows`. Normalization always runs over the
+ *   last axis ("Emily.Bumblebee.FastKernels", What's not rewritten: only
+ *   norms over the last axis are fused).
+ *   Element types. RN_F32 (IEEE binary32) or RN_BF16 (bfloat16). Inputs,
+ *   outputs, weights and biases of one call share one element type. All
+ *   arithmetic is binary32 with binary32 accumulation; the result is rounded
+ *   once (round to nearest even) to the output element type.
+ *   eps. A binary32 value >= 0, finite (norm_fusion.rs keeps the epsilon as
+ *   f32 bits). It is added to the mean square (RMSNorm) or the variance
+ *   (LayerNorm) inside the square root.
+ *   Memory. Every pointer is a device pointer on the calling thread's current
+ *   CUDA device (memory from cudaMalloc or a framework allocator). The
+ *   caller owns all memory; the library allocates nothing and keeps no
+ *   per-call state. Base pointers must be aligned to the element size.
+ *   Streams. `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *   Calls are asynchronous: they enqueue one kernel launch and return.
+ *   Aliasing. An output view may be identical to its input view (same data
+ *   pointer and row stride: in place). Any other overlap between an output
+ *   and any input or other output is rejected with RN_ERR_OVERLAP.
+ *   Errors. Every argument is validated on the host before anything is
+ *   enqueued; a rejected call launches nothing and returns a nonzero
+ *   rn_status. There is no fallback to another implementation: inputs the
+ *   kernels do not support are rejected, never silently degraded.
+ *   rows == 0 is valid and enqueues nothing.
+ *   Determinism. The summation order of every row is fixed by (element type,
+ *   dim, and the 16-byte phase of the row's address); repeated calls on the
+ *   same data and addresses return bit-identical results, independently of
+ *   the grid size. rn_dual_head_rms_norm returns exactly the bits of two
+ *   rn_rms_norm calls on the same views.
+ */
+#ifndef ROWNORM_H_
+#define ROWNORM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define RN_API __attribute__((visibility("default")))
+#else
+#define RN_API
+#endif
+
+#define RN_ABI_VERSION 1
+
+/* Largest supported dim. Rows are held on chip (registers) between reading
+ * and writing, so x is read from HBM exactly once; wider rows are rejected
+ * with RN_ERR_UNSUPPORTED. */
+#define RN_MAX_DIM_BF16 32768
+#define RN_MAX_DIM_F32 16384
+/* rn_dual_head_rms_norm: both head dims at most this (one launch keeps the
+ * query and key rows in one warp-level kernel). */
+#define RN_MAX_HEAD_DIM 1024
+
+typedef enum rn_dtype { RN_F32 = 0, RN_BF16 = 1 } rn_dtype;
+
+typedef enum rn_status {
+    RN_OK = 0,
+    RN_ERR_NULL = 1,        /* a required pointer is NULL                     */
+    RN_ERR_SHAPE = 2,       /* rows < 0, dim < 1, row_stride < dim, or views  */
+                            /* of one call disagree in rows/dim               */
+    RN_ERR_DTYPE = 3,       /* unknown element type or mixed element types    */
+    RN_ERR_EPS = 4,         /* eps is negative, NaN or infinite               */
+    RN_ERR_ALIGN = 5,       /* a pointer not aligned to its element size      */
+    RN_ERR_OVERLAP = 6,     /* an output partially overlaps an input/output  */
+    RN_ERR_UNSUPPORTED = 7, /* dim beyond RN_MAX_DIM_*, or a dual head dim    */
+                            /* beyond RN_MAX_HEAD_DIM                         */
+    RN_ERR_CUDA = 8         /* the CUDA runtime reported an error (device    */
+                            /* query or launch); see rn_last_error()          */
+} rn_status;
+
+typedef struct rn_view {
+    void *data;         /* device pointer to element [0, 0]                 */
+    int64_t rows;       /* number of rows, >= 0                              */
+    int64_t dim;        /* elements per row (the normalized axis), >= 1      */
+    int64_t row_stride; /* elements between the starts of consecutive rows  */
+    int32_t dtype;      /* rn_dtype                                          */
+} rn_view;
+
+/*
+ * RMSNorm of every row:  y[r, j] = x[r, j] * rsqrt(mean_i(x[r, i]^2) + eps) * w[j]
+ * ("Emily.Fast", rms_norm/3; composed form x / sqrt(mean(x^2) + eps) * w in
+ * "Fused transformer kernels on Emily", Part 1).
+ *   x       input view.
+ *   weight  device pointer to dim elements of x's type, or NULL (all ones).
+ *   eps     binary32, >= 0 and finite.
+ *   y       output view, same rows, dim and dtype as x (row_stride may
+ *           differ); may be x itself.
+ * Returns RN_OK or an rn_status; nothing is enqueued on error.
+ */
+RN_API int rn_rms_norm(const rn_view *x, const void *weight, float eps,
+                       const rn_view *y, void *stream);
+
+/*
+ * LayerNorm of every row:
+ *   mean = mean_i x[r, i];  var = mean_i (x[r, i] - mean)^2   (population)
+ *   y[r, j] = (x[r, j] - mean) * rsqrt(var + eps) * w[j] + b[j]
+ * ("Emily.Fast", layer_norm/4).
+ *   weight, bias  device pointers to dim elements of x's type, or NULL
+ *                 (weight all ones / bias all zeros).
+ * Other arguments as rn_rms_norm. A row whose elements are all equal returns
+ * exactly the bias (its deviations are exactly zero).
+ */
+RN_API int rn_layer_norm(const rn_view *x, const void *weight, const void *bias,
+                         float eps, const rn_view *y, void *stream);
+
+/*
+ * Dual-output query/key head RMSNorm in ONE kernel launch
+ * ("norm_fusion.rs", MlxCompiledDualHeadNorm / apply_compiled_dual_head_norm):
+ *   yq = rms_norm(q, wq, eps),  yk = rms_norm(k, wk, eps)
+ * Queries first, keys second; one eps shared by both. q [T*Hq, Dq] and
+ * k [T*Hk, Dk] are the head rows (leading dims folded into rows); Dq and Dk
+ * may differ and must each be <= RN_MAX_HEAD_DIM. q and k share one dtype.
+ *   wq, wk  device pointers to Dq / Dk elements; both REQUIRED (non-NULL).
+ *   yq, yk  outputs shaped like q and k; each may be its own input.
+ * The bits of yq and yk equal those of rn_rms_norm(q, wq, eps, yq) and
+ * rn_rms_norm(k, wk, eps, yk).
+ */
+RN_API int rn_dual_head_rms_norm(const rn_view *q, const rn_view *k,
+                                 const void *wq, const void *wk, float eps,
+                                 const rn_view *yq, const rn_view *yk,
+                                 void *stream);
+
+/* Static text for an rn_status value ("unknown status" otherwise). */
+RN_API const char *rn_status_string(int status);
+
+/* Detail of the most recent failed call on the calling thread (which
+ * argument, which CUDA error). Valid until the thread's next call. */
+RN_API const char *rn_last_error(void);
+
+/* RN_ABI_VERSION of the loaded library. */
+RN_API int rn_abi_version(void);
+
+/* ---------------------------------------------------------------------------
+ * Launch introspection and testing controls.
+ */
+
+typedef struct rn_launch_info {
+    int32_t family;         /* 0: a group of lanes of one warp per row;    */
+                            /* 1: one thread block (CTA) per row           */
+    int32_t threads_per_row;/* lanes sharing one row                        */
+    int32_t chunks_per_thread; /* 16-byte chunks of a row each thread holds */
+    int32_t smem_bytes;     /* dynamic shared memory per block (weight and  */
+                            /* bias columns of each thread's chunks)        */
+    int32_t block_threads;  /* threads per block                            */
+    int32_t grid_blocks;    /* blocks launched (persistent: <= SMs x blocks */
+                            /* resident per SM)                             */
+    int32_t blocks_per_sm;  /* resident blocks per SM for this kernel       */
+    int32_t vector_y;       /* 1: y rows share x's 16-byte phase (16-byte   */
+                            /* stores); 0: y written element by element     */
+    int32_t phase_period;   /* distinct 16-byte phases among x's rows       */
+    int32_t exact;          /* 1: every row of x and y starts 16-byte       */
+                            /* aligned and dim fills whole 16-byte chunks   */
+} rn_launch_info;
+
+enum { RN_OP_RMS = 0, RN_OP_LN = 1, RN_OP_DUAL = 2 };
+
+/*
+ * The launch the library would make for op (RN_OP_*) on these arguments,
+ * without launching. For RN_OP_DUAL, x/y are q/yq and x2/y2 are k/yk (the
+ * weight and bias arguments are wq and wk); otherwise x2/y2 are ignored.
+ * Queries the current device (SM count, occupancy), so it needs a GPU.
+ */
+RN_API int rn_plan(int op, const rn_view *x, const rn_view *y,
+                   const rn_view *x2, const rn_view *y2, const void *weight,
+                   const void *bias, rn_launch_info *info);
+
+/* Testing control: launch exactly `blocks` blocks (> 0) instead of the
+ * automatic persistent grid; 0 restores the automatic choice. Results do not
+ * depend on it (rows are statically strided over blocks). Process-wide. */
+RN_API int rn_set_grid_override(int blocks);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ROWNORM_H_ */

@@ -1,0 +1,197 @@
+"""The C-ABI library on the host (CPU only): it loads, exports every entry
+point the header declares, and validates arguments before any CUDA call.
+Only invalid calls and rows == 0 calls are made here; they return before the
+library touches the CUDA runtime, so no GPU is needed."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import transformer_row_normalization_b200 as rn
+from transformer_row_normalization_b200 import rn_view
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rownorm.h")
+
+FAKE = 0x7F0000000000  # a 256-byte-aligned address; never dereferenced
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from transformer_row_normalization_b200 import build_lib
+    build_lib.build()
+    return rn.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"RN_API\s+[\w\s\*]+?\b(rn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("rn_rms_norm", "rn_layer_norm", "rn_dual_head_rms_norm", "rn_status_string",
+              "rn_last_error", "rn_abi_version", "rn_plan", "rn_set_grid_override"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in rownorm.h but not exported"
+
+
+def test_only_declared_symbols_are_exported(lib):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", rn.library_path()],
+                         capture_output=True, text=True, check=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    exported = {e for e in exported if not e.startswith("_")}
+    assert exported == set(declared_functions())
+
+
+def test_status_strings_and_version(lib):
+    assert lib.rn_abi_version() == 1
+    assert lib.rn_status_string(0) == b"ok"
+    for st in range(1, 9):
+        assert lib.rn_status_string(st) not in (b"ok", b"unknown status")
+    assert lib.rn_status_string(99) == b"unknown status"
+
+
+def V(data=FAKE, rows=4, dim=64, stride=None, dtype=1):
+    return rn_view(data, rows, dim, dim if stride is None else stride, dtype)
+
+
+def rms(lib, x, y, w=None, eps=1e-6):
+    return lib.rn_rms_norm(ctypes.byref(x) if x is not None else None, w, eps,
+                           ctypes.byref(y) if y is not None else None, None)
+
+
+def ln(lib, x, y, w=None, b=None, eps=1e-5):
+    return lib.rn_layer_norm(ctypes.byref(x), w, b, eps, ctypes.byref(y), None)
+
+
+def test_rejects_null_views_and_data(lib):
+    assert rms(lib, None, V()) == 1
+    assert rms(lib, V(), None) == 1
+    assert rms(lib, V(data=None), V(data=FAKE + 4096)) == 1
+    assert b"data is NULL" in lib.rn_last_error()
+
+
+def test_rejects_bad_shapes(lib):
+    y = V(data=FAKE + (1 << 20))
+    assert rms(lib, V(rows=-1), y) == 2
+    assert rms(lib, V(dim=0), V(data=FAKE + (1 << 20), dim=0)) == 2
+    assert rms(lib, V(stride=63), y) == 2
+    assert rms(lib, V(rows=4), V(data=FAKE + (1 << 20), rows=5)) == 2
+    assert rms(lib, V(dim=64), V(data=FAKE + (1 << 20), dim=65)) == 2
+    assert rms(lib, V(rows=1 << 40, stride=1 << 40), V(data=FAKE + (1 << 20))) == 2
+
+
+def test_rejects_bad_dtypes(lib):
+    assert rms(lib, V(dtype=7), V(data=FAKE + 4096, dtype=7)) == 3
+    assert rms(lib, V(dtype=0), V(data=FAKE + 4096, dtype=1)) == 3
+
+
+def test_rejects_bad_eps(lib):
+    y = V(data=FAKE + 4096)
+    for eps in (float("nan"), -1e-6, float("inf")):
+        assert rms(lib, V(), y, eps=eps) == 4
+        assert ln(lib, V(), y, eps=eps) == 4
+    assert rms(lib, V(), V(data=FAKE + 4096, rows=0), eps=0.0) == 2  # rows differ
+    assert rms(lib, V(rows=0), V(data=FAKE + 4096, rows=0), eps=0.0) == 0
+
+
+def test_rejects_misalignment(lib):
+    assert rms(lib, V(data=FAKE + 1), V(data=FAKE + 4096)) == 5
+    assert rms(lib, V(dtype=0, data=FAKE + 2), V(dtype=0, data=FAKE + 4096)) == 5
+    assert rms(lib, V(), V(data=FAKE + 4096), w=ctypes.c_void_p(FAKE + 8191)) == 5
+    assert ln(lib, V(), V(data=FAKE + 4096), b=ctypes.c_void_p(FAKE + 8193)) == 5
+
+
+def test_rejects_overlap_but_allows_in_place(lib):
+    x = V(rows=0)  # rows == 0: an exact alias is OK and enqueues nothing
+    assert rms(lib, x, V(rows=0)) == 0
+    # partial overlap: y starts inside x
+    assert rms(lib, V(), V(data=FAKE + 64)) == 6
+    # same data, different stride: overlapping, not identical
+    assert rms(lib, V(stride=128), V(stride=64)) == 6
+    # output over the weight
+    assert rms(lib, V(), V(data=FAKE + 4096), w=ctypes.c_void_p(FAKE + 4096 + 64)) == 6
+    assert ln(lib, V(), V(data=FAKE + 4096), b=ctypes.c_void_p(FAKE + 4096 + 64)) == 6
+
+
+def test_rejects_unsupported_widths(lib):
+    y = V(data=FAKE + (1 << 30), dim=32769)
+    assert rms(lib, V(dim=32769), y) == 7
+    y = V(data=FAKE + (1 << 30), dim=16385, dtype=0)
+    assert rms(lib, V(dim=16385, dtype=0), y) == 7
+
+
+def test_rows_zero_is_a_no_op(lib):
+    assert rms(lib, V(rows=0), V(data=FAKE + 4096, rows=0)) == 0
+    assert ln(lib, V(rows=0), V(data=FAKE + 4096, rows=0)) == 0
+
+
+def dual(lib, q, k, yq, yk, wq=FAKE + (3 << 20), wk=FAKE + (3 << 20) + 4096, eps=1e-6):
+    return lib.rn_dual_head_rms_norm(ctypes.byref(q), ctypes.byref(k),
+                                     None if wq is None else ctypes.c_void_p(wq),
+                                     None if wk is None else ctypes.c_void_p(wk), eps,
+                                     ctypes.byref(yq), ctypes.byref(yk), None)
+
+
+def test_dual_validation(lib):
+    M = 1 << 20
+    q, k = V(rows=0, dim=128), V(data=FAKE + M, rows=0, dim=128)
+    yq, yk = V(data=FAKE + 2 * M, rows=0, dim=128), V(data=FAKE + 2 * M + 8192, rows=0, dim=128)
+    assert dual(lib, q, k, yq, yk) == 0
+    assert dual(lib, q, k, yq, yk, wq=None) == 1
+    assert dual(lib, q, k, yq, yk, wk=None) == 1
+    assert dual(lib, q, V(data=FAKE + M, rows=0, dim=128, dtype=0), yq,
+                V(data=FAKE + 2 * M + 8192, rows=0, dim=128, dtype=0)) == 3
+    big = V(rows=0, dim=2048)
+    assert dual(lib, big, k, V(data=FAKE + 2 * M, rows=0, dim=2048), yk) == 7
+    # yq over k, yk over q
+    q4, k4 = V(rows=4, dim=128), V(data=FAKE + M, rows=4, dim=128)
+    assert dual(lib, q4, k4, V(data=FAKE + M, rows=4, dim=128),
+                V(data=FAKE + 2 * M, rows=4, dim=128)) == 6
+    assert dual(lib, q4, k4, V(data=FAKE + 2 * M, rows=4, dim=128),
+                V(data=FAKE, rows=4, dim=128)) == 6
+    # yq and yk over each other
+    assert dual(lib, q4, k4, V(data=FAKE + 2 * M, rows=4, dim=128),
+                V(data=FAKE + 2 * M + 256, rows=4, dim=128)) == 6
+    assert dual(lib, q, k, yq, yk, eps=float("nan")) == 4
+
+
+def test_grid_override_control(lib):
+    assert lib.rn_set_grid_override(-1) == 2
+    assert lib.rn_set_grid_override(0) == 0
+
+
+@pytest.mark.parametrize("shape,strides,want", [
+    ((4, 128, 1024), (128 * 1024, 1024, 1), (512, 1024, 1024)),
+    ((1024,), (1,), (1, 1024, 1024)),
+    ((8, 7), (10, 1), (8, 7, 10)),
+    ((2, 1, 3, 5), (30, 99, 10, 1), (6, 5, 10)),
+    ((1, 1, 9), (9, 9, 1), (1, 9, 9)),
+    ((0, 16), (16, 1), (0, 16, 16)),
+])
+def test_view_params_folds_leading_axes(shape, strides, want):
+    assert rn.view_params(shape, strides) == want
+
+
+@pytest.mark.parametrize("shape,strides", [
+    ((4, 8), (8, 2)),          # last axis not contiguous
+    ((2, 3, 8), (40, 8, 1)),   # leading axes do not fold (40 != 3 * 8)
+    ((4, 8), (4, 1)),          # rows overlap
+])
+def test_view_params_rejects(shape, strides):
+    with pytest.raises(ValueError):
+        rn.view_params(shape, strides)
+
+
+def test_cpu_tensors_are_rejected_loudly():
+    import torch
+    x = torch.zeros(2, 8)
+    with pytest.raises(TypeError, match="CUDA"):
+        rn.rms_norm(x, None, 1e-6)

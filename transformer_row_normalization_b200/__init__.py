@@ -1,0 +1,232 @@
+"""Fused last-axis row normalization on NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``librownorm.so`` (declared in
+``include/rownorm.h``). This module only marshals arguments: it turns torch
+CUDA tensors into ``rn_view`` descriptors (data pointer, rows, dim, row
+stride, dtype), passes the current CUDA stream, and raises on a nonzero
+status. Every step of the computation runs in the library's CUDA kernels;
+there is no CPU or framework fallback, and calling with CPU tensors or
+without the built library raises.
+
+    rn_rms_norm(x, weight, eps, out=None)               RMSNorm
+    rn_layer_norm(x, weight, bias, eps, out=None)       LayerNorm
+    rn_dual_head_rms_norm(q, k, wq, wk, eps, ...)       q/k head RMSNorm, one launch
+
+``rms_norm``, ``layer_norm`` and ``dual_head_rms_norm`` are the same calls.
+"""
+import ctypes
+import os
+
+__all__ = [
+    "RowNormError", "rn_rms_norm", "rn_layer_norm", "rn_dual_head_rms_norm",
+    "rms_norm", "layer_norm", "dual_head_rms_norm", "plan", "set_grid_override",
+    "library_path", "load_library", "view_params",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librownorm.so")
+
+RN_F32, RN_BF16 = 0, 1
+RN_OP_RMS, RN_OP_LN, RN_OP_DUAL = 0, 1, 2
+STATUS_NAMES = {0: "RN_OK", 1: "RN_ERR_NULL", 2: "RN_ERR_SHAPE", 3: "RN_ERR_DTYPE",
+                4: "RN_ERR_EPS", 5: "RN_ERR_ALIGN", 6: "RN_ERR_OVERLAP",
+                7: "RN_ERR_UNSUPPORTED", 8: "RN_ERR_CUDA"}
+
+
+class RowNormError(RuntimeError):
+    def __init__(self, status, detail):
+        self.status = status
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {detail}")
+
+
+class rn_view(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("rows", ctypes.c_int64),
+                ("dim", ctypes.c_int64), ("row_stride", ctypes.c_int64),
+                ("dtype", ctypes.c_int32)]
+
+
+class rn_launch_info(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "family", "threads_per_row", "chunks_per_thread", "smem_bytes", "block_threads",
+        "grid_blocks", "blocks_per_sm", "vector_y", "phase_period", "exact")]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return LIB_PATH
+
+
+def load_library():
+    """Load librownorm.so (once). Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is not built; build it with "
+                "`python -m transformer_row_normalization_b200.build_lib`")
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, f32 = ctypes.c_void_p, ctypes.c_float
+        pv = ctypes.POINTER(rn_view)
+        lib.rn_rms_norm.argtypes = [pv, vp, f32, pv, vp]
+        lib.rn_layer_norm.argtypes = [pv, vp, vp, f32, pv, vp]
+        lib.rn_dual_head_rms_norm.argtypes = [pv, pv, vp, vp, f32, pv, pv, vp]
+        lib.rn_plan.argtypes = [ctypes.c_int, pv, pv, pv, pv, vp, vp,
+                                ctypes.POINTER(rn_launch_info)]
+        lib.rn_set_grid_override.argtypes = [ctypes.c_int]
+        lib.rn_status_string.argtypes = [ctypes.c_int]
+        lib.rn_status_string.restype = ctypes.c_char_p
+        lib.rn_last_error.argtypes = []
+        lib.rn_last_error.restype = ctypes.c_char_p
+        for fn in (lib.rn_rms_norm, lib.rn_layer_norm, lib.rn_dual_head_rms_norm,
+                   lib.rn_plan, lib.rn_set_grid_override, lib.rn_abi_version):
+            fn.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _check(status):
+    if status != 0:
+        lib = load_library()
+        raise RowNormError(status, lib.rn_last_error().decode())
+
+
+def view_params(shape, strides):
+    """(rows, dim, row_stride) of a [..., dim] layout whose last axis is
+    contiguous and whose leading axes fold into one row axis; raises
+    ValueError otherwise. Pure shape arithmetic (no copies)."""
+    shape, strides = tuple(shape), tuple(strides)
+    if len(shape) == 0:
+        raise ValueError("a row view needs at least one dimension")
+    dim = shape[-1]
+    if dim > 1 and strides[-1] != 1:
+        raise ValueError("the last axis must be contiguous (stride 1)")
+    rows = 1
+    for s in shape[:-1]:
+        rows *= s
+    if len(shape) == 1:
+        return rows, dim, dim
+    lead = [(n, st) for n, st in zip(shape[:-1], strides[:-1]) if n != 1]
+    if not lead:
+        return rows, dim, dim
+    row_stride = lead[-1][1]
+    expect = row_stride
+    for n, st in reversed(lead):
+        if st != expect:
+            raise ValueError("leading axes do not fold into one row axis")
+        expect = st * n
+    if rows > 1 and row_stride < dim:
+        raise ValueError("rows overlap (row stride < dim)")
+    return rows, dim, row_stride
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.float32:
+        return RN_F32
+    if t.dtype == torch.bfloat16:
+        return RN_BF16
+    raise TypeError(f"row normalization supports float32 and bfloat16, not {t.dtype}")
+
+
+def _require_cuda(*tensors):
+    for t in tensors:
+        if t is not None and not t.is_cuda:
+            raise TypeError("tensors must live on a CUDA device: this library has no CPU path")
+
+
+def _view(t):
+    rows, dim, row_stride = view_params(t.shape, t.stride())
+    return rn_view(t.data_ptr() if t.numel() else None, rows, dim, row_stride, _dtype_code(t))
+
+
+def _vector(v, dim, like):
+    if v is None:
+        return None
+    if v.dim() != 1 or v.shape[0] != dim or v.stride(0) != 1:
+        raise ValueError(f"weight/bias must be a contiguous vector of length {dim}")
+    if v.dtype != like.dtype or v.device != like.device:
+        raise TypeError("weight/bias must match the input's dtype and device")
+    return ctypes.c_void_p(v.data_ptr())
+
+
+def _stream(t, stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream(t.device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def rn_rms_norm(x, weight, eps=1e-6, out=None, stream=None):
+    """RMSNorm over the last axis of the CUDA tensor ``x``; returns ``out``."""
+    import torch
+    _require_cuda(x, weight, out)
+    out = torch.empty_like(x) if out is None else out
+    xv, yv = _view(x), _view(out)
+    lib = load_library()
+    with torch.cuda.device(x.device):
+        _check(lib.rn_rms_norm(ctypes.byref(xv), _vector(weight, xv.dim, x), float(eps),
+                               ctypes.byref(yv), _stream(x, stream)))
+    return out
+
+
+def rn_layer_norm(x, weight, bias, eps=1e-5, out=None, stream=None):
+    """LayerNorm over the last axis of the CUDA tensor ``x``; returns ``out``."""
+    import torch
+    _require_cuda(x, weight, bias, out)
+    out = torch.empty_like(x) if out is None else out
+    xv, yv = _view(x), _view(out)
+    lib = load_library()
+    with torch.cuda.device(x.device):
+        _check(lib.rn_layer_norm(ctypes.byref(xv), _vector(weight, xv.dim, x),
+                                 _vector(bias, xv.dim, x), float(eps), ctypes.byref(yv),
+                                 _stream(x, stream)))
+    return out
+
+
+def rn_dual_head_rms_norm(q, k, wq, wk, eps=1e-6, out_q=None, out_k=None, stream=None):
+    """(RMSNorm(q, wq), RMSNorm(k, wk)) from one kernel launch; queries first."""
+    import torch
+    _require_cuda(q, k, wq, wk, out_q, out_k)
+    out_q = torch.empty_like(q) if out_q is None else out_q
+    out_k = torch.empty_like(k) if out_k is None else out_k
+    qv, kv, yqv, ykv = _view(q), _view(k), _view(out_q), _view(out_k)
+    if wq is None or wk is None:
+        raise ValueError("dual head norm needs both wq and wk")
+    lib = load_library()
+    with torch.cuda.device(q.device):
+        _check(lib.rn_dual_head_rms_norm(
+            ctypes.byref(qv), ctypes.byref(kv), _vector(wq, qv.dim, q), _vector(wk, kv.dim, k),
+            float(eps), ctypes.byref(yqv), ctypes.byref(ykv), _stream(q, stream)))
+    return out_q, out_k
+
+
+rms_norm = rn_rms_norm
+layer_norm = rn_layer_norm
+dual_head_rms_norm = rn_dual_head_rms_norm
+
+
+def plan(op, x, out=None, weight=None, bias=None, k=None, out_k=None):
+    """The launch configuration the library picks (see rn_launch_info)."""
+    import torch
+    out = torch.empty_like(x) if out is None else out
+    xv, yv = _view(x), _view(out)
+    info = rn_launch_info()
+    lib = load_library()
+    with torch.cuda.device(x.device):
+        if op == RN_OP_DUAL:
+            out_k = torch.empty_like(k) if out_k is None else out_k
+            kv, ykv = _view(k), _view(out_k)
+            _check(lib.rn_plan(op, ctypes.byref(xv), ctypes.byref(yv), ctypes.byref(kv),
+                               ctypes.byref(ykv), _vector(weight, xv.dim, x),
+                               _vector(bias, kv.dim, k), ctypes.byref(info)))
+        else:
+            _check(lib.rn_plan(op, ctypes.byref(xv), ctypes.byref(yv), None, None,
+                               _vector(weight, xv.dim, x), _vector(bias, xv.dim, x),
+                               ctypes.byref(info)))
+    return {n: getattr(info, n) for n, _ in rn_launch_info._fields_}
+
+
+def set_grid_override(blocks: int):
+    """Testing control: launch exactly ``blocks`` blocks (0 = automatic)."""
+    _check(load_library().rn_set_grid_override(int(blocks)))
