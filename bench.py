@@ -1,0 +1,525 @@
+"""Benchmark: fused row normalization on B200, one JSON line on stdout.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the whole hot path over the large bf16 workloads:
+  dual q/k head RMSNorm   q [8192, 32, 128] + k [8192, 8, 128]  (one launch)
+  RMSNorm                 [16, 4096, 4096]
+  LayerNorm               [65536, D] for D in 768, 1000, 4097, 8192, 16384
+i.e. 7 launches, 720,896 normalized rows and ~9.2 GB of algorithmic HBM
+traffic per step. Inputs live in HBM before timing starts (seeded, drawn on
+the device). Every step reads ~4.6 GB, far more than the 126 MB L2, so no
+L2 flush is needed between steps. The device time of K steps is taken with
+CUDA events on the launching stream, bracketed by a barrier and a
+synchronize, and the maximum over ranks is reported.
+
+Multi-GPU (torchrun): each rank normalizes its own copy of the workload (weak
+scaling; rows are independent, so there is no data-path collective); the
+only collective is the max-over-ranks of the timings.
+
+--impl reference runs the fp64 CPU oracle on the host cores instead, on a
+bounded sample of the same workloads per step (rank 0 only).
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from transformer_row_normalization_b200 import workloads as wl  # noqa: E402
+
+METRIC = "normalized rows/sec and achieved HBM GB/s as % of B200 peak, 1 GPU"
+FALLBACK_HBM_GBS = 6650.0
+CSRC = os.path.join(ROOT, "transformer_row_normalization_b200", "csrc")
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (host logic; covered by tests on gloo)
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def max_over_ranks(value, dist, device):
+    """The maximum of a float over all ranks (the value itself at N=1)."""
+    if dist is None:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device):
+    if dist is not None:
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def rank_seed(seed, rank):
+    """Each rank draws its own inputs (same recipe, different seed)."""
+    return seed + 1000 * rank
+
+
+# ---------------------------------------------------------------------------
+# measured peaks, clocks, profile bookkeeping
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest():
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(CSRC, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name):
+    """DRAM bytes per launch from an ncu capture recorded in
+    profiles/ncu_traffic.json, if that capture was taken of the current
+    kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = d.get(workload_name)
+    if not e or e.get("source_digest") != source_digest():
+        return None
+    return e.get("traffic_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed
+    region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.target = None
+        try:
+            p = torch.cuda.get_device_properties(device)
+            self.target = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+        except Exception:
+            self.target = str(device.index or 0)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", self.target],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        return self.parse(out)
+
+    @staticmethod
+    def parse(text):
+        """Median SM clock, max clock, peak power and the throttle reasons
+        seen in nvidia-smi CSV samples of FIELDS."""
+        rows = [[c.strip() for c in l.split(",")] for l in text.strip().splitlines()
+                if l.count(",") >= 7]
+        rows = [r for r in rows if r[0].replace(".", "", 1).isdigit()]
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[4:8]) if v == "Active"})
+        power = [float(r[2]) for r in rows if r[2].replace(".", "", 1).isdigit()]
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][1]),
+                "power_w_max": max(power) if power else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# the step
+
+
+class Step:
+    """The large bf16 workloads on one device, with outputs preallocated."""
+
+    def __init__(self, device, rank):
+        import transformer_row_normalization_b200 as rn
+        self.rn = rn
+        self.device = device
+        self.items = []
+        for name in wl.LARGE_SUITE:
+            w = wl.WORKLOADS[name]
+            rw = wl.Workload(w.name, w.op, w.dtype, w.shape, w.eps, rank_seed(w.seed, rank),
+                             k_shape=w.k_shape)
+            a = wl.make_inputs(rw, device=device)
+            if w.op == "dual":
+                out = (torch.empty_like(a["q"]), torch.empty_like(a["k"]))
+            else:
+                out = (torch.empty_like(a["x"]),)
+            self.items.append((w, a, out))
+        torch.cuda.synchronize(device)
+
+    @property
+    def rows(self):
+        return sum(w.total_rows for w, _, _ in self.items)
+
+    @property
+    def bytes(self):
+        return sum(w.algorithmic_bytes() for w, _, _ in self.items)
+
+    def launch(self, i, stream=None):
+        w, a, out = self.items[i]
+        rn = self.rn
+        if w.op == "dual":
+            rn.dual_head_rms_norm(a["q"], a["k"], a["wq"], a["wk"], w.eps, out_q=out[0],
+                                  out_k=out[1], stream=stream)
+        elif w.op == "rms":
+            rn.rms_norm(a["x"], a["w"], w.eps, out=out[0], stream=stream)
+        else:
+            rn.layer_norm(a["x"], a["w"], a["b"], w.eps, out=out[0], stream=stream)
+
+    def run(self, stream=None):
+        for i in range(len(self.items)):
+            self.launch(i, stream)
+
+
+def time_steps(step, k, stream):
+    """Device time of k steps (ms) and per-launch times (ms, per workload,
+    averaged), all from CUDA events on `stream`."""
+    n = len(step.items)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(k)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for s in range(k):
+            ev[s][0].record(stream)
+            for i in range(n):
+                step.launch(i, stream)
+                ev[s][i + 1].record(stream)
+        end.record(stream)
+    end.synchronize()
+    total = start.elapsed_time(end)
+    per = [sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(k)) / k for i in range(n)]
+    return total, per
+
+
+def time_e2e(step, k, stream):
+    """Through the public API with HOST buffers: every step copies each
+    workload's inputs from pinned host memory to the device, normalizes, and
+    copies the outputs back to pinned host memory."""
+    host_in, host_out = [], []
+    h2d = d2h = 0
+    for w, a, out in step.items:
+        hi = {key: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for key, t in a.items()}
+        for key, t in a.items():
+            hi[key].copy_(t)
+        ho = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in out]
+        host_in.append(hi)
+        host_out.append(ho)
+        h2d += sum(t.numel() * t.element_size() for t in a.values())
+        d2h += sum(t.numel() * t.element_size() for t in out)
+    torch.cuda.synchronize(step.device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(k):
+            for i, (w, a, out) in enumerate(step.items):
+                for key, t in a.items():
+                    t.copy_(host_in[i][key], non_blocking=True)
+                step.launch(i, stream)
+                for dst, src in zip(host_out[i], out):
+                    dst.copy_(src, non_blocking=True)
+        end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end), h2d, d2h
+
+
+def cpu_baseline(step, chunk_rows=2048):
+    """The fp64 oracle on the host cores over every row of one step (copied
+    from the device in chunks of `chunk_rows` rows; only the oracle calls are
+    timed)."""
+    import oracle
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    # warm-up (page faults, thread pool) on a few rows
+    w0, a0, _ = step.items[1]
+    oracle.rms_norm(a0["x"].reshape(-1, w0.dim)[:64].cpu(), a0["w"].cpu(), w0.eps, nthreads=cores)
+    busy = 0.0
+    rows = 0
+    for w, a, _ in step.items:
+        if w.op == "dual":
+            parts = [(a["q"].reshape(-1, w.dim), a["wq"]), (a["k"].reshape(-1, w.k_shape[-1]), a["wk"])]
+            bias = None
+        else:
+            parts = [(a["x"].reshape(-1, w.dim), a["w"])]
+            bias = a["b"].cpu() if "b" in a else None
+        for x, wt in parts:
+            wt = wt.cpu()
+            for r0 in range(0, x.shape[0], chunk_rows):
+                xc = x[r0:r0 + chunk_rows].cpu()
+                t0 = time.perf_counter()
+                if w.op == "ln":
+                    oracle.layer_norm(xc, wt, bias, w.eps, nthreads=cores)
+                else:
+                    oracle.rms_norm(xc, wt, w.eps, nthreads=cores)
+                busy += time.perf_counter() - t0
+                rows += xc.shape[0]
+    return {"value": round(rows / busy, 1), "unit": "rows/s", "cores": cores, "kind": "oracle",
+            "sample": f"one full step ({rows} rows, every workload), fp64, {cores} threads, "
+                      f"{busy:.1f} s of oracle time"}
+
+
+# ---------------------------------------------------------------------------
+
+
+def config_dict(rows, nbytes, world):
+    return {
+        "workload": "large bf16 suite: dual q/k head RMSNorm q[8192,32,128]+k[8192,8,128] "
+                    "(1 launch); RMSNorm [16,4096,4096] with 1% x50 outliers; LayerNorm "
+                    "[65536,D] D in {768,1000,4097,8192,16384} with constant rows",
+        "rows_per_step": rows,
+        "algorithmic_bytes_per_step": nbytes,
+        "launches_per_step": 7,
+        "l2": "no flush: each step reads ~4.6 GB and writes ~4.6 GB (126 MB L2)",
+        "parallelism": f"dp{world} (weak: each rank its own copy of the suite)",
+    }
+
+
+def run_ours(args):
+    world, rank, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = init_dist(world, "nccl")
+    peak, peak_kind = measured_peak()
+    step = Step(device, rank)
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step.run(stream)
+    stream.synchronize()
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    clocks = ClockSampler(device) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.2)
+    total_ms, per_ms = time_steps(step, args.steps, stream)
+    torch.cuda.synchronize(device)
+    clk = clocks.stop() if clocks else None
+    barrier(dist, device)
+    total_ms = max_over_ranks(total_ms, dist, device)
+    per_ms = [max_over_ranks(t, dist, device) for t in per_ms]
+
+    rows = step.rows
+    nbytes = step.bytes
+    seconds = total_ms / 1e3
+    value = world * rows * args.steps / seconds
+    gbs = nbytes * args.steps / seconds / 1e9
+
+    per_config = []
+    for (w, _, _), t in zip(step.items, per_ms):
+        g = w.algorithmic_bytes() / (t * 1e-3) / 1e9
+        per_config.append({"workload": w.name, "us": round(t * 1e3, 2),
+                           "rows_per_s": round(w.total_rows / (t * 1e-3)),
+                           "gbs": round(g, 1), "frac": round(g / peak, 4)})
+    dom = max(range(len(per_ms)), key=lambda i: per_ms[i])
+    dw = step.items[dom][0]
+    achieved = dw.algorithmic_bytes() / (per_ms[dom] * 1e-3) / 1e9
+    traffic = recorded_traffic(dw.name)
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "kernel_workload": dw.name, "peak_source": peak_kind,
+                "algorithmic_bytes_per_launch": dw.algorithmic_bytes()}
+
+    e2e_steps = max(1, min(3, args.steps))
+    e2e_ms, h2d, d2h = time_e2e(step, e2e_steps, stream)
+    e2e_ms = max_over_ranks(e2e_ms, dist, device)
+    e2e = {"value": world * rows * e2e_steps / (e2e_ms / 1e3), "unit": "rows/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+
+    base = cpu_baseline(step) if (rank == 0 and world == 1) else None
+    if dist is not None:
+        barrier(dist, device)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "rows/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded on the device with the workloads' shapes and distributions",
+            "config": config_dict(rows, nbytes, world),
+            "hbm": {"gbs": round(gbs, 1), "peak_gbs": peak, "frac": round(gbs / peak, 4),
+                    "peak_source": peak_kind},
+            "roofline": roofline, "cpu_baseline": base, "e2e": e2e,
+            "gpu_launches": 7 * args.steps, "clocks": clk, "per_config": per_config,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The fp64 oracle on the host cores, each step a bounded sample of the
+    workloads (rows_per_workload rows of each)."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    samples = []
+    per_wl = max(4, min(64, 6000 // max(1, args.steps + args.warmup)))
+    for name in wl.LARGE_SUITE:
+        w = wl.WORKLOADS[name]
+        if w.op == "dual":
+            sw = wl.Workload(w.name, w.op, w.dtype, (per_wl, 32, 128), w.eps, w.seed,
+                             k_shape=(per_wl, 8, 128))
+        else:
+            sw = wl.Workload(w.name, w.op, w.dtype, (per_wl * 4, w.dim), w.eps, w.seed)
+        samples.append((sw, wl.make_inputs(sw)))
+
+    def one_step():
+        n = 0
+        for sw, a in samples:
+            if sw.op == "dual":
+                oracle.dual_head_rms_norm(a["q"].reshape(-1, 128), a["k"].reshape(-1, 128),
+                                          a["wq"], a["wk"], sw.eps, nthreads=cores)
+            elif sw.op == "rms":
+                oracle.rms_norm(a["x"], a["w"], sw.eps, nthreads=cores)
+            else:
+                oracle.layer_norm(a["x"], a["w"], a["b"], sw.eps, nthreads=cores)
+            n += sw.total_rows
+        return n
+
+    for _ in range(args.warmup):
+        one_step()
+    t0 = time.perf_counter()
+    rows = 0
+    for _ in range(args.steps):
+        rows += one_step()
+    dt = time.perf_counter() - t0
+    value = rows / dt
+    sample = (f"per step {rows // args.steps} rows: {per_wl * 40} dual head rows and "
+              f"{per_wl * 4} rows of each other workload, fp64, {cores} threads")
+    full_rows = sum(wl.WORKLOADS[n].total_rows for n in wl.LARGE_SUITE)
+    full_bytes = sum(wl.WORKLOADS[n].algorithmic_bytes() for n in wl.LARGE_SUITE)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "rows/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic: seeded on the host with the workloads' shapes and distributions",
+        "config": config_dict(full_rows, full_bytes, world),
+        "cpu_baseline": {"value": round(value, 1), "unit": "rows/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 1), "unit": "rows/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_profile_case(args):
+    """One workload, launched --steps times after --warmup launches, for
+    profiler captures: OP:DTYPE:ROWS:DIM, e.g. ln:bf16:8192:16384. Prints the
+    median CUDA-event time per launch (each launch after a 256 MB read that
+    evicts L2) on stderr; this is not the benchmark line."""
+    import transformer_row_normalization_b200 as rn
+    op, dt, rows, dim = args.profile_case.split(":")
+    dtype = torch.bfloat16 if dt == "bf16" else torch.float32
+    rows, dim = int(rows), int(dim)
+    device = torch.device("cuda", 0)
+    x = wl.random_rows(rows, dim, dtype, seed=1, device=device, mean=0.5, std=2.0)
+    w = wl.random_vector(dim, dtype, seed=2, device=device)
+    b = wl.random_vector(dim, dtype, seed=3, device=device, mean=0.0, std=0.1)
+    y = torch.empty_like(x)
+    rn.set_path_override(args.path)
+    evict = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=device)
+    times = []
+    for i in range(args.warmup + args.steps):
+        evict.sum()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        if op == "rms":
+            rn.rms_norm(x, w, 1e-5, out=y)
+        else:
+            rn.layer_norm(x, w, b, 1e-5, out=y)
+        e.record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(s.elapsed_time(e) * 1e3)
+    plan = rn.plan(rn.RN_OP_LN if op == "ln" else rn.RN_OP_RMS, x, weight=w,
+                   bias=b if op == "ln" else None)
+    log(f"{args.profile_case} path={args.path} median {sorted(times)[len(times) // 2]:.1f} us "
+        f"plan={plan} timeouts={rn.device_error_count()}")
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--profile-case", default=None,
+                    help="OP:DTYPE:ROWS:DIM -- launch one workload for a profiler capture")
+    ap.add_argument("--path", type=int, default=0,
+                    help="with --profile-case: 0 automatic, 1 register, 2 staged kernels")
+    args = ap.parse_args(argv)
+    if args.profile_case:
+        return run_profile_case(args)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world, _, _ = dist_env()
+    if world != args.gpus and world > 1:
+        log(f"note: WORLD_SIZE={world} but --gpus {args.gpus}")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

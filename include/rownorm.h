@@ -175,6 +175,10 @@ typedef struct rn_launch_info {
     int32_t phase_period;   /* distinct 16-byte phases among x's rows       */
     int32_t exact;          /* 1: every row of x and y starts 16-byte       */
                             /* aligned and dim fills whole 16-byte chunks   */
+    int32_t staged;         /* 1: rows stream through shared memory by bulk */
+                            /* copies (S stages); 0: loaded into registers  */
+    int32_t stages;         /* staged: stages per block                     */
+    int32_t stage_bytes;    /* staged: bytes per stage                      */
 } rn_launch_info;
 
 enum { RN_OP_RMS = 0, RN_OP_LN = 1, RN_OP_DUAL = 2 };
@@ -193,6 +197,19 @@ RN_API int rn_plan(int op, const rn_view *x, const rn_view *y,
  * automatic persistent grid; 0 restores the automatic choice. Results do not
  * depend on it (rows are statically strided over blocks). Process-wide. */
 RN_API int rn_set_grid_override(int blocks);
+
+/* Kernel choice: 0 automatic (the register-resident kernels, measured
+ * fastest on B200); 1 register kernels; 2 the bulk-copy staged kernels
+ * (rows streamed through shared memory) wherever the shape allows. The
+ * per-row arithmetic is identical in both kinds of kernel, so results do not
+ * depend on it. Process-wide; meant for tests and measurements. */
+RN_API int rn_set_path_override(int path);
+
+/* Number of stage waits in the staged kernels that gave up after their time
+ * limit (each makes its block stop early, so a nonzero count means some
+ * outputs were not written). Reading synchronizes the current device; reset
+ * != 0 clears the counter. Needs a GPU. */
+RN_API int rn_device_error_count(unsigned int *count, int reset);
 
 #ifdef __cplusplus
 }

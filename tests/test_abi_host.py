@@ -163,9 +163,12 @@ def test_dual_validation(lib):
     assert dual(lib, q, k, yq, yk, eps=float("nan")) == 4
 
 
-def test_grid_override_control(lib):
+def test_testing_controls(lib):
     assert lib.rn_set_grid_override(-1) == 2
     assert lib.rn_set_grid_override(0) == 0
+    assert lib.rn_set_path_override(3) == 2
+    assert lib.rn_set_path_override(0) == 0
+    assert lib.rn_device_error_count(None, 0) == 1
 
 
 @pytest.mark.parametrize("shape,strides,want", [

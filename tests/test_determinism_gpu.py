@@ -64,3 +64,62 @@ def test_dual_is_one_launch_plan():
     w = torch.ones(128, dtype=torch.bfloat16, device="cuda")
     p = rn.plan(rn.RN_OP_DUAL, q, weight=w, bias=w, k=k)
     assert p["family"] == 0 and p["grid_blocks"] >= 1
+
+
+PATH_CASES = [
+    # (dtype, rows, dim, offset) -- offset > 0 makes rows start off the 16-byte grid
+    (torch.bfloat16, 3000, 128, 0), (torch.bfloat16, 2000, 768, 0), (torch.bfloat16, 2000, 1000, 0),
+    (torch.float32, 1500, 1024, 0), (torch.bfloat16, 700, 4096, 0), (torch.bfloat16, 700, 4097, 0),
+    (torch.bfloat16, 600, 8192, 0), (torch.bfloat16, 300, 16384, 0), (torch.bfloat16, 100, 32768, 0),
+    (torch.float32, 500, 4099, 0), (torch.float32, 200, 16384, 0), (torch.bfloat16, 900, 2048, 3),
+    (torch.bfloat16, 1200, 64, 0), (torch.float32, 900, 1536, 1),
+]
+
+
+@pytest.mark.parametrize("dtype,rows,dim,offset", PATH_CASES)
+def test_register_and_staged_kernels_agree_bitwise(dtype, rows, dim, offset):
+    big = wl.random_rows(rows, dim + offset, dtype, seed=dim, mean=0.5, std=2.0).cuda()
+    x = big[:, offset:offset + dim] if offset else big
+    w = wl.random_vector(dim, dtype, seed=1).cuda()
+    b = wl.random_vector(dim, dtype, seed=2, mean=0.0, std=0.1).cuda()
+    out = {}
+    try:
+        for path in (1, 2):
+            rn.set_path_override(path)
+            out[path] = (rn.rms_norm(x, w, 1e-6), rn.layer_norm(x, w, b, 1e-5),
+                         rn.plan(rn.RN_OP_LN, x, weight=w, bias=b)["staged"])
+    finally:
+        rn.set_path_override(0)
+    assert out[1][2] == 0
+    assert torch.equal(out[1][0], out[2][0])
+    assert torch.equal(out[1][1], out[2][1])
+    assert rn.device_error_count(reset=True) == 0
+
+
+def test_staged_dual_agrees_with_register_dual():
+    q = wl.random_rows(8192 * 4, 128, torch.bfloat16, seed=9).cuda()
+    k = wl.random_rows(8192, 128, torch.bfloat16, seed=10).cuda()
+    wq = wl.random_vector(128, torch.bfloat16, seed=11).cuda()
+    wk = wl.random_vector(128, torch.bfloat16, seed=12).cuda()
+    res = {}
+    try:
+        for path in (1, 2):
+            rn.set_path_override(path)
+            res[path] = rn.dual_head_rms_norm(q, k, wq, wk, 1e-6)
+    finally:
+        rn.set_path_override(0)
+    assert torch.equal(res[1][0], res[2][0]) and torch.equal(res[1][1], res[2][1])
+    assert rn.device_error_count(reset=True) == 0
+
+
+def test_staged_plans_for_the_large_workloads():
+    try:
+        for dim in (4096, 8192, 16384, 4097):
+            x = torch.empty(65536, dim, dtype=torch.bfloat16, device="cuda")
+            assert rn.plan(rn.RN_OP_LN, x)["staged"] == 0  # default: register kernels
+            rn.set_path_override(2)
+            p = rn.plan(rn.RN_OP_LN, x)
+            rn.set_path_override(0)
+            assert p["staged"] == 1 and p["stages"] >= 2, (dim, p)
+    finally:
+        rn.set_path_override(0)

@@ -20,6 +20,7 @@ import os
 __all__ = [
     "RowNormError", "rn_rms_norm", "rn_layer_norm", "rn_dual_head_rms_norm",
     "rms_norm", "layer_norm", "dual_head_rms_norm", "plan", "set_grid_override",
+    "set_path_override", "device_error_count",
     "library_path", "load_library", "view_params",
 ]
 
@@ -48,7 +49,8 @@ class rn_view(ctypes.Structure):
 class rn_launch_info(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "family", "threads_per_row", "chunks_per_thread", "smem_bytes", "block_threads",
-        "grid_blocks", "blocks_per_sm", "vector_y", "phase_period", "exact")]
+        "grid_blocks", "blocks_per_sm", "vector_y", "phase_period", "exact", "staged",
+        "stages", "stage_bytes")]
 
 
 _lib = None
@@ -75,12 +77,15 @@ def load_library():
         lib.rn_plan.argtypes = [ctypes.c_int, pv, pv, pv, pv, vp, vp,
                                 ctypes.POINTER(rn_launch_info)]
         lib.rn_set_grid_override.argtypes = [ctypes.c_int]
+        lib.rn_set_path_override.argtypes = [ctypes.c_int]
+        lib.rn_device_error_count.argtypes = [ctypes.POINTER(ctypes.c_uint), ctypes.c_int]
         lib.rn_status_string.argtypes = [ctypes.c_int]
         lib.rn_status_string.restype = ctypes.c_char_p
         lib.rn_last_error.argtypes = []
         lib.rn_last_error.restype = ctypes.c_char_p
         for fn in (lib.rn_rms_norm, lib.rn_layer_norm, lib.rn_dual_head_rms_norm,
-                   lib.rn_plan, lib.rn_set_grid_override, lib.rn_abi_version):
+                   lib.rn_plan, lib.rn_set_grid_override, lib.rn_abi_version,
+                   lib.rn_set_path_override, lib.rn_device_error_count):
             fn.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -230,3 +235,15 @@ def plan(op, x, out=None, weight=None, bias=None, k=None, out_k=None):
 def set_grid_override(blocks: int):
     """Testing control: launch exactly ``blocks`` blocks (0 = automatic)."""
     _check(load_library().rn_set_grid_override(int(blocks)))
+
+
+def set_path_override(path: int):
+    """Testing control: 0 automatic, 1 register kernels, 2 staged kernels."""
+    _check(load_library().rn_set_path_override(int(path)))
+
+
+def device_error_count(reset: bool = False) -> int:
+    """Stage waits that timed out in the staged kernels (synchronizes)."""
+    n = ctypes.c_uint(0)
+    _check(load_library().rn_device_error_count(ctypes.byref(n), int(reset)))
+    return n.value

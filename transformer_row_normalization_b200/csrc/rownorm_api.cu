@@ -13,11 +13,13 @@
 #include "rownorm.h"
 #include "rownorm_kernels.cuh"
 #include "rownorm_launch.h"
+#include "rownorm_staged.cuh"
 
 namespace {
 
 thread_local char g_last_error[512] = "";
 int g_grid_override = 0;
+int g_path_override = 0;  // 0 automatic, 1 register kernels, 2 staged kernels
 
 int fail(int status, const char* fmt, ...) {
   va_list ap;
@@ -173,9 +175,8 @@ SegPlan plan_segment(const rn_view* x, const rn_view* y, const void* w, const vo
     p.phase_period = period;
   }
   p.exact = rows_aligned && ya % 16 == 0 &&
-            (y->rows <= 1 || (y->row_stride * es) % 16 == 0);
-  (void)w;
-  (void)b;
+            (y->rows <= 1 || (y->row_stride * es) % 16 == 0) &&
+            reinterpret_cast<uintptr_t>(w) % 16 == 0 && reinterpret_cast<uintptr_t>(b) % 16 == 0;
   return p;
 }
 
@@ -190,40 +191,77 @@ const void* kernel_for(int dtype, int op, const SegPlan& p) {
 
 struct DeviceInfo {
   int sms = 0;
+  int smem_per_sm = 0;
+  int smem_per_block = 0;
+};
+
+struct OccKey {
+  const void* fn;
+  int smem;
+  bool operator==(const OccKey& o) const { return fn == o.fn && smem == o.smem; }
+};
+struct OccKeyHash {
+  size_t operator()(const OccKey& k) const {
+    return std::hash<const void*>()(k.fn) ^ (std::hash<int>()(k.smem) << 1);
+  }
 };
 
 std::mutex g_mu;
 DeviceInfo g_dev[64];
-std::unordered_map<const void*, int> g_occ[64];
+std::unordered_map<OccKey, int, OccKeyHash> g_occ[64];  // resident blocks per SM
+std::unordered_map<const void*, int> g_smem_attr[64];   // kernels given the opt-in limit
 
 int device_sms(int dev, int* sms) {
   std::lock_guard<std::mutex> lk(g_mu);
   if (dev < 0 || dev >= 64) return fail(RN_ERR_CUDA, "device ordinal %d out of range", dev);
   if (!g_dev[dev].sms) {
-    cudaError_t e = cudaDeviceGetAttribute(&g_dev[dev].sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return fail(RN_ERR_CUDA, "SM count query: %s", cudaGetErrorString(e));
+    DeviceInfo d;
+    cudaError_t e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+      e = cudaDeviceGetAttribute(&d.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    if (e == cudaSuccess)
+      e = cudaDeviceGetAttribute(&d.smem_per_block, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return fail(RN_ERR_CUDA, "device query: %s", cudaGetErrorString(e));
+    g_dev[dev] = d;
   }
   *sms = g_dev[dev].sms;
   return RN_OK;
 }
 
-// Also raises the kernel's dynamic shared memory limit the first time a
-// configuration needs more than the default 48 KB.
+DeviceInfo device_info(int dev) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  return g_dev[dev];
+}
+
+// Resident blocks per SM of `fn` at `smem` bytes of dynamic shared memory.
+// The first query of a kernel on a device also lifts its dynamic shared
+// memory limit to the device's opt-in maximum (the default is 48 KB).
 int blocks_per_sm(int dev, const void* fn, int threads, int smem, int* out) {
   std::lock_guard<std::mutex> lk(g_mu);
-  auto it = g_occ[dev].find(fn);
+  auto it = g_occ[dev].find(OccKey{fn, smem});
   if (it != g_occ[dev].end()) {
     *out = it->second;
     return RN_OK;
   }
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess)
-    return fail(RN_ERR_CUDA, "shared memory attribute: %s", cudaGetErrorString(e));
+  cudaError_t e;
+  if (!g_smem_attr[dev].count(fn)) {
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, fn);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               g_dev[dev].smem_per_block - (int)fa.sharedSizeBytes);
+    if (e != cudaSuccess)
+      return fail(RN_ERR_CUDA, "shared memory attribute: %s", cudaGetErrorString(e));
+    g_smem_attr[dev][fn] = g_dev[dev].smem_per_block - (int)fa.sharedSizeBytes;
+  }
+  if (smem > g_smem_attr[dev][fn])
+    return fail(RN_ERR_UNSUPPORTED, "%d B of shared memory above the limit %d B", smem,
+                g_smem_attr[dev][fn]);
   int n = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, smem);
   if (e != cudaSuccess) return fail(RN_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
-  if (n < 1) n = 1;
-  g_occ[dev][fn] = n;
+  if (n < 1) return fail(RN_ERR_UNSUPPORTED, "kernel does not fit on an SM (%d B shared)", smem);
+  g_occ[dev][OccKey{fn, smem}] = n;
   *out = n;
   return RN_OK;
 }
@@ -231,12 +269,115 @@ int blocks_per_sm(int dev, const void* fn, int threads, int smem, int* out) {
 struct Launch {
   const void* fn;
   int smem;
+  int staged;       // 1: rows_staged_kernel with StagedParams
   rn_launch_info info;
+  // staged kernels only
+  int stages, stage_bytes, tile_rows[2], contiguous[2], cache_offset;
+  int64_t tiles[2];
 };
 
-// Plans the launch for one or two segments that share one kernel.
-int plan_launch(int dtype, int op, const SegPlan* plans, const int64_t* rows, int nseg,
-                Launch* out) {
+constexpr int kNarrowTileBytes = 16 * 1024;  // rows per stage ~ 16 KB (lane-group rows)
+constexpr int kMaxStages = 8;
+
+int round_up(int64_t v, int64_t m) { return (int)((v + m - 1) / m * m); }
+
+// Plans a bulk-copy staged launch (selected with rn_set_path_override(2))
+// when the shape qualifies: rows wider than the lane-group limit (one block
+// per row, any layout), or lane-group rows in an EXACT layout. Returns false
+// (and leaves the register-kernel plan in charge) otherwise.
+bool plan_staged(int dtype, int op, const SegPlan* plans, const rn_view* const* xs,
+                 const void* const* ws, const void* const* bs, int nseg, int dev, int sms,
+                 Launch* out) {
+  // The register kernels are the default: measured on B200 they sustain more
+  // HBM bandwidth than this staged pipeline at every shape tried (the staged
+  // kernel keeps more bytes in flight but runs fewer warps per SM and pays a
+  // block barrier per tile). The staged kernel stays selectable.
+  if (g_path_override != 2) return false;
+  const int es = elem_size(dtype);
+  const bool wide = plans[0].family == 1;
+  for (int i = 0; i < nseg; ++i) {
+    if (plans[i].family != plans[0].family) return false;
+    if (!wide && !plans[i].exact) return false;
+  }
+  int chunks = 0;
+  bool exact = true;
+  for (int i = 0; i < nseg; ++i) {
+    chunks = plans[i].chunks > chunks ? plans[i].chunks : chunks;
+    exact = exact && plans[i].exact;
+  }
+  const int threads = wide ? plans[0].lanes : 256;
+  const void* fn = dtype == RN_F32 ? rn::staged_kernel_f32(op, wide, exact, threads, chunks)
+                                   : rn::staged_kernel_bf16(op, wide, exact, threads, chunks);
+  if (!fn) return false;
+  Launch l{};
+  l.staged = 1;
+  int64_t stage_bytes = 0;
+  for (int i = 0; i < nseg; ++i) {
+    const int64_t row_bytes = xs[i]->dim * es;
+    int64_t tr = 1;
+    if (!wide) {
+      tr = kNarrowTileBytes / row_bytes;
+      if (tr < 1) tr = 1;
+      if (tr > xs[i]->rows) tr = xs[i]->rows > 0 ? xs[i]->rows : 1;
+    }
+    l.tile_rows[i] = (int)tr;
+    l.contiguous[i] = xs[i]->rows <= 1 || xs[i]->row_stride == xs[i]->dim;
+    l.tiles[i] = ceil_div(xs[i]->rows, tr);
+    const int64_t b = tr * row_bytes;
+    if (b > stage_bytes) stage_bytes = b;
+  }
+  l.stage_bytes = round_up(stage_bytes, 128);
+  const int affine = exact ? 0 : rn::affine_cache_smem_bytes(op, threads, chunks);
+  const DeviceInfo di = device_info(dev);
+  // blocks per SM: as many as leave each block its weight cache and four
+  // stages, at most 1024 threads per SM
+  const int64_t want = affine + 4LL * l.stage_bytes + 1024 + 512;
+  int blocks_target = (int)(di.smem_per_sm / want);
+  if (blocks_target > (threads >= 1024 ? 1 : 1024 / threads))
+    blocks_target = threads >= 1024 ? 1 : 1024 / threads;
+  if (blocks_target < 1) blocks_target = 1;
+  // per block: the SM's shared memory split over the target block count, less
+  // the 1 KB the hardware reserves per block and the kernel's static arrays
+  int64_t budget = di.smem_per_sm / blocks_target - 1024 - 512;
+  if (budget > di.smem_per_block - 512) budget = di.smem_per_block - 512;
+  int64_t stages = (budget - affine) / l.stage_bytes;
+  if (stages > kMaxStages) stages = kMaxStages;
+  if (stages < 2) return false;
+  l.stages = (int)stages;
+  l.cache_offset = (int)(stages * l.stage_bytes);
+  l.fn = fn;
+  l.smem = l.cache_offset + affine;
+  int bps = 0;
+  if (blocks_per_sm(dev, fn, threads, l.smem, &bps)) return false;
+  int64_t needed = 1;
+  for (int i = 0; i < nseg; ++i) needed = l.tiles[i] > needed ? l.tiles[i] : needed;
+  int64_t grid = (int64_t)sms * bps;
+  if (wide && grid >= plans[0].phase_period) grid -= grid % plans[0].phase_period;
+  if (needed < grid) grid = needed;
+  if (g_grid_override > 0) grid = g_grid_override;
+  rn_launch_info& in = l.info;
+  in.family = plans[0].family;
+  in.threads_per_row = plans[0].lanes;
+  in.chunks_per_thread = chunks;
+  in.smem_bytes = l.smem;
+  in.block_threads = threads;
+  in.grid_blocks = (int32_t)grid;
+  in.blocks_per_sm = bps;
+  in.vector_y = plans[0].vector_y;
+  in.phase_period = plans[0].phase_period;
+  in.exact = exact;
+  in.staged = 1;
+  in.stages = l.stages;
+  in.stage_bytes = l.stage_bytes;
+  *out = l;
+  return true;
+}
+
+// Plans the launch for one or two segments that share one kernel: the
+// bulk-copy staged kernel where it applies, else the register kernels.
+int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* xs,
+                const void* const* ws, const void* const* bs, int nseg, Launch* out) {
+  int64_t rows[2] = {xs[0]->rows, nseg > 1 ? xs[1]->rows : 0};
   SegPlan merged = plans[0];
   for (int i = 1; i < nseg; ++i) {
     if (plans[i].chunks > merged.chunks) merged.chunks = plans[i].chunks;
@@ -250,8 +391,9 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const int64_t* rows, in
   int sms = 0, bps = 0;
   int st = device_sms(dev, &sms);
   if (st) return st;
+  if (plan_staged(dtype, op, plans, xs, ws, bs, nseg, dev, sms, out)) return RN_OK;
   const int threads = merged.family == 0 ? rn::kWarpBlock : merged.lanes;
-  const int smem = rn::affine_smem_bytes(op, threads, merged.chunks);
+  const int smem = merged.exact ? 0 : rn::affine_cache_smem_bytes(op, threads, merged.chunks);
   st = blocks_per_sm(dev, fn, threads, smem, &bps);
   if (st) return st;
   int64_t needed = 1;
@@ -275,6 +417,7 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const int64_t* rows, in
   if (g_grid_override > 0) grid = g_grid_override;
   out->fn = fn;
   out->smem = smem;
+  out->staged = 0;
   rn_launch_info& in = out->info;
   in.family = merged.family;
   in.threads_per_row = plans[0].lanes;
@@ -306,10 +449,30 @@ rn::Segment make_segment(const rn_view* x, const rn_view* y, const void* w, cons
 }
 
 int launch(const Launch& l, const rn::Params& params, void* stream) {
-  void* args[] = {const_cast<rn::Params*>(&params)};
-  cudaError_t e = cudaLaunchKernel(l.fn, dim3((unsigned)l.info.grid_blocks),
-                                   dim3((unsigned)l.info.block_threads), args, (size_t)l.smem,
-                                   static_cast<cudaStream_t>(stream));
+  cudaError_t e;
+  if (l.staged) {
+    rn::StagedParams sp{};
+    for (int i = 0; i < 2; ++i) {
+      sp.seg[i] = params.seg[i];
+      sp.tile_rows[i] = l.tile_rows[i];
+      sp.contiguous[i] = l.contiguous[i];
+      sp.tiles[i] = i < params.nseg ? l.tiles[i] : 0;
+    }
+    sp.nseg = params.nseg;
+    sp.eps = params.eps;
+    sp.stages = l.stages;
+    sp.stage_bytes = l.stage_bytes;
+    sp.cache_offset = l.cache_offset;
+    void* args[] = {&sp};
+    e = cudaLaunchKernel(l.fn, dim3((unsigned)l.info.grid_blocks),
+                         dim3((unsigned)l.info.block_threads), args, (size_t)l.smem,
+                         static_cast<cudaStream_t>(stream));
+  } else {
+    void* args[] = {const_cast<rn::Params*>(&params)};
+    e = cudaLaunchKernel(l.fn, dim3((unsigned)l.info.grid_blocks),
+                         dim3((unsigned)l.info.block_threads), args, (size_t)l.smem,
+                         static_cast<cudaStream_t>(stream));
+  }
   if (e != cudaSuccess) return fail(RN_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
   return RN_OK;
 }
@@ -336,8 +499,10 @@ int run_single(int op, const rn_view* x, const void* w, const void* b, float eps
   if (x->rows == 0 && !plan_only) return RN_OK;
   const SegPlan p = plan_segment(x, y, w, b);
   Launch l{};
-  const int64_t rows = x->rows > 0 ? x->rows : 1;
-  if ((st = plan_launch(x->dtype, op, &p, &rows, 1, &l))) return st;
+  const rn_view* xs[1] = {x};
+  const void* ws[1] = {w};
+  const void* bs[1] = {b};
+  if ((st = plan_launch(x->dtype, op, &p, xs, ws, bs, 1, &l))) return st;
   if (plan_only) {
     *plan_only = l.info;
     return RN_OK;
@@ -374,9 +539,11 @@ int run_dual(const rn_view* q, const rn_view* k, const void* wq, const void* wk,
   if ((st = check_output(yk, k, not_yk, 1, vecs, dims, 2, "yk"))) return st;
   if (q->rows == 0 && k->rows == 0 && !plan_only) return RN_OK;
   const SegPlan plans[2] = {plan_segment(q, yq, wq, nullptr), plan_segment(k, yk, wk, nullptr)};
-  const int64_t rows[2] = {q->rows, k->rows};
+  const rn_view* xs[2] = {q, k};
+  const void* ws[2] = {wq, wk};
+  const void* bs[2] = {nullptr, nullptr};
   Launch l{};
-  if ((st = plan_launch(q->dtype, rn::kOpRms, plans, rows, 2, &l))) return st;
+  if ((st = plan_launch(q->dtype, rn::kOpRms, plans, xs, ws, bs, 2, &l))) return st;
   if (plan_only) {
     *plan_only = l.info;
     return RN_OK;
@@ -441,6 +608,23 @@ RN_API int rn_plan(int op, const rn_view* x, const rn_view* y, const rn_view* x2
 RN_API int rn_set_grid_override(int blocks) {
   if (blocks < 0) return fail(RN_ERR_SHAPE, "grid override must be >= 0");
   g_grid_override = blocks;
+  return RN_OK;
+}
+
+RN_API int rn_set_path_override(int path) {
+  if (path < 0 || path > 2) return fail(RN_ERR_SHAPE, "path override must be 0, 1 or 2");
+  g_path_override = path;
+  return RN_OK;
+}
+
+RN_API int rn_device_error_count(unsigned int* count, int reset) {
+  if (!count) return fail(RN_ERR_NULL, "count is NULL");
+  unsigned int a = 0, b = 0;
+  int e = rn::staged_timeouts_f32(&a, reset != 0);
+  if (e == 0) e = rn::staged_timeouts_bf16(&b, reset != 0);
+  if (e != 0)
+    return fail(RN_ERR_CUDA, "device error counter: %s", cudaGetErrorString((cudaError_t)e));
+  *count = a + b;
   return RN_OK;
 }
 

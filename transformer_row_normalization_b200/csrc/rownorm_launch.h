@@ -10,8 +10,9 @@ constexpr int kCtaMinChunks = 2;             // chunks per thread, block family
 constexpr int kCtaMaxChunks = 5;
 constexpr int kTargetChunksPerThread = 4;    // 64 bytes of loads in flight per thread
 
-// Shared memory holding each thread's weight (and bias) chunk slots.
-constexpr int affine_smem_bytes(int op, int threads, int chunks) {
+// Shared memory of the realigned weight/bias cache (layouts that are not
+// EXACT): each thread's chunk slots of the weight (and bias).
+constexpr int affine_cache_smem_bytes(int op, int threads, int chunks) {
   return threads * chunks * 16 * (op == 1 ? 2 : 1);
 }
 
@@ -22,15 +23,27 @@ constexpr int cta_key(int op, bool exact, int threads, int chunks) {
   return ((op * 2 + (exact ? 1 : 0)) * 2048 + threads) * 8 + chunks;
 }
 
+constexpr int staged_key(int op, bool wide, bool exact, int threads, int chunks) {
+  return (((op * 2 + (wide ? 1 : 0)) * 2 + (exact ? 1 : 0)) * 2048 + threads) * 16 + chunks;
+}
+
 // Kernel entry for (op, exact, chunks per lane) in the warp family; nullptr
 // if that configuration is not compiled. op: 0 RMSNorm, 1 LayerNorm. exact:
-// every row of x and y starts 16-byte aligned and dim is a multiple of the
-// 16-byte vector width.
+// every row of x and y starts 16-byte aligned, dim is a multiple of the
+// 16-byte vector width, and the weight and bias start 16-byte aligned.
 const void* warp_kernel_f32(int op, bool exact, int chunks);
 const void* warp_kernel_bf16(int op, bool exact, int chunks);
 // Kernel entry for (op, exact, threads per block, chunks per thread) in the
 // block family; nullptr if not compiled.
 const void* cta_kernel_f32(int op, bool exact, int threads, int chunks);
 const void* cta_kernel_bf16(int op, bool exact, int threads, int chunks);
+// Bulk-copy staged kernels: wide (one block per row) or narrow (lane groups,
+// rows 16-byte aligned); nullptr if not compiled.
+const void* staged_kernel_f32(int op, bool wide, bool exact, int threads, int chunks);
+const void* staged_kernel_bf16(int op, bool wide, bool exact, int threads, int chunks);
+// Timed-out stage waits recorded by the staged kernels of each element type
+// (optionally resetting the counter); returns a cudaError_t value.
+int staged_timeouts_f32(unsigned int* count, bool reset);
+int staged_timeouts_bf16(unsigned int* count, bool reset);
 
 }  // namespace rn
