@@ -317,7 +317,7 @@ def cpu_baseline(step, chunk_rows=2048):
 # ---------------------------------------------------------------------------
 
 
-def config_dict(rows, nbytes, world):
+def config_dict(rows, nbytes, world, path=0):
     return {
         "workload": "large bf16 suite: dual q/k head RMSNorm q[8192,32,128]+k[8192,8,128] "
                     "(1 launch); RMSNorm [16,4096,4096] with 1% x50 outliers; LayerNorm "
@@ -327,6 +327,7 @@ def config_dict(rows, nbytes, world):
         "launches_per_step": 7,
         "l2": "no flush: each step reads ~4.6 GB and writes ~4.6 GB (126 MB L2)",
         "parallelism": f"dp{world} (weak: each rank its own copy of the suite)",
+        "kernel_path": path,
     }
 
 
@@ -337,6 +338,7 @@ def run_ours(args):
     dist = init_dist(world, "nccl")
     peak, peak_kind = measured_peak()
     step = Step(device, rank)
+    step.rn.set_path_override(args.path)
     stream = torch.cuda.Stream(device)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -392,7 +394,7 @@ def run_ours(args):
             "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic: seeded on the device with the workloads' shapes and distributions",
-            "config": config_dict(rows, nbytes, world),
+            "config": config_dict(rows, nbytes, world, args.path),
             "hbm": {"gbs": round(gbs, 1), "peak_gbs": peak, "frac": round(gbs / peak, 4),
                     "peak_source": peak_kind},
             "roofline": roofline, "cpu_baseline": base, "e2e": e2e,
@@ -506,7 +508,8 @@ def main(argv=None):
     ap.add_argument("--profile-case", default=None,
                     help="OP:DTYPE:ROWS:DIM -- launch one workload for a profiler capture")
     ap.add_argument("--path", type=int, default=0,
-                    help="with --profile-case: 0 automatic, 1 register, 2 staged kernels")
+                    help="kernel choice: 0 automatic, 1 register, 2 staged, "
+                         "3 register with next-row prefetch")
     args = ap.parse_args(argv)
     if args.profile_case:
         return run_profile_case(args)

@@ -198,11 +198,12 @@ RN_API int rn_plan(int op, const rn_view *x, const rn_view *y,
  * depend on it (rows are statically strided over blocks). Process-wide. */
 RN_API int rn_set_grid_override(int blocks);
 
-/* Kernel choice: 0 automatic (the register-resident kernels, measured
- * fastest on B200); 1 register kernels; 2 the bulk-copy staged kernels
- * (rows streamed through shared memory) wherever the shape allows. The
- * per-row arithmetic is identical in both kinds of kernel, so results do not
- * depend on it. Process-wide; meant for tests and measurements. */
+/* Kernel choice: 0 automatic; 1 register-resident kernels loading rows
+ * directly; 2 the bulk-copy staged kernels (rows streamed through shared
+ * memory) wherever the shape allows; 3 register-resident kernels with a
+ * per-thread next-row prefetch through shared memory (cp.async). The per-row
+ * arithmetic is identical in every kind of kernel, so results do not depend
+ * on it. Process-wide; meant for tests and measurements. */
 RN_API int rn_set_path_override(int path);
 
 /* Number of stage waits in the staged kernels that gave up after their time

@@ -166,7 +166,7 @@ def test_dual_validation(lib):
 def test_testing_controls(lib):
     assert lib.rn_set_grid_override(-1) == 2
     assert lib.rn_set_grid_override(0) == 0
-    assert lib.rn_set_path_override(3) == 2
+    assert lib.rn_set_path_override(4) == 2
     assert lib.rn_set_path_override(0) == 0
     assert lib.rn_device_error_count(None, 0) == 1
 

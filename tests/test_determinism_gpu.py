@@ -84,15 +84,16 @@ def test_register_and_staged_kernels_agree_bitwise(dtype, rows, dim, offset):
     b = wl.random_vector(dim, dtype, seed=2, mean=0.0, std=0.1).cuda()
     out = {}
     try:
-        for path in (1, 2):
+        for path in (1, 2, 3):
             rn.set_path_override(path)
             out[path] = (rn.rms_norm(x, w, 1e-6), rn.layer_norm(x, w, b, 1e-5),
                          rn.plan(rn.RN_OP_LN, x, weight=w, bias=b)["staged"])
     finally:
         rn.set_path_override(0)
-    assert out[1][2] == 0
-    assert torch.equal(out[1][0], out[2][0])
-    assert torch.equal(out[1][1], out[2][1])
+    assert out[1][2] == 0 and out[3][2] == 0
+    for path in (2, 3):
+        assert torch.equal(out[1][0], out[path][0]), path
+        assert torch.equal(out[1][1], out[path][1]), path
     assert rn.device_error_count(reset=True) == 0
 
 

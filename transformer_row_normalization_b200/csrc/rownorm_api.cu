@@ -19,7 +19,7 @@ namespace {
 
 thread_local char g_last_error[512] = "";
 int g_grid_override = 0;
-int g_path_override = 0;  // 0 automatic, 1 register kernels, 2 staged kernels
+int g_path_override = 0;  // 0 automatic, 1 register, 2 staged, 3 register + prefetch
 
 int fail(int status, const char* fmt, ...) {
   va_list ap;
@@ -159,7 +159,12 @@ SegPlan plan_segment(const rn_view* x, const rn_view* y, const void* w, const vo
     p.chunks = (int)ceil_div(nch, p.lanes);
   } else {
     p.family = 1;
-    int nt = pow2_ceil(ceil_div(ceil_div(D, V), per_thread));
+    // the fewest threads (a power of two, 128..1024) that hold a row of any
+    // 16-byte phase in at most kCtaMaxChunks chunks each: the block
+    // reductions and the per-row setup are paid once per row per thread, so
+    // more work per thread is cheaper (a function of dtype and D only)
+    const int64_t nch_any_phase = (D + 2 * V - 2) / V;
+    int nt = pow2_ceil(ceil_div(nch_any_phase, rn::kCtaMaxChunks));
     p.lanes = nt < 128 ? 128 : (nt > 1024 ? 1024 : nt);
     p.chunks = (int)ceil_div(nch, p.lanes);
     if (p.chunks < rn::kCtaMinChunks) p.chunks = rn::kCtaMinChunks;
@@ -269,6 +274,7 @@ int blocks_per_sm(int dev, const void* fn, int threads, int smem, int* out) {
 struct Launch {
   const void* fn;
   int smem;
+  int prefetch;     // register kernels: next-row prefetch through shared memory
   int staged;       // 1: rows_staged_kernel with StagedParams
   rn_launch_info info;
   // staged kernels only
@@ -393,7 +399,19 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
   if (st) return st;
   if (plan_staged(dtype, op, plans, xs, ws, bs, nseg, dev, sms, out)) return RN_OK;
   const int threads = merged.family == 0 ? rn::kWarpBlock : merged.lanes;
-  const int smem = merged.exact ? 0 : rn::affine_cache_smem_bytes(op, threads, merged.chunks);
+  const int cache = merged.exact ? 0 : rn::affine_cache_smem_bytes(op, threads, merged.chunks);
+  const int slots = rn::prefetch_slots_smem_bytes(threads, merged.chunks);
+  // Next-row prefetch where it measured faster on B200: lane-group rows and
+  // blocks of 256 or more threads (few blocks per SM, so few rows in
+  // flight); blocks of 128 threads already keep 8+ rows per SM in flight and
+  // ran slower with it. Only when the slots fit beside the weight cache
+  // (with a margin for the kernel's static shared memory).
+  const bool want_prefetch =
+      g_path_override == 3 ||
+      (g_path_override == 0 && (merged.family == 0 || merged.lanes >= 256));
+  const int prefetch =
+      want_prefetch && cache + slots <= device_info(dev).smem_per_block - 1024 ? 1 : 0;
+  const int smem = cache + (prefetch ? slots : 0);
   st = blocks_per_sm(dev, fn, threads, smem, &bps);
   if (st) return st;
   int64_t needed = 1;
@@ -417,6 +435,7 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
   if (g_grid_override > 0) grid = g_grid_override;
   out->fn = fn;
   out->smem = smem;
+  out->prefetch = prefetch;
   out->staged = 0;
   rn_launch_info& in = out->info;
   in.family = merged.family;
@@ -468,7 +487,9 @@ int launch(const Launch& l, const rn::Params& params, void* stream) {
                          dim3((unsigned)l.info.block_threads), args, (size_t)l.smem,
                          static_cast<cudaStream_t>(stream));
   } else {
-    void* args[] = {const_cast<rn::Params*>(&params)};
+    rn::Params pr = params;
+    pr.prefetch = l.prefetch;
+    void* args[] = {&pr};
     e = cudaLaunchKernel(l.fn, dim3((unsigned)l.info.grid_blocks),
                          dim3((unsigned)l.info.block_threads), args, (size_t)l.smem,
                          static_cast<cudaStream_t>(stream));
@@ -612,7 +633,7 @@ RN_API int rn_set_grid_override(int blocks) {
 }
 
 RN_API int rn_set_path_override(int path) {
-  if (path < 0 || path > 2) return fail(RN_ERR_SHAPE, "path override must be 0, 1 or 2");
+  if (path < 0 || path > 3) return fail(RN_ERR_SHAPE, "path override must be 0, 1, 2 or 3");
   g_path_override = path;
   return RN_OK;
 }

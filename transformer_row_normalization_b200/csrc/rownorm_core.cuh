@@ -3,13 +3,13 @@
 // What is computed (per row of D elements, binary32 arithmetic):
 //   RMSNorm   ("Emily.Fast", rms_norm/3):
 //               ss   = sum_i x_i^2
-//               rstd = rsqrt(ss / D + eps)
+//               rstd = rsqrt(ss * (1/D) + eps)
 //               y_j  = (x_j * rstd) * w_j
 //   LayerNorm ("Emily.Fast", layer_norm/4; population variance):
 //               K    = x_0                       (shift: a constant row gives
 //               d_i  = x_i - K                    exactly zero deviations)
-//               mean = (sum_i d_i) / D
-//               var  = (sum_i (d_i - mean)^2) / D
+//               mean = (sum_i d_i) * (1/D)
+//               var  = (sum_i (d_i - mean)^2) * (1/D)
 //               rstd = rsqrt(var + eps)
 //               y_j  = ((d_j - mean) * rstd) * w_j + b_j   (one fused multiply-add)
 //   The page calls its LayerNorm statistic "Welford-style"; the two passes
@@ -27,6 +27,7 @@
 // Arithmetic. Elements are processed as pairs (columns 2j, 2j+1 of a chunk)
 // with the packed binary32 instructions of sm_100 (add/sub/mul/fma .f32x2);
 // each lane of a packed instruction rounds exactly like its scalar form.
+// (1/D) is the binary32 reciprocal of D, rounded to nearest.
 //
 // Summation order (fixed; it depends only on D, the element type, the
 // threads per row and the row's 16-byte phase):
@@ -64,40 +65,62 @@ struct Segment {
 
 // ---------------------------------------------------------------------------
 // packed binary32 pairs
+//
+// A pair lives in one 64-bit register (low half = the element at the even
+// column), so the packed instructions take their operands without any
+// register shuffling.
 
-__device__ __forceinline__ float2 add2(float2 a, float2 b) {
-  float2 d;
-  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
-      " add.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+struct F2 {
+  unsigned long long v;
+};
+
+__device__ __forceinline__ F2 make2(float lo, float hi) {
+  F2 d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d.v) : "f"(lo), "f"(hi));
   return d;
 }
-__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
-  float2 d;
-  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
-      " sub.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+__device__ __forceinline__ F2 make2_bits(uint32_t lo, uint32_t hi) {
+  F2 d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d.v) : "r"(lo), "r"(hi));
   return d;
 }
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-  float2 d;
-  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
-      " mul.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+__device__ __forceinline__ void split2(F2 a, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(a.v));
+}
+__device__ __forceinline__ F2 zero2() { return F2{0ull}; }
+__device__ __forceinline__ F2 splat(float v) { return make2(v, v); }
+__device__ __forceinline__ F2 add2(F2 a, F2 b) {
+  F2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d.v) : "l"(a.v), "l"(b.v));
   return d;
 }
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
-  float2 d;
-  asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
-      " mov.b64 rc, {%6, %7};\n fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+__device__ __forceinline__ F2 sub2(F2 a, F2 b) {
+  F2 d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d.v) : "l"(a.v), "l"(b.v));
   return d;
 }
-__device__ __forceinline__ float2 splat(float v) { return make_float2(v, v); }
+__device__ __forceinline__ F2 mul2(F2 a, F2 b) {
+  F2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d.v) : "l"(a.v), "l"(b.v));
+  return d;
+}
+__device__ __forceinline__ F2 fma2(F2 a, F2 b, F2 c) {
+  F2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d.v) : "l"(a.v), "l"(b.v), "l"(c.v));
+  return d;
+}
+// Keep the low / high element or replace it by +0 (masks of partial chunks).
+__device__ __forceinline__ F2 mask2(F2 a, bool keep_lo, bool keep_hi) {
+  float lo, hi;
+  split2(a, lo, hi);
+  return make2(keep_lo ? lo : 0.f, keep_hi ? hi : 0.f);
+}
+// lo + hi, rounded once.
+__device__ __forceinline__ float hsum2(F2 a) {
+  float lo, hi;
+  split2(a, lo, hi);
+  return __fadd_rn(lo, hi);
+}
 
 // ---------------------------------------------------------------------------
 // element types: a 16-byte chunk <-> P = V/2 binary32 pairs
@@ -115,13 +138,15 @@ struct Elem<float> {
     return __float_as_uint(*p);
   }
   static __device__ __forceinline__ void put(float* p, float v) { *p = v; }
-  static __device__ __forceinline__ void unpack(const uint4& u, float2 (&f)[2]) {
-    f[0] = make_float2(__uint_as_float(u.x), __uint_as_float(u.y));
-    f[1] = make_float2(__uint_as_float(u.z), __uint_as_float(u.w));
+  static __device__ __forceinline__ void unpack(const uint4& u, F2 (&f)[2]) {
+    f[0] = make2_bits(u.x, u.y);
+    f[1] = make2_bits(u.z, u.w);
   }
-  static __device__ __forceinline__ uint4 pack(const float2 (&f)[2]) {
-    return make_uint4(__float_as_uint(f[0].x), __float_as_uint(f[0].y),
-                      __float_as_uint(f[1].x), __float_as_uint(f[1].y));
+  static __device__ __forceinline__ uint4 pack(const F2 (&f)[2]) {
+    uint4 u;
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(u.x), "=r"(u.y) : "l"(f[0].v));
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(u.z), "=r"(u.w) : "l"(f[1].v));
+    return u;
   }
   static __device__ __forceinline__ uint4 assemble(const uint32_t (&e)[4]) {
     return make_uint4(e[0], e[1], e[2], e[3]);
@@ -142,22 +167,24 @@ struct Elem<__nv_bfloat16> {
   static __device__ __forceinline__ void put(__nv_bfloat16* p, float v) {
     *p = __float2bfloat16_rn(v);
   }
-  static __device__ __forceinline__ float2 pair(uint32_t w) {
-    __nv_bfloat162 h;
-    *reinterpret_cast<uint32_t*>(&h) = w;
-    return __bfloat1622float2(h);
+  // bfloat16 is the upper half of a binary32 pattern: widening is exact bit
+  // placement (low element: shift up; high element: clear the low half).
+  static __device__ __forceinline__ F2 pair(uint32_t w) {
+    return make2_bits(w << 16, w & 0xffff0000u);
   }
-  static __device__ __forceinline__ uint32_t pack_pair(float2 v) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+  static __device__ __forceinline__ uint32_t pack_pair(F2 v) {
+    float lo, hi;
+    split2(v, lo, hi);
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
   }
-  static __device__ __forceinline__ void unpack(const uint4& u, float2 (&f)[4]) {
+  static __device__ __forceinline__ void unpack(const uint4& u, F2 (&f)[4]) {
     f[0] = pair(u.x);
     f[1] = pair(u.y);
     f[2] = pair(u.z);
     f[3] = pair(u.w);
   }
-  static __device__ __forceinline__ uint4 pack(const float2 (&f)[4]) {
+  static __device__ __forceinline__ uint4 pack(const F2 (&f)[4]) {
     return make_uint4(pack_pair(f[0]), pack_pair(f[1]), pack_pair(f[2]), pack_pair(f[3]));
   }
   static __device__ __forceinline__ uint4 assemble(const uint32_t (&e)[8]) {
@@ -177,6 +204,24 @@ __device__ __forceinline__ void store_stream(void* p, const uint4& v) {
 }
 __device__ __forceinline__ uint4 load_cached(const void* p) {
   return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Per-thread asynchronous 16-byte copy global -> shared (L2 only, not L1),
+// grouped with commit/wait; a thread waits only for its own copies.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(smem_dst)), "l"(gsrc)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // Geometry of one row.
@@ -211,26 +256,61 @@ __device__ __forceinline__ bool chunk_full(const Row<T>& g, int k) {
   return k < g.nch && (k > 0 || g.phase == 0) && (k < g.nch - 1 || g.tail_full);
 }
 
+// Whether the thread whose slots are k0, k0 + step, ... owns one of the (at
+// most two) partial chunks of the row: chunk 0 when the row does not start on
+// a 16-byte boundary, chunk nch-1 when it does not end on one. Every chunk
+// k < nch is owned by thread k % step. Threads without a partial chunk take
+// straight-line code for the row; the others take the checked code.
+template <typename T, bool EXACT>
+__device__ __forceinline__ bool owns_partial(const Row<T>& g, int k0, int step) {
+  if constexpr (EXACT) return false;
+  return (g.phase > 0 && k0 == 0) || (!g.tail_full && (g.nch - 1) % step == k0);
+}
+
 // Chunk k of a row from global memory; columns outside [0, D) (and chunks
 // past the row) read as 0 and are never dereferenced.
 template <typename T, bool EXACT>
 __device__ __forceinline__ void load_chunk(const Row<T>& g, int D, int k,
-                                           float2 (&f)[Elem<T>::P]) {
+                                           F2 (&f)[Elem<T>::P]) {
   constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
   if (chunk_full<T, EXACT>(g, k)) {
     Elem<T>::unpack(load_stream(g.x_al + (long long)k * V), f);
   } else if constexpr (EXACT) {
 #pragma unroll
-    for (int j = 0; j < P; ++j) f[j] = make_float2(0.f, 0.f);
+    for (int j = 0; j < P; ++j) f[j] = zero2();
   } else {
 #pragma unroll
     for (int j = 0; j < P; ++j) {
       const int c = k * V + 2 * j - g.phase;
-      f[j].x = ((unsigned)c < (unsigned)D) ? Elem<T>::get(g.x_al + k * V + 2 * j) : 0.f;
-      f[j].y = ((unsigned)(c + 1) < (unsigned)D) ? Elem<T>::get(g.x_al + k * V + 2 * j + 1)
-                                                 : 0.f;
+      const float lo = ((unsigned)c < (unsigned)D) ? Elem<T>::get(g.x_al + k * V + 2 * j) : 0.f;
+      const float hi =
+          ((unsigned)(c + 1) < (unsigned)D) ? Elem<T>::get(g.x_al + k * V + 2 * j + 1) : 0.f;
+      f[j] = make2(lo, hi);
     }
+  }
+}
+
+// All of a thread's slots of one row from global memory.
+template <typename T, bool EXACT, int NSLOT>
+__device__ __forceinline__ void load_row(const Row<T>& g, int D, int k0, int step, bool edge,
+                                         F2 (&v)[NSLOT][Elem<T>::P]) {
+  constexpr int V = Elem<T>::V;
+  constexpr int P = Elem<T>::P;
+  if (!edge) {
+#pragma unroll
+    for (int p = 0; p < NSLOT; ++p) {
+      const int k = k0 + step * p;
+      if (k < g.nch) {
+        Elem<T>::unpack(load_stream(g.x_al + (long long)k * V), v[p]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < P; ++j) v[p][j] = zero2();
+      }
+    }
+  } else {
+#pragma unroll
+    for (int p = 0; p < NSLOT; ++p) load_chunk<T, false>(g, D, k0 + step * p, v[p]);
   }
 }
 
@@ -239,78 +319,86 @@ __device__ __forceinline__ void load_chunk(const Row<T>& g, int D, int k,
 
 // RMSNorm: sum of squares (absent columns hold zeros, which add nothing).
 template <typename T, int NSLOT>
-__device__ __forceinline__ float sum_squares(const float2 (&v)[NSLOT][Elem<T>::P]) {
+__device__ __forceinline__ float sum_squares(const F2 (&v)[NSLOT][Elem<T>::P]) {
   constexpr int P = Elem<T>::P;
-  float2 acc = make_float2(0.f, 0.f);
+  F2 acc = zero2();
 #pragma unroll
   for (int p = 0; p < NSLOT; ++p)
 #pragma unroll
     for (int j = 0; j < P; ++j) acc = fma2(v[p][j], v[p][j], acc);
-  return __fadd_rn(acc.x, acc.y);
+  return hsum2(acc);
 }
 
 // LayerNorm pass 1: replaces x by d = x - K (zero outside the row) and
 // returns the thread's sum of d.
 template <typename T, bool EXACT, int NSLOT>
-__device__ __forceinline__ float shift_and_sum(float2 (&v)[NSLOT][Elem<T>::P], const Row<T>& g,
-                                               int D, int k0, int step, float K) {
+__device__ __forceinline__ float shift_and_sum(F2 (&v)[NSLOT][Elem<T>::P], const Row<T>& g,
+                                               int D, int k0, int step, float K, bool edge) {
   constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
-  const float2 K2 = splat(K);
-  float2 acc = make_float2(0.f, 0.f);
+  const F2 K2 = splat(K);
+  F2 acc = zero2();
+  if (!edge) {
 #pragma unroll
-  for (int p = 0; p < NSLOT; ++p) {
-    const int k = k0 + step * p;
-    if (chunk_full<T, EXACT>(g, k)) {
+    for (int p = 0; p < NSLOT; ++p) {
+      if (k0 + step * p < g.nch) {
 #pragma unroll
-      for (int j = 0; j < P; ++j) {
-        v[p][j] = sub2(v[p][j], K2);
-        acc = add2(acc, v[p][j]);
+        for (int j = 0; j < P; ++j) {
+          v[p][j] = sub2(v[p][j], K2);
+          acc = add2(acc, v[p][j]);
+        }
       }
-    } else if constexpr (!EXACT) {
+    }
+  } else {
+#pragma unroll
+    for (int p = 0; p < NSLOT; ++p) {
+      const int k = k0 + step * p;
 #pragma unroll
       for (int j = 0; j < P; ++j) {
         const int c = k * V + 2 * j - g.phase;
-        const float2 d = sub2(v[p][j], K2);
-        v[p][j].x = ((unsigned)c < (unsigned)D) ? d.x : 0.f;
-        v[p][j].y = ((unsigned)(c + 1) < (unsigned)D) ? d.y : 0.f;
+        v[p][j] = mask2(sub2(v[p][j], K2), (unsigned)c < (unsigned)D,
+                        (unsigned)(c + 1) < (unsigned)D);
         acc = add2(acc, v[p][j]);
       }
     }
   }
-  return __fadd_rn(acc.x, acc.y);
+  return hsum2(acc);
 }
 
 // LayerNorm pass 2: the thread's sum of (d - mean)^2 over the row's columns.
 template <typename T, bool EXACT, int NSLOT>
-__device__ __forceinline__ float sum_dev_squares(const float2 (&v)[NSLOT][Elem<T>::P],
+__device__ __forceinline__ float sum_dev_squares(const F2 (&v)[NSLOT][Elem<T>::P],
                                                  const Row<T>& g, int D, int k0, int step,
-                                                 float mean) {
+                                                 float mean, bool edge) {
   constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
-  const float2 M2 = splat(mean);
-  float2 acc = make_float2(0.f, 0.f);
+  const F2 M2 = splat(mean);
+  F2 acc = zero2();
+  if (!edge) {
 #pragma unroll
-  for (int p = 0; p < NSLOT; ++p) {
-    const int k = k0 + step * p;
-    if (chunk_full<T, EXACT>(g, k)) {
+    for (int p = 0; p < NSLOT; ++p) {
+      if (k0 + step * p < g.nch) {
 #pragma unroll
-      for (int j = 0; j < P; ++j) {
-        const float2 t = sub2(v[p][j], M2);
-        acc = fma2(t, t, acc);
+        for (int j = 0; j < P; ++j) {
+          const F2 t = sub2(v[p][j], M2);
+          acc = fma2(t, t, acc);
+        }
       }
-    } else if constexpr (!EXACT) {
+    }
+  } else {
+#pragma unroll
+    for (int p = 0; p < NSLOT; ++p) {
+      const int k = k0 + step * p;
 #pragma unroll
       for (int j = 0; j < P; ++j) {
         const int c = k * V + 2 * j - g.phase;
-        float2 t = sub2(v[p][j], M2);
-        t.x = ((unsigned)c < (unsigned)D) ? t.x : 0.f;
-        t.y = ((unsigned)(c + 1) < (unsigned)D) ? t.y : 0.f;
+        const F2 t = mask2(sub2(v[p][j], M2), (unsigned)c < (unsigned)D,
+                           (unsigned)(c + 1) < (unsigned)D);
         acc = fma2(t, t, acc);
       }
     }
   }
-  return __fadd_rn(acc.x, acc.y);
+  return hsum2(acc);
 }
 
 // ---------------------------------------------------------------------------
@@ -355,22 +443,22 @@ template <typename T, bool BIAS>
 struct AffineDirect {
   const T* w;
   const T* b;
-  __device__ __forceinline__ void get(int /*p*/, int k, float2 (&wf)[Elem<T>::P],
-                                      float2 (&bf)[Elem<T>::P]) const {
+  __device__ __forceinline__ void get(int /*p*/, int k, F2 (&wf)[Elem<T>::P],
+                                      F2 (&bf)[Elem<T>::P]) const {
     constexpr int V = Elem<T>::V;
     constexpr int P = Elem<T>::P;
     if (w) {
       Elem<T>::unpack(load_cached(w + k * V), wf);
     } else {
 #pragma unroll
-      for (int j = 0; j < P; ++j) wf[j] = make_float2(1.f, 1.f);
+      for (int j = 0; j < P; ++j) wf[j] = splat(1.f);
     }
     if constexpr (BIAS) {
       if (b) {
         Elem<T>::unpack(load_cached(b + k * V), bf);
       } else {
 #pragma unroll
-        for (int j = 0; j < P; ++j) bf[j] = make_float2(0.f, 0.f);
+        for (int j = 0; j < P; ++j) bf[j] = zero2();
       }
     }
   }
@@ -421,8 +509,8 @@ struct AffineCache {
     phase = row_phase;
   }
 
-  __device__ __forceinline__ void get(int p, int /*k*/, float2 (&wf)[Elem<T>::P],
-                                      float2 (&bf)[Elem<T>::P]) const {
+  __device__ __forceinline__ void get(int p, int /*k*/, F2 (&wf)[Elem<T>::P],
+                                      F2 (&bf)[Elem<T>::P]) const {
     Elem<T>::unpack(w[p * blockDim.x + threadIdx.x], wf);
     if constexpr (BIAS) Elem<T>::unpack(b[p * blockDim.x + threadIdx.x], bf);
   }
@@ -436,19 +524,19 @@ constexpr int affine_cache_bytes(int threads) {
 // Normalize the thread's chunks of one row, apply weight (and bias), store.
 template <typename T, int OP, bool EXACT, int NSLOT, typename Src>
 __device__ __forceinline__ void normalize_store(const Segment& s, const Row<T>& g,
-                                                const float2 (&v)[NSLOT][Elem<T>::P],
+                                                const F2 (&v)[NSLOT][Elem<T>::P],
                                                 const Src& src, int k0, int step, float rstd,
-                                                float mean) {
+                                                float mean, bool edge) {
   constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
   const int D = s.dim;
-  const float2 R2 = splat(rstd);
-  const float2 M2 = splat(mean);
+  const F2 R2 = splat(rstd);
+  const F2 M2 = splat(mean);
 #pragma unroll
   for (int p = 0; p < NSLOT; ++p) {
     const int k = k0 + step * p;
     if (k >= g.nch) continue;
-    float2 wf[P], bf[P], o[P];
+    F2 wf[P], bf[P], o[P];
     src.get(p, k, wf, bf);
 #pragma unroll
     for (int j = 0; j < P; ++j) {
@@ -457,14 +545,16 @@ __device__ __forceinline__ void normalize_store(const Segment& s, const Row<T>& 
       else
         o[j] = fma2(mul2(sub2(v[p][j], M2), R2), wf[j], bf[j]);
     }
-    if (EXACT || (s.vector_y && chunk_full<T, EXACT>(g, k))) {
+    if (EXACT || (s.vector_y && (!edge || chunk_full<T, EXACT>(g, k)))) {
       store_stream(g.y_row - g.phase + (long long)k * V, Elem<T>::pack(o));
     } else {
 #pragma unroll
       for (int j = 0; j < P; ++j) {
         const int c = k * V + 2 * j - g.phase;
-        if ((unsigned)c < (unsigned)D) Elem<T>::put(g.y_row + c, o[j].x);
-        if ((unsigned)(c + 1) < (unsigned)D) Elem<T>::put(g.y_row + c + 1, o[j].y);
+        float lo, hi;
+        split2(o[j], lo, hi);
+        if ((unsigned)c < (unsigned)D) Elem<T>::put(g.y_row + c, lo);
+        if ((unsigned)(c + 1) < (unsigned)D) Elem<T>::put(g.y_row + c + 1, hi);
       }
     }
   }
@@ -473,19 +563,21 @@ __device__ __forceinline__ void normalize_store(const Segment& s, const Row<T>& 
 // rstd (and mean) of one row from the thread's slots, with `reduce` summing
 // a per-thread partial over the threads of the row.
 template <typename T, int OP, bool EXACT, int NSLOT, typename Reduce>
-__device__ __forceinline__ void row_stats(float2 (&v)[NSLOT][Elem<T>::P], const Row<T>& g,
+__device__ __forceinline__ void row_stats(F2 (&v)[NSLOT][Elem<T>::P], const Row<T>& g,
                                           int D, int k0, int step, float K, float eps,
-                                          Reduce reduce, float& rstd, float& mean) {
-  const float d_f = (float)D;
+                                          bool edge, Reduce reduce, float& rstd, float& mean) {
+  // Means are sums times 1/D rounded to binary32 (one multiply instead of a
+  // divide per row; exact for power-of-two D, within 2 ulps otherwise).
+  const float inv_d = __frcp_rn((float)D);
   if (OP == kOpRms) {
     const float ss = reduce(sum_squares<T, NSLOT>(v));
     mean = 0.f;
-    rstd = rsqrtf(__fadd_rn(__fdiv_rn(ss, d_f), eps));
+    rstd = rsqrtf(__fadd_rn(__fmul_rn(ss, inv_d), eps));
   } else {
-    const float s1 = reduce(shift_and_sum<T, EXACT, NSLOT>(v, g, D, k0, step, K));
-    mean = __fdiv_rn(s1, d_f);
-    const float s2 = reduce(sum_dev_squares<T, EXACT, NSLOT>(v, g, D, k0, step, mean));
-    rstd = rsqrtf(__fadd_rn(__fdiv_rn(s2, d_f), eps));
+    const float s1 = reduce(shift_and_sum<T, EXACT, NSLOT>(v, g, D, k0, step, K, edge));
+    mean = __fmul_rn(s1, inv_d);
+    const float s2 = reduce(sum_dev_squares<T, EXACT, NSLOT>(v, g, D, k0, step, mean, edge));
+    rstd = rsqrtf(__fadd_rn(__fmul_rn(s2, inv_d), eps));
   }
 }
 

@@ -1,8 +1,8 @@
 // Register-resident row normalization kernels (sm_100a).
 //
-// Each row is read from HBM once into registers (as binary32 pairs), reduced
-// and written back; the per-row arithmetic, layout and summation order are
-// those of rownorm_core.cuh. Two families:
+// Each row is read from HBM once and normalized from registers (as binary32
+// pairs); the per-row arithmetic, layout and summation order are those of
+// rownorm_core.cuh. Two families:
 //   rows_warp_kernel  a group of G lanes (a power of two <= 32) of one warp
 //                     owns a row; G is chosen so each lane holds about four
 //                     16-byte chunks. Used for D <= 1024.
@@ -15,9 +15,15 @@
 // grid is a multiple of the phase period), so the realigned weight/bias
 // cache of non-aligned layouts is filled once.
 //
+// Prefetch. While a thread normalizes row r, its chunks of its next row are
+// already on their way: each thread copies its own full chunks of row
+// r + stride into its own shared memory slots with cp.async and waits only
+// for its own copies (cp.async.wait_group), so the HBM latency of a row hides
+// behind the previous row's arithmetic without any barrier. The shift K of
+// the next row (LayerNorm) is loaded at the same time.
+//
 // The bulk-copy staged kernels (rownorm_staged.cuh) run the same per-row
-// code on rows streamed through shared memory; the planner prefers them for
-// large row counts, and the two give identical bits.
+// code; which kernel the planner picks never changes a bit.
 #pragma once
 
 #include "rownorm_core.cuh"
@@ -28,6 +34,7 @@ struct Params {
   Segment seg[2];
   int nseg;
   float eps;
+  int prefetch;  // 1: next-row prefetch through shared memory; 0: direct loads
 };
 
 __device__ __forceinline__ Segment pick_segment(const Segment (&seg)[2], int i) {
@@ -40,12 +47,65 @@ constexpr int kWarpBlock = 256;
 constexpr int kMinThreadsPerSmWarp = 768;
 constexpr int kMinThreadsPerSm = 1024;
 
+// Per-thread prefetch slots: [2 stages][NSLOT][blockDim.x] 16-byte words.
+// When the slots do not fit in shared memory next to the weight cache (the
+// planner decides), `on` is 0: nothing is copied ahead and rows are loaded
+// straight from global memory when they are taken.
+template <typename T, int NSLOT>
+struct Prefetch {
+  uint4* base;
+  int on;
+  __device__ __forceinline__ uint4* slot(int stage, int p) const {
+    return base + ((stage * NSLOT + p) * blockDim.x + threadIdx.x);
+  }
+  // Start the copies of the thread's full chunks of row g into `stage`.
+  template <bool EXACT>
+  __device__ __forceinline__ void issue(const Row<T>& g, int k0, int step, int stage) const {
+    constexpr int V = Elem<T>::V;
+    if (!on) return;
+#pragma unroll
+    for (int p = 0; p < NSLOT; ++p) {
+      const int k = k0 + step * p;
+      if (chunk_full<T, EXACT>(g, k)) cp_async16(slot(stage, p), g.x_al + (long long)k * V);
+    }
+  }
+  // The thread's slots of row g: full chunks from `stage` (copies complete),
+  // partial chunks element by element from global memory, absent ones zero.
+  template <bool EXACT>
+  __device__ __forceinline__ void take(const Row<T>& g, int D, int k0, int step, int stage,
+                                       bool edge, F2 (&v)[NSLOT][Elem<T>::P]) const {
+    constexpr int P = Elem<T>::P;
+    if (!on) {
+      load_row<T, EXACT, NSLOT>(g, D, k0, step, edge, v);
+      return;
+    }
+#pragma unroll
+    for (int p = 0; p < NSLOT; ++p) {
+      const int k = k0 + step * p;
+      if (k < g.nch && (!edge || chunk_full<T, EXACT>(g, k))) {
+        Elem<T>::unpack(*slot(stage, p), v[p]);
+      } else if (edge) {
+        load_chunk<T, false>(g, D, k, v[p]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < P; ++j) v[p][j] = zero2();
+      }
+    }
+  }
+};
+
+template <int NSLOT>
+__host__ __device__ constexpr int prefetch_smem_bytes(int threads) {
+  return 2 * NSLOT * threads * 16;
+}
+
 template <typename T, int OP, bool EXACT, int VPL>
 __global__ void __launch_bounds__(kWarpBlock, kMinThreadsPerSmWarp / kWarpBlock)
 rows_warp_kernel(const Params p) {
   constexpr int P = Elem<T>::P;
   constexpr bool BIAS = OP == kOpLn;
   extern __shared__ __align__(128) unsigned char smem[];
+  const Prefetch<T, VPL> pf{reinterpret_cast<uint4*>(smem), p.prefetch};
   const int lane = threadIdx.x & 31;
   const long long warp = (long long)blockIdx.x * (kWarpBlock / 32) + (threadIdx.x >> 5);
   const long long nwarps = (long long)gridDim.x * (kWarpBlock / 32);
@@ -59,27 +119,46 @@ rows_warp_kernel(const Params p) {
     const unsigned mask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << (gi * G));
     const long long ngroups = nwarps * per_warp;
     const int D = s.dim;
+    const T* x = static_cast<const T*>(s.x);
     AffineCache<T, VPL, BIAS> cache;
-    if constexpr (!EXACT) cache.init(smem);
+    if constexpr (!EXACT)
+      cache.init(smem + (p.prefetch ? prefetch_smem_bytes<VPL>(kWarpBlock) : 0));
     const AffineDirect<T, BIAS> direct{static_cast<const T*>(s.w), static_cast<const T*>(s.b)};
     auto reduce = [&](float t) { return group_sum(t, G, mask); };
+    long long r = warp * per_warp + gi;
+    Row<T> gn;
+    float Kn = 0.f;
+    if (r < s.rows) {
+      gn = row_geometry<T, EXACT>(s, r);
+      pf.template issue<EXACT>(gn, gl, G, 0);
+      if (OP == kOpLn) Kn = Elem<T>::get(x + r * s.x_stride);
+    }
+    cp_async_commit();
 #pragma unroll 1
-    for (long long r = warp * per_warp + gi; r < s.rows; r += ngroups) {
-      float2 v[VPL][P];
-      const Row<T> g = row_geometry<T, EXACT>(s, r);
-#pragma unroll
-      for (int q = 0; q < VPL; ++q) load_chunk<T, EXACT>(g, D, gl + G * q, v[q]);
-      const float K =
-          OP == kOpLn ? Elem<T>::get(static_cast<const T*>(s.x) + r * s.x_stride) : 0.f;
+    for (int i = 0; r < s.rows; ++i, r += ngroups) {
+      const Row<T> g = gn;
+      const float K = Kn;
+      const long long rn = r + ngroups;
+      if (rn < s.rows) {
+        gn = row_geometry<T, EXACT>(s, rn);
+        pf.template issue<EXACT>(gn, gl, G, (i + 1) & 1);
+        if (OP == kOpLn) Kn = Elem<T>::get(x + rn * s.x_stride);
+      }
+      cp_async_commit();
+      cp_async_wait<1>();
+      const bool edge = owns_partial<T, EXACT>(g, gl, G);
+      F2 v[VPL][P];
+      pf.template take<EXACT>(g, D, gl, G, i & 1, edge, v);
       float rstd, mean;
-      row_stats<T, OP, EXACT, VPL>(v, g, D, gl, G, K, p.eps, reduce, rstd, mean);
+      row_stats<T, OP, EXACT, VPL>(v, g, D, gl, G, K, p.eps, edge, reduce, rstd, mean);
       if constexpr (EXACT) {
-        normalize_store<T, OP, EXACT, VPL>(s, g, v, direct, gl, G, rstd, mean);
+        normalize_store<T, OP, EXACT, VPL>(s, g, v, direct, gl, G, rstd, mean, edge);
       } else {
         if (g.phase != cache.phase) cache.fill(s, g.phase, gl, G);
-        normalize_store<T, OP, EXACT, VPL>(s, g, v, cache, gl, G, rstd, mean);
+        normalize_store<T, OP, EXACT, VPL>(s, g, v, cache, gl, G, rstd, mean, edge);
       }
     }
+    cp_async_wait<0>();
   }
 }
 
@@ -92,6 +171,7 @@ rows_cta_kernel(const Params p) {
   // thread has passed the barrier of the reduction in between.
   __shared__ float red[2][NT / 32];
   extern __shared__ __align__(128) unsigned char smem[];
+  const Prefetch<T, VPT> pf{reinterpret_cast<uint4*>(smem), p.prefetch};
   int slot = 0;
   const int tid = threadIdx.x;
   auto reduce = [&](float t) {
@@ -103,26 +183,44 @@ rows_cta_kernel(const Params p) {
   for (int si = 0; si < p.nseg; ++si) {
     const Segment s = pick_segment(p.seg, si);
     const int D = s.dim;
+    const T* x = static_cast<const T*>(s.x);
     AffineCache<T, VPT, BIAS> cache;
-    if constexpr (!EXACT) cache.init(smem);
+    if constexpr (!EXACT) cache.init(smem + (p.prefetch ? prefetch_smem_bytes<VPT>(NT) : 0));
     const AffineDirect<T, BIAS> direct{static_cast<const T*>(s.w), static_cast<const T*>(s.b)};
+    long long r = blockIdx.x;
+    Row<T> gn;
+    float Kn = 0.f;
+    if (r < s.rows) {
+      gn = row_geometry<T, EXACT>(s, r);
+      pf.template issue<EXACT>(gn, tid, NT, 0);
+      if (OP == kOpLn) Kn = Elem<T>::get(x + r * s.x_stride);
+    }
+    cp_async_commit();
 #pragma unroll 1
-    for (long long r = blockIdx.x; r < s.rows; r += gridDim.x) {
-      float2 v[VPT][P];
-      const Row<T> g = row_geometry<T, EXACT>(s, r);
-#pragma unroll
-      for (int q = 0; q < VPT; ++q) load_chunk<T, EXACT>(g, D, tid + NT * q, v[q]);
-      const float K =
-          OP == kOpLn ? Elem<T>::get(static_cast<const T*>(s.x) + r * s.x_stride) : 0.f;
+    for (int i = 0; r < s.rows; ++i, r += gridDim.x) {
+      const Row<T> g = gn;
+      const float K = Kn;
+      const long long rn = r + gridDim.x;
+      if (rn < s.rows) {
+        gn = row_geometry<T, EXACT>(s, rn);
+        pf.template issue<EXACT>(gn, tid, NT, (i + 1) & 1);
+        if (OP == kOpLn) Kn = Elem<T>::get(x + rn * s.x_stride);
+      }
+      cp_async_commit();
+      cp_async_wait<1>();
+      const bool edge = owns_partial<T, EXACT>(g, tid, NT);
+      F2 v[VPT][P];
+      pf.template take<EXACT>(g, D, tid, NT, i & 1, edge, v);
       float rstd, mean;
-      row_stats<T, OP, EXACT, VPT>(v, g, D, tid, NT, K, p.eps, reduce, rstd, mean);
+      row_stats<T, OP, EXACT, VPT>(v, g, D, tid, NT, K, p.eps, edge, reduce, rstd, mean);
       if constexpr (EXACT) {
-        normalize_store<T, OP, EXACT, VPT>(s, g, v, direct, tid, NT, rstd, mean);
+        normalize_store<T, OP, EXACT, VPT>(s, g, v, direct, tid, NT, rstd, mean, edge);
       } else {
         if (g.phase != cache.phase) cache.fill(s, g.phase, tid, NT);
-        normalize_store<T, OP, EXACT, VPT>(s, g, v, cache, tid, NT, rstd, mean);
+        normalize_store<T, OP, EXACT, VPT>(s, g, v, cache, tid, NT, rstd, mean, edge);
       }
     }
+    cp_async_wait<0>();
   }
 }
 

@@ -15,6 +15,11 @@ constexpr int kTargetChunksPerThread = 4;    // 64 bytes of loads in flight per 
 constexpr int affine_cache_smem_bytes(int op, int threads, int chunks) {
   return threads * chunks * 16 * (op == 1 ? 2 : 1);
 }
+// Shared memory of the register kernels' prefetch slots (two stages of each
+// thread's chunk slots).
+constexpr int prefetch_slots_smem_bytes(int threads, int chunks) {
+  return 2 * chunks * threads * 16;
+}
 
 constexpr int warp_key(int op, bool exact, int chunks) {
   return (op * 2 + (exact ? 1 : 0)) * 16 + chunks;

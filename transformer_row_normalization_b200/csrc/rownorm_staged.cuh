@@ -51,10 +51,6 @@ struct StagedParams {
   int cache_offset;    // byte offset of the weight/bias cache in shared memory
 };
 
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
 __device__ __forceinline__ unsigned long long global_timer() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -157,7 +153,7 @@ __device__ __forceinline__ void issue_tile(const StagedParams& p, long long mine
 // ends element by element from global memory.
 template <typename T, bool EXACT>
 __device__ __forceinline__ void stage_chunk(const Row<T>& g, const unsigned char* stage, int D,
-                                            int k, float2 (&f)[Elem<T>::P]) {
+                                            int k, F2 (&f)[Elem<T>::P]) {
   constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
   if (chunk_full<T, EXACT>(g, k)) {
@@ -165,15 +161,9 @@ __device__ __forceinline__ void stage_chunk(const Row<T>& g, const unsigned char
     Elem<T>::unpack(*reinterpret_cast<const uint4*>(stage + 16 * j), f);
   } else if constexpr (EXACT) {
 #pragma unroll
-    for (int q = 0; q < P; ++q) f[q] = make_float2(0.f, 0.f);
+    for (int q = 0; q < P; ++q) f[q] = zero2();
   } else {
-#pragma unroll
-    for (int q = 0; q < P; ++q) {
-      const int c = k * V + 2 * q - g.phase;
-      f[q].x = ((unsigned)c < (unsigned)D) ? Elem<T>::get(g.x_al + k * V + 2 * q) : 0.f;
-      f[q].y = ((unsigned)(c + 1) < (unsigned)D) ? Elem<T>::get(g.x_al + k * V + 2 * q + 1)
-                                                 : 0.f;
-    }
+    load_chunk<T, false>(g, D, k, f);
   }
 }
 
@@ -242,20 +232,21 @@ rows_staged_kernel(const StagedParams p) {
     if constexpr (WIDE) {
       const int D = s.dim;
       const Row<T> g = row_geometry<T, EXACT>(s, tile);
-      float2 v[VPT][P];
+      F2 v[VPT][P];
 #pragma unroll
       for (int q = 0; q < VPT; ++q) stage_chunk<T, EXACT>(g, stage, D, tid + NT * q, v[q]);
       float K = 0.f;
       if (OP == kOpLn)
         K = g.phase ? Elem<T>::get(g.x_al + g.phase)
                     : Elem<T>::get(reinterpret_cast<const T*>(stage));
+      const bool edge = owns_partial<T, EXACT>(g, tid, NT);
       float rstd, mean;
-      row_stats<T, OP, EXACT, VPT>(v, g, D, tid, NT, K, p.eps, block_reduce, rstd, mean);
+      row_stats<T, OP, EXACT, VPT>(v, g, D, tid, NT, K, p.eps, edge, block_reduce, rstd, mean);
       if constexpr (EXACT) {
-        normalize_store<T, OP, EXACT, VPT>(s, g, v, direct, tid, NT, rstd, mean);
+        normalize_store<T, OP, EXACT, VPT>(s, g, v, direct, tid, NT, rstd, mean, edge);
       } else {
         if (g.phase != cache.phase) cache.fill(s, g.phase, tid, NT);
-        normalize_store<T, OP, EXACT, VPT>(s, g, v, cache, tid, NT, rstd, mean);
+        normalize_store<T, OP, EXACT, VPT>(s, g, v, cache, tid, NT, rstd, mean, edge);
       }
     } else {
       const int G = s.lanes;
@@ -275,7 +266,7 @@ rows_staged_kernel(const StagedParams p) {
       for (int rr = group; rr < nr; rr += groups) {
         const Row<T> g = row_geometry<T, true>(s, r0 + rr);
         const unsigned char* row = stage + rr * row_bytes;
-        float2 v[VPT][P];
+        F2 v[VPT][P];
 #pragma unroll
         for (int q = 0; q < VPT; ++q) {
           const int k = gl + G * q;
@@ -283,13 +274,13 @@ rows_staged_kernel(const StagedParams p) {
             Elem<T>::unpack(*reinterpret_cast<const uint4*>(row + 16 * k), v[q]);
           } else {
 #pragma unroll
-            for (int j = 0; j < P; ++j) v[q][j] = make_float2(0.f, 0.f);
+            for (int j = 0; j < P; ++j) v[q][j] = zero2();
           }
         }
         const float K = OP == kOpLn ? Elem<T>::get(reinterpret_cast<const T*>(row)) : 0.f;
         float rstd, mean;
-        row_stats<T, OP, true, VPT>(v, g, D, gl, G, K, p.eps, group_reduce, rstd, mean);
-        normalize_store<T, OP, true, VPT>(s, g, v, direct, gl, G, rstd, mean);
+        row_stats<T, OP, true, VPT>(v, g, D, gl, G, K, p.eps, false, group_reduce, rstd, mean);
+        normalize_store<T, OP, true, VPT>(s, g, v, direct, gl, G, rstd, mean, false);
       }
     }
   }
