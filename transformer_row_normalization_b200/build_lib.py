@@ -21,7 +21,7 @@ LIB = os.path.join(PKG, "librownorm.so")
 SOURCES = ["rownorm_api.cu", "rownorm_warp_f32.cu", "rownorm_warp_bf16.cu",
            "rownorm_cta_f32.cu", "rownorm_cta_bf16.cu", "rownorm_staged_f32.cu",
            "rownorm_staged_bf16.cu"]
-HEADERS = ["rownorm_kernels.cuh", "rownorm_staged.cuh", "rownorm_launch.h"]
+HEADERS = ["rownorm_core.cuh", "rownorm_kernels.cuh", "rownorm_staged.cuh", "rownorm_launch.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
