@@ -138,10 +138,12 @@ struct SegPlan {
   int exact;         // every x and y row 16-byte aligned, dim % V == 0
 };
 
-// The lane count / block size is a function of (dtype, dim) only, so the
-// summation tree of a row never depends on the call; `chunks` (register
-// capacity) may grow for rows that are not 16-byte aligned, which only adds
-// empty slots.
+// The lane count / block size is a function of (dtype, dim) and, for lane
+// groups, of whether every row of x starts on a 16-byte boundary with
+// dim % V == 0; so the summation tree of a row never depends on anything
+// else about the call. Rows that are not so aligned have up to 2 (V - 1)
+// edge elements, one per thread, so their lane groups hold at least that
+// many lanes (blocks always do).
 SegPlan plan_segment(const rn_view* x, const rn_view* y, const void* w, const void* b) {
   const int es = elem_size(x->dtype);
   const int V = 16 / es;
@@ -149,24 +151,25 @@ SegPlan plan_segment(const rn_view* x, const rn_view* y, const void* w, const vo
   const uintptr_t xa = reinterpret_cast<uintptr_t>(x->data);
   const bool rows_aligned = (xa % 16 == 0) && (D % V == 0) &&
                             (x->rows <= 1 || (x->row_stride * es) % 16 == 0);
-  const int64_t nch = rows_aligned ? D / V : (D + 2 * V - 2) / V;
+  const int64_t nfull = D / V;  // full chunks of a row, at most (any phase)
   SegPlan p{};
   const int per_thread = rn::kTargetChunksPerThread;
   if (D <= kWarpFamilyMaxDim) {
     p.family = 0;
     int g = pow2_ceil(ceil_div(ceil_div(D, V), per_thread));
+    if (!rows_aligned && g < pow2_ceil(2 * (V - 1))) g = pow2_ceil(2 * (V - 1));
     p.lanes = g > 32 ? 32 : g;
-    p.chunks = (int)ceil_div(nch, p.lanes);
+    p.chunks = (int)ceil_div(nfull, p.lanes);
+    if (p.chunks < 1) p.chunks = 1;
   } else {
     p.family = 1;
-    // the fewest threads (a power of two, 128..1024) that hold a row of any
-    // 16-byte phase in at most kCtaMaxChunks chunks each: the block
-    // reductions and the per-row setup are paid once per row per thread, so
-    // more work per thread is cheaper (a function of dtype and D only)
-    const int64_t nch_any_phase = (D + 2 * V - 2) / V;
-    int nt = pow2_ceil(ceil_div(nch_any_phase, rn::kCtaMaxChunks));
+    // the fewest threads (a power of two, 128..1024) that hold a row in at
+    // most kCtaMaxChunks chunks each: the block reductions and the per-row
+    // setup are paid once per row per thread, so more work per thread is
+    // cheaper
+    int nt = pow2_ceil(ceil_div(nfull, rn::kCtaMaxChunks));
     p.lanes = nt < 128 ? 128 : (nt > 1024 ? 1024 : nt);
-    p.chunks = (int)ceil_div(nch, p.lanes);
+    p.chunks = (int)ceil_div(nfull, p.lanes);
     if (p.chunks < rn::kCtaMinChunks) p.chunks = rn::kCtaMinChunks;
   }
   const uintptr_t ya = reinterpret_cast<uintptr_t>(y->data);

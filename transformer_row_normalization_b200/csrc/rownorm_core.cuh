@@ -17,12 +17,13 @@
 //   and give the same population mean and variance.
 //
 // Row layout. A row is moved as 16-byte chunks on the 16-byte address grid:
-// chunk k of a row whose first element sits `phase` elements past a 16-byte
-// boundary covers columns [k*V - phase, k*V - phase + V), V = 16 / element
-// size. Chunks wholly inside the row move with one 16-byte access; the (at
-// most two) partial chunks at the row ends move element by element, so no
-// byte outside the caller's views is touched. A thread owns chunks
-// k0, k0 + step, k0 + 2*step, ... of every row it works on (slots).
+// the columns between the first and the last 16-byte boundary inside the row
+// form its full chunks, each moved with one 16-byte access; the at most
+// 2 (V - 1) columns before the first and after the last boundary (V = 16 /
+// element size) are its edge elements, moved one by one, so no byte outside
+// the caller's views is touched. A thread owns the full chunks k0,
+// k0 + step, k0 + 2*step, ... of every row it works on (slots) and at most
+// one edge element.
 //
 // Arithmetic. Elements are processed as pairs (columns 2j, 2j+1 of a chunk)
 // with the packed binary32 instructions of sm_100 (add/sub/mul/fma .f32x2);
@@ -33,7 +34,8 @@
 // threads per row and the row's 16-byte phase):
 //   1. each thread keeps two partial sums, one over the elements at even
 //      positions of its chunks and one over the odd positions, each added in
-//      slot order then position order; its partial is even + odd;
+//      slot order then position order; its partial is even + odd, plus the
+//      term of its edge element if it owns one;
 //   2. an xor butterfly over the G lanes sharing the row (offsets G/2 .. 1);
 //   3. for rows owned by a whole block of NW warps, the per-warp sums are
 //      combined by the same xor butterfly over lanes 0 .. NW-1 (warp w's sum
@@ -108,12 +110,6 @@ __device__ __forceinline__ F2 fma2(F2 a, F2 b, F2 c) {
   F2 d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d.v) : "l"(a.v), "l"(b.v), "l"(c.v));
   return d;
-}
-// Keep the low / high element or replace it by +0 (masks of partial chunks).
-__device__ __forceinline__ F2 mask2(F2 a, bool keep_lo, bool keep_hi) {
-  float lo, hi;
-  split2(a, lo, hi);
-  return make2(keep_lo ? lo : 0.f, keep_hi ? hi : 0.f);
 }
 // lo + hi, rounded once.
 __device__ __forceinline__ float hsum2(F2 a) {
@@ -224,181 +220,157 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Geometry of one row.
+// Geometry of one row. Its D columns split into three runs: `head` edge
+// elements before the first 16-byte boundary inside the row, `nfull` full
+// 16-byte chunks starting there (x_full), and the tail edge elements after
+// the last such boundary; nedge = head + tail <= 2 (V - 1).
+//
+// Ownership: of the `step` threads that share a row, thread k0 owns the full
+// chunks f = k0, k0 + step, k0 + 2 step, ... (its slots) and, when
+// k0 < nedge, edge element k0 (the head elements first, then the tail). The
+// planner gives rows that can have edge elements at least 2 (V - 1) threads,
+// so every edge element has an owner and all threads run the same
+// straight-line code on whole chunks.
 template <typename T>
 struct Row {
-  const T* x_al;   // x row start minus phase: 16-byte aligned
-  T* y_row;        // y row start
-  int phase;       // elements between the 16-byte boundary and the row start
-  int nch;         // chunks touched by the row
-  int tail_full;   // 1: the last chunk ends exactly at the row end
+  const T* x_row;   // x row start
+  const T* x_full;  // first full chunk (16-byte aligned)
+  T* y_row;         // y row start
+  int phase;        // elements between the 16-byte boundary and the row start
+  int head;         // edge elements before the first full chunk
+  int nfull;        // full chunks
+  int nedge;        // edge elements
 };
 
 // EXACT: the planner guarantees that every x and y row starts on a 16-byte
 // boundary, D is a multiple of V, and the weight and bias (where present)
-// start on 16-byte boundaries; so the phase is 0 and every chunk is full.
+// start on 16-byte boundaries; so the phase is 0 and there are no edges.
 template <typename T, bool EXACT>
 __device__ __forceinline__ Row<T> row_geometry(const Segment& s, long long r) {
   constexpr int V = Elem<T>::V;
   Row<T> g;
-  const T* xr = static_cast<const T*>(s.x) + r * s.x_stride;
-  g.phase = EXACT ? 0 : (int)((reinterpret_cast<uintptr_t>(xr) & 15u) / sizeof(T));
-  g.x_al = xr - g.phase;
+  g.x_row = static_cast<const T*>(s.x) + r * s.x_stride;
   g.y_row = static_cast<T*>(s.y) + r * s.y_stride;
-  g.nch = EXACT ? s.dim / V : (g.phase + s.dim + V - 1) / V;
-  g.tail_full = EXACT ? 1 : (((g.phase + s.dim) % V) == 0);
+  if constexpr (EXACT) {
+    g.phase = 0;
+    g.head = 0;
+    g.nfull = s.dim / V;
+    g.nedge = 0;
+  } else {
+    g.phase = (int)((reinterpret_cast<uintptr_t>(g.x_row) & 15u) / sizeof(T));
+    g.head = g.phase ? min(V - g.phase, s.dim) : 0;
+    g.nfull = (s.dim - g.head) / V;
+    g.nedge = s.dim - g.nfull * V;
+  }
+  g.x_full = g.x_row + g.head;
   return g;
 }
 
-template <typename T, bool EXACT>
-__device__ __forceinline__ bool chunk_full(const Row<T>& g, int k) {
-  if constexpr (EXACT) return k < g.nch;
-  return k < g.nch && (k > 0 || g.phase == 0) && (k < g.nch - 1 || g.tail_full);
+// Column of edge element e < nedge.
+template <typename T>
+__device__ __forceinline__ int edge_column(const Row<T>& g, int D, int e) {
+  return e < g.head ? e : D - g.nedge + e;
 }
 
-// Whether the thread whose slots are k0, k0 + step, ... owns one of the (at
-// most two) partial chunks of the row: chunk 0 when the row does not start on
-// a 16-byte boundary, chunk nch-1 when it does not end on one. Every chunk
-// k < nch is owned by thread k % step. Threads without a partial chunk take
-// straight-line code for the row; the others take the checked code.
+// The edge element of thread k0 (0 when it owns none), read on its own so
+// that no byte outside the row is touched.
 template <typename T, bool EXACT>
-__device__ __forceinline__ bool owns_partial(const Row<T>& g, int k0, int step) {
-  if constexpr (EXACT) return false;
-  return (g.phase > 0 && k0 == 0) || (!g.tail_full && (g.nch - 1) % step == k0);
+__device__ __forceinline__ float load_edge(const Row<T>& g, int D, int k0) {
+  if constexpr (EXACT) return 0.f;
+  return k0 < g.nedge ? Elem<T>::get(g.x_row + edge_column(g, D, k0)) : 0.f;
 }
 
-// Chunk k of a row from global memory; columns outside [0, D) (and chunks
-// past the row) read as 0 and are never dereferenced.
-template <typename T, bool EXACT>
-__device__ __forceinline__ void load_chunk(const Row<T>& g, int D, int k,
-                                           F2 (&f)[Elem<T>::P]) {
-  constexpr int V = Elem<T>::V;
-  constexpr int P = Elem<T>::P;
-  if (chunk_full<T, EXACT>(g, k)) {
-    Elem<T>::unpack(load_stream(g.x_al + (long long)k * V), f);
-  } else if constexpr (EXACT) {
-#pragma unroll
-    for (int j = 0; j < P; ++j) f[j] = zero2();
-  } else {
-#pragma unroll
-    for (int j = 0; j < P; ++j) {
-      const int c = k * V + 2 * j - g.phase;
-      const float lo = ((unsigned)c < (unsigned)D) ? Elem<T>::get(g.x_al + k * V + 2 * j) : 0.f;
-      const float hi =
-          ((unsigned)(c + 1) < (unsigned)D) ? Elem<T>::get(g.x_al + k * V + 2 * j + 1) : 0.f;
-      f[j] = make2(lo, hi);
-    }
-  }
-}
-
-// All of a thread's slots of one row from global memory.
-template <typename T, bool EXACT, int NSLOT>
-__device__ __forceinline__ void load_row(const Row<T>& g, int D, int k0, int step, bool edge,
+// All of a thread's slots of one row from global memory (absent ones zero).
+template <typename T, int NSLOT>
+__device__ __forceinline__ void load_row(const Row<T>& g, int k0, int step,
                                          F2 (&v)[NSLOT][Elem<T>::P]) {
   constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
-  if (!edge) {
 #pragma unroll
-    for (int p = 0; p < NSLOT; ++p) {
-      const int k = k0 + step * p;
-      if (k < g.nch) {
-        Elem<T>::unpack(load_stream(g.x_al + (long long)k * V), v[p]);
-      } else {
+  for (int p = 0; p < NSLOT; ++p) {
+    const int f = k0 + step * p;
+    if (f < g.nfull) {
+      Elem<T>::unpack(load_stream(g.x_full + (long long)f * V), v[p]);
+    } else {
 #pragma unroll
-        for (int j = 0; j < P; ++j) v[p][j] = zero2();
-      }
+      for (int j = 0; j < P; ++j) v[p][j] = zero2();
     }
-  } else {
-#pragma unroll
-    for (int p = 0; p < NSLOT; ++p) load_chunk<T, false>(g, D, k0 + step * p, v[p]);
   }
 }
 
 // ---------------------------------------------------------------------------
-// per-thread partial sums over the slots of one row
+// per-thread partial sums over the slots and the edge element of one row
+//
+// Each is (sum over the even positions) + (sum over the odd positions) of
+// the thread's slots, then, for a thread that owns an edge element, that
+// element's term added (a square by one fused multiply-add).
 
-// RMSNorm: sum of squares (absent columns hold zeros, which add nothing).
-template <typename T, int NSLOT>
-__device__ __forceinline__ float sum_squares(const F2 (&v)[NSLOT][Elem<T>::P]) {
+// RMSNorm: sum of squares (absent slots hold zeros, which add nothing).
+template <typename T, bool EXACT, int NSLOT>
+__device__ __forceinline__ float sum_squares(const F2 (&v)[NSLOT][Elem<T>::P], float xe,
+                                             bool has_edge) {
   constexpr int P = Elem<T>::P;
   F2 acc = zero2();
 #pragma unroll
   for (int p = 0; p < NSLOT; ++p)
 #pragma unroll
     for (int j = 0; j < P; ++j) acc = fma2(v[p][j], v[p][j], acc);
-  return hsum2(acc);
+  float s = hsum2(acc);
+  if (!EXACT && has_edge) s = __fmaf_rn(xe, xe, s);
+  return s;
 }
 
-// LayerNorm pass 1: replaces x by d = x - K (zero outside the row) and
+// LayerNorm pass 1: replaces x by d = x - K (slots and edge element) and
 // returns the thread's sum of d.
 template <typename T, bool EXACT, int NSLOT>
-__device__ __forceinline__ float shift_and_sum(F2 (&v)[NSLOT][Elem<T>::P], const Row<T>& g,
-                                               int D, int k0, int step, float K, bool edge) {
-  constexpr int V = Elem<T>::V;
+__device__ __forceinline__ float shift_and_sum(F2 (&v)[NSLOT][Elem<T>::P], float& xe,
+                                               const Row<T>& g, int k0, int step, float K,
+                                               bool has_edge) {
   constexpr int P = Elem<T>::P;
   const F2 K2 = splat(K);
   F2 acc = zero2();
-  if (!edge) {
 #pragma unroll
-    for (int p = 0; p < NSLOT; ++p) {
-      if (k0 + step * p < g.nch) {
-#pragma unroll
-        for (int j = 0; j < P; ++j) {
-          v[p][j] = sub2(v[p][j], K2);
-          acc = add2(acc, v[p][j]);
-        }
-      }
-    }
-  } else {
-#pragma unroll
-    for (int p = 0; p < NSLOT; ++p) {
-      const int k = k0 + step * p;
+  for (int p = 0; p < NSLOT; ++p) {
+    if (k0 + step * p < g.nfull) {
 #pragma unroll
       for (int j = 0; j < P; ++j) {
-        const int c = k * V + 2 * j - g.phase;
-        v[p][j] = mask2(sub2(v[p][j], K2), (unsigned)c < (unsigned)D,
-                        (unsigned)(c + 1) < (unsigned)D);
+        v[p][j] = sub2(v[p][j], K2);
         acc = add2(acc, v[p][j]);
       }
     }
   }
-  return hsum2(acc);
+  float s = hsum2(acc);
+  if (!EXACT && has_edge) {
+    xe = __fsub_rn(xe, K);
+    s = __fadd_rn(s, xe);
+  }
+  return s;
 }
 
-// LayerNorm pass 2: the thread's sum of (d - mean)^2 over the row's columns.
+// LayerNorm pass 2: the thread's sum of (d - mean)^2.
 template <typename T, bool EXACT, int NSLOT>
-__device__ __forceinline__ float sum_dev_squares(const F2 (&v)[NSLOT][Elem<T>::P],
-                                                 const Row<T>& g, int D, int k0, int step,
-                                                 float mean, bool edge) {
-  constexpr int V = Elem<T>::V;
+__device__ __forceinline__ float sum_dev_squares(const F2 (&v)[NSLOT][Elem<T>::P], float xe,
+                                                 const Row<T>& g, int k0, int step, float mean,
+                                                 bool has_edge) {
   constexpr int P = Elem<T>::P;
   const F2 M2 = splat(mean);
   F2 acc = zero2();
-  if (!edge) {
 #pragma unroll
-    for (int p = 0; p < NSLOT; ++p) {
-      if (k0 + step * p < g.nch) {
-#pragma unroll
-        for (int j = 0; j < P; ++j) {
-          const F2 t = sub2(v[p][j], M2);
-          acc = fma2(t, t, acc);
-        }
-      }
-    }
-  } else {
-#pragma unroll
-    for (int p = 0; p < NSLOT; ++p) {
-      const int k = k0 + step * p;
+  for (int p = 0; p < NSLOT; ++p) {
+    if (k0 + step * p < g.nfull) {
 #pragma unroll
       for (int j = 0; j < P; ++j) {
-        const int c = k * V + 2 * j - g.phase;
-        const F2 t = mask2(sub2(v[p][j], M2), (unsigned)c < (unsigned)D,
-                           (unsigned)(c + 1) < (unsigned)D);
+        const F2 t = sub2(v[p][j], M2);
         acc = fma2(t, t, acc);
       }
     }
   }
-  return hsum2(acc);
+  float s = hsum2(acc);
+  if (!EXACT && has_edge) {
+    const float t = __fsub_rn(xe, mean);
+    s = __fmaf_rn(t, t, s);
+  }
+  return s;
 }
 
 // ---------------------------------------------------------------------------
@@ -437,59 +409,68 @@ __device__ __forceinline__ float block_sum(float x, float* red) {
 // ---------------------------------------------------------------------------
 // weight and bias
 
-// EXACT rows: the weight/bias columns of chunk k are one aligned 16-byte
-// chunk of each vector (L1-resident after the first row).
+// EXACT rows: the weight/bias columns of chunk f are one aligned 16-byte
+// chunk of each vector (L1-resident after the first row). EXACT rows have
+// no edge elements.
 template <typename T, bool BIAS>
 struct AffineDirect {
   const T* w;
   const T* b;
-  __device__ __forceinline__ void get(int /*p*/, int k, F2 (&wf)[Elem<T>::P],
+  __device__ __forceinline__ void get(int /*p*/, int f, F2 (&wf)[Elem<T>::P],
                                       F2 (&bf)[Elem<T>::P]) const {
     constexpr int V = Elem<T>::V;
     constexpr int P = Elem<T>::P;
     if (w) {
-      Elem<T>::unpack(load_cached(w + k * V), wf);
+      Elem<T>::unpack(load_cached(w + f * V), wf);
     } else {
 #pragma unroll
       for (int j = 0; j < P; ++j) wf[j] = splat(1.f);
     }
     if constexpr (BIAS) {
       if (b) {
-        Elem<T>::unpack(load_cached(b + k * V), bf);
+        Elem<T>::unpack(load_cached(b + f * V), bf);
       } else {
 #pragma unroll
         for (int j = 0; j < P; ++j) bf[j] = zero2();
       }
     }
   }
+  __device__ __forceinline__ void edge(float& w_, float& b_) const {
+    w_ = 1.f;
+    b_ = 0.f;
+  }
 };
 
 // Any layout: the weight/bias columns of each of the thread's slots,
 // realigned to the row phase, in the thread's own shared memory entries
 // [slot][thread] (no other thread touches them, so no barrier; consecutive
-// threads use consecutive 16-byte words, so no bank conflicts). Refilled
-// when a row with another phase arrives. NULL weight = ones, NULL bias =
-// zeros.
+// threads use consecutive 16-byte words, so no bank conflicts), and those of
+// its edge element in registers. Refilled when a row with another phase
+// arrives (the split of a row into edge elements and chunks depends only on
+// D and the phase). NULL weight = ones, NULL bias = zeros.
 template <typename T, int NSLOT, bool BIAS>
 struct AffineCache {
   uint4* w;  // [NSLOT][blockDim.x]
   uint4* b;  // [NSLOT][blockDim.x] (BIAS)
+  float we, be;
   int phase;
 
   __device__ __forceinline__ void init(unsigned char* smem) {
     w = reinterpret_cast<uint4*>(smem);
     b = w + NSLOT * blockDim.x;
+    we = 1.f;
+    be = 0.f;
     phase = -1;
   }
 
-  __device__ __forceinline__ void fill(const Segment& s, int row_phase, int k0, int step) {
+  __device__ __forceinline__ void fill(const Segment& s, const Row<T>& g, int k0, int step) {
     constexpr int V = Elem<T>::V;
     const T* wv = static_cast<const T*>(s.w);
     const T* bv = static_cast<const T*>(s.b);
     const int D = s.dim;
 #pragma unroll 1
     for (int p = 0; p < NSLOT; ++p) {
-      const int c0 = (k0 + step * p) * V - row_phase;
+      const int c0 = g.head + (k0 + step * p) * V;
       uint32_t e[V];
 #pragma unroll
       for (int i = 0; i < V; ++i) {
@@ -506,13 +487,22 @@ struct AffineCache {
         b[p * blockDim.x + threadIdx.x] = Elem<T>::assemble(e);
       }
     }
-    phase = row_phase;
+    if (k0 < g.nedge) {
+      const int c = edge_column(g, D, k0);
+      we = wv ? Elem<T>::get(wv + c) : 1.f;
+      be = (BIAS && bv) ? Elem<T>::get(bv + c) : 0.f;
+    }
+    phase = g.phase;
   }
 
-  __device__ __forceinline__ void get(int p, int /*k*/, F2 (&wf)[Elem<T>::P],
+  __device__ __forceinline__ void get(int p, int /*f*/, F2 (&wf)[Elem<T>::P],
                                       F2 (&bf)[Elem<T>::P]) const {
     Elem<T>::unpack(w[p * blockDim.x + threadIdx.x], wf);
     if constexpr (BIAS) Elem<T>::unpack(b[p * blockDim.x + threadIdx.x], bf);
+  }
+  __device__ __forceinline__ void edge(float& w_, float& b_) const {
+    w_ = we;
+    b_ = be;
   }
 };
 
@@ -521,23 +511,23 @@ constexpr int affine_cache_bytes(int threads) {
   return threads * NSLOT * 16 * (BIAS ? 2 : 1);
 }
 
-// Normalize the thread's chunks of one row, apply weight (and bias), store.
+// Normalize the thread's chunks and edge element of one row, apply weight
+// (and bias), store.
 template <typename T, int OP, bool EXACT, int NSLOT, typename Src>
 __device__ __forceinline__ void normalize_store(const Segment& s, const Row<T>& g,
-                                                const F2 (&v)[NSLOT][Elem<T>::P],
+                                                const F2 (&v)[NSLOT][Elem<T>::P], float xe,
                                                 const Src& src, int k0, int step, float rstd,
-                                                float mean, bool edge) {
+                                                float mean, bool has_edge) {
   constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
-  const int D = s.dim;
   const F2 R2 = splat(rstd);
   const F2 M2 = splat(mean);
 #pragma unroll
   for (int p = 0; p < NSLOT; ++p) {
-    const int k = k0 + step * p;
-    if (k >= g.nch) continue;
+    const int f = k0 + step * p;
+    if (f >= g.nfull) continue;
     F2 wf[P], bf[P], o[P];
-    src.get(p, k, wf, bf);
+    src.get(p, f, wf, bf);
 #pragma unroll
     for (int j = 0; j < P; ++j) {
       if constexpr (OP == kOpRms)
@@ -545,38 +535,48 @@ __device__ __forceinline__ void normalize_store(const Segment& s, const Row<T>& 
       else
         o[j] = fma2(mul2(sub2(v[p][j], M2), R2), wf[j], bf[j]);
     }
-    if (EXACT || (s.vector_y && (!edge || chunk_full<T, EXACT>(g, k)))) {
-      store_stream(g.y_row - g.phase + (long long)k * V, Elem<T>::pack(o));
+    T* yc = g.y_row + g.head + (long long)f * V;
+    if (EXACT || s.vector_y) {
+      store_stream(yc, Elem<T>::pack(o));
     } else {
 #pragma unroll
       for (int j = 0; j < P; ++j) {
-        const int c = k * V + 2 * j - g.phase;
         float lo, hi;
         split2(o[j], lo, hi);
-        if ((unsigned)c < (unsigned)D) Elem<T>::put(g.y_row + c, lo);
-        if ((unsigned)(c + 1) < (unsigned)D) Elem<T>::put(g.y_row + c + 1, hi);
+        Elem<T>::put(yc + 2 * j, lo);
+        Elem<T>::put(yc + 2 * j + 1, hi);
       }
     }
   }
+  if (!EXACT && has_edge) {
+    float we, be;
+    src.edge(we, be);
+    const float o = OP == kOpRms
+                        ? __fmul_rn(__fmul_rn(xe, rstd), we)
+                        : __fmaf_rn(__fmul_rn(__fsub_rn(xe, mean), rstd), we, be);
+    Elem<T>::put(g.y_row + edge_column(g, s.dim, k0), o);
+  }
 }
 
-// rstd (and mean) of one row from the thread's slots, with `reduce` summing
-// a per-thread partial over the threads of the row.
+// rstd (and mean) of one row from the thread's slots and edge element, with
+// `reduce` summing a per-thread partial over the threads of the row.
 template <typename T, int OP, bool EXACT, int NSLOT, typename Reduce>
-__device__ __forceinline__ void row_stats(F2 (&v)[NSLOT][Elem<T>::P], const Row<T>& g,
-                                          int D, int k0, int step, float K, float eps,
-                                          bool edge, Reduce reduce, float& rstd, float& mean) {
+__device__ __forceinline__ void row_stats(F2 (&v)[NSLOT][Elem<T>::P], float& xe,
+                                          const Row<T>& g, int D, int k0, int step, float K,
+                                          float eps, bool has_edge, Reduce reduce, float& rstd,
+                                          float& mean) {
   // Means are sums times 1/D rounded to binary32 (one multiply instead of a
   // divide per row; exact for power-of-two D, within 2 ulps otherwise).
   const float inv_d = __frcp_rn((float)D);
   if (OP == kOpRms) {
-    const float ss = reduce(sum_squares<T, NSLOT>(v));
+    const float ss = reduce(sum_squares<T, EXACT, NSLOT>(v, xe, has_edge));
     mean = 0.f;
     rstd = rsqrtf(__fadd_rn(__fmul_rn(ss, inv_d), eps));
   } else {
-    const float s1 = reduce(shift_and_sum<T, EXACT, NSLOT>(v, g, D, k0, step, K, edge));
+    const float s1 = reduce(shift_and_sum<T, EXACT, NSLOT>(v, xe, g, k0, step, K, has_edge));
     mean = __fmul_rn(s1, inv_d);
-    const float s2 = reduce(sum_dev_squares<T, EXACT, NSLOT>(v, g, D, k0, step, mean, edge));
+    const float s2 =
+        reduce(sum_dev_squares<T, EXACT, NSLOT>(v, xe, g, k0, step, mean, has_edge));
     rstd = rsqrtf(__fadd_rn(__fmul_rn(s2, inv_d), eps));
   }
 }

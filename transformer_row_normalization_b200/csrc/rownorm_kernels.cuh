@@ -15,12 +15,13 @@
 // grid is a multiple of the phase period), so the realigned weight/bias
 // cache of non-aligned layouts is filled once.
 //
-// Prefetch. While a thread normalizes row r, its chunks of its next row are
-// already on their way: each thread copies its own full chunks of row
+// Prefetch. While a thread normalizes row r, its share of its next row is
+// already on its way: each thread copies its own full chunks of row
 // r + stride into its own shared memory slots with cp.async and waits only
 // for its own copies (cp.async.wait_group), so the HBM latency of a row hides
 // behind the previous row's arithmetic without any barrier. The shift K of
-// the next row (LayerNorm) is loaded at the same time.
+// the next row (LayerNorm) and the thread's edge element of it are loaded
+// into registers at the same time.
 //
 // The bulk-copy staged kernels (rownorm_staged.cuh) run the same per-row
 // code; which kernel the planner picks never changes a bit.
@@ -59,33 +60,27 @@ struct Prefetch {
     return base + ((stage * NSLOT + p) * blockDim.x + threadIdx.x);
   }
   // Start the copies of the thread's full chunks of row g into `stage`.
-  template <bool EXACT>
   __device__ __forceinline__ void issue(const Row<T>& g, int k0, int step, int stage) const {
     constexpr int V = Elem<T>::V;
     if (!on) return;
 #pragma unroll
     for (int p = 0; p < NSLOT; ++p) {
-      const int k = k0 + step * p;
-      if (chunk_full<T, EXACT>(g, k)) cp_async16(slot(stage, p), g.x_al + (long long)k * V);
+      const int f = k0 + step * p;
+      if (f < g.nfull) cp_async16(slot(stage, p), g.x_full + (long long)f * V);
     }
   }
-  // The thread's slots of row g: full chunks from `stage` (copies complete),
-  // partial chunks element by element from global memory, absent ones zero.
-  template <bool EXACT>
-  __device__ __forceinline__ void take(const Row<T>& g, int D, int k0, int step, int stage,
-                                       bool edge, F2 (&v)[NSLOT][Elem<T>::P]) const {
+  // The thread's slots of row g from `stage` (copies complete); absent ones zero.
+  __device__ __forceinline__ void take(const Row<T>& g, int k0, int step, int stage,
+                                       F2 (&v)[NSLOT][Elem<T>::P]) const {
     constexpr int P = Elem<T>::P;
     if (!on) {
-      load_row<T, EXACT, NSLOT>(g, D, k0, step, edge, v);
+      load_row<T, NSLOT>(g, k0, step, v);
       return;
     }
 #pragma unroll
     for (int p = 0; p < NSLOT; ++p) {
-      const int k = k0 + step * p;
-      if (k < g.nch && (!edge || chunk_full<T, EXACT>(g, k))) {
+      if (k0 + step * p < g.nfull) {
         Elem<T>::unpack(*slot(stage, p), v[p]);
-      } else if (edge) {
-        load_chunk<T, false>(g, D, k, v[p]);
       } else {
 #pragma unroll
         for (int j = 0; j < P; ++j) v[p][j] = zero2();
@@ -119,7 +114,6 @@ rows_warp_kernel(const Params p) {
     const unsigned mask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << (gi * G));
     const long long ngroups = nwarps * per_warp;
     const int D = s.dim;
-    const T* x = static_cast<const T*>(s.x);
     AffineCache<T, VPL, BIAS> cache;
     if constexpr (!EXACT)
       cache.init(smem + (p.prefetch ? prefetch_smem_bytes<VPL>(kWarpBlock) : 0));
@@ -127,35 +121,38 @@ rows_warp_kernel(const Params p) {
     auto reduce = [&](float t) { return group_sum(t, G, mask); };
     long long r = warp * per_warp + gi;
     Row<T> gn;
-    float Kn = 0.f;
+    float Kn = 0.f, En = 0.f;
     if (r < s.rows) {
       gn = row_geometry<T, EXACT>(s, r);
-      pf.template issue<EXACT>(gn, gl, G, 0);
-      if (OP == kOpLn) Kn = Elem<T>::get(x + r * s.x_stride);
+      pf.issue(gn, gl, G, 0);
+      if (OP == kOpLn) Kn = Elem<T>::get(gn.x_row);
+      En = load_edge<T, EXACT>(gn, D, gl);
     }
     cp_async_commit();
 #pragma unroll 1
     for (int i = 0; r < s.rows; ++i, r += ngroups) {
       const Row<T> g = gn;
       const float K = Kn;
+      float xe = En;
       const long long rn = r + ngroups;
       if (rn < s.rows) {
         gn = row_geometry<T, EXACT>(s, rn);
-        pf.template issue<EXACT>(gn, gl, G, (i + 1) & 1);
-        if (OP == kOpLn) Kn = Elem<T>::get(x + rn * s.x_stride);
+        pf.issue(gn, gl, G, (i + 1) & 1);
+        if (OP == kOpLn) Kn = Elem<T>::get(gn.x_row);
+        En = load_edge<T, EXACT>(gn, D, gl);
       }
       cp_async_commit();
       cp_async_wait<1>();
-      const bool edge = owns_partial<T, EXACT>(g, gl, G);
+      const bool has_edge = !EXACT && gl < g.nedge;
       F2 v[VPL][P];
-      pf.template take<EXACT>(g, D, gl, G, i & 1, edge, v);
+      pf.take(g, gl, G, i & 1, v);
       float rstd, mean;
-      row_stats<T, OP, EXACT, VPL>(v, g, D, gl, G, K, p.eps, edge, reduce, rstd, mean);
+      row_stats<T, OP, EXACT, VPL>(v, xe, g, D, gl, G, K, p.eps, has_edge, reduce, rstd, mean);
       if constexpr (EXACT) {
-        normalize_store<T, OP, EXACT, VPL>(s, g, v, direct, gl, G, rstd, mean, edge);
+        normalize_store<T, OP, EXACT, VPL>(s, g, v, xe, direct, gl, G, rstd, mean, has_edge);
       } else {
-        if (g.phase != cache.phase) cache.fill(s, g.phase, gl, G);
-        normalize_store<T, OP, EXACT, VPL>(s, g, v, cache, gl, G, rstd, mean, edge);
+        if (g.phase != cache.phase) cache.fill(s, g, gl, G);
+        normalize_store<T, OP, EXACT, VPL>(s, g, v, xe, cache, gl, G, rstd, mean, has_edge);
       }
     }
     cp_async_wait<0>();
@@ -166,6 +163,7 @@ template <typename T, int OP, bool EXACT, int NT, int VPT>
 __global__ void __launch_bounds__(NT, kMinThreadsPerSm / NT)
 rows_cta_kernel(const Params p) {
   constexpr int P = Elem<T>::P;
+  static_assert(NT >= 2 * (Elem<T>::V - 1), "every edge element needs its own thread");
   constexpr bool BIAS = OP == kOpLn;
   // Two alternating reduction buffers: a buffer is rewritten only after every
   // thread has passed the barrier of the reduction in between.
@@ -183,41 +181,43 @@ rows_cta_kernel(const Params p) {
   for (int si = 0; si < p.nseg; ++si) {
     const Segment s = pick_segment(p.seg, si);
     const int D = s.dim;
-    const T* x = static_cast<const T*>(s.x);
     AffineCache<T, VPT, BIAS> cache;
     if constexpr (!EXACT) cache.init(smem + (p.prefetch ? prefetch_smem_bytes<VPT>(NT) : 0));
     const AffineDirect<T, BIAS> direct{static_cast<const T*>(s.w), static_cast<const T*>(s.b)};
     long long r = blockIdx.x;
     Row<T> gn;
-    float Kn = 0.f;
+    float Kn = 0.f, En = 0.f;
     if (r < s.rows) {
       gn = row_geometry<T, EXACT>(s, r);
-      pf.template issue<EXACT>(gn, tid, NT, 0);
-      if (OP == kOpLn) Kn = Elem<T>::get(x + r * s.x_stride);
+      pf.issue(gn, tid, NT, 0);
+      if (OP == kOpLn) Kn = Elem<T>::get(gn.x_row);
+      En = load_edge<T, EXACT>(gn, D, tid);
     }
     cp_async_commit();
 #pragma unroll 1
     for (int i = 0; r < s.rows; ++i, r += gridDim.x) {
       const Row<T> g = gn;
       const float K = Kn;
+      float xe = En;
       const long long rn = r + gridDim.x;
       if (rn < s.rows) {
         gn = row_geometry<T, EXACT>(s, rn);
-        pf.template issue<EXACT>(gn, tid, NT, (i + 1) & 1);
-        if (OP == kOpLn) Kn = Elem<T>::get(x + rn * s.x_stride);
+        pf.issue(gn, tid, NT, (i + 1) & 1);
+        if (OP == kOpLn) Kn = Elem<T>::get(gn.x_row);
+        En = load_edge<T, EXACT>(gn, D, tid);
       }
       cp_async_commit();
       cp_async_wait<1>();
-      const bool edge = owns_partial<T, EXACT>(g, tid, NT);
+      const bool has_edge = !EXACT && tid < g.nedge;
       F2 v[VPT][P];
-      pf.template take<EXACT>(g, D, tid, NT, i & 1, edge, v);
+      pf.take(g, tid, NT, i & 1, v);
       float rstd, mean;
-      row_stats<T, OP, EXACT, VPT>(v, g, D, tid, NT, K, p.eps, edge, reduce, rstd, mean);
+      row_stats<T, OP, EXACT, VPT>(v, xe, g, D, tid, NT, K, p.eps, has_edge, reduce, rstd, mean);
       if constexpr (EXACT) {
-        normalize_store<T, OP, EXACT, VPT>(s, g, v, direct, tid, NT, rstd, mean, edge);
+        normalize_store<T, OP, EXACT, VPT>(s, g, v, xe, direct, tid, NT, rstd, mean, has_edge);
       } else {
-        if (g.phase != cache.phase) cache.fill(s, g.phase, tid, NT);
-        normalize_store<T, OP, EXACT, VPT>(s, g, v, cache, tid, NT, rstd, mean, edge);
+        if (g.phase != cache.phase) cache.fill(s, g, tid, NT);
+        normalize_store<T, OP, EXACT, VPT>(s, g, v, xe, cache, tid, NT, rstd, mean, has_edge);
       }
     }
     cp_async_wait<0>();

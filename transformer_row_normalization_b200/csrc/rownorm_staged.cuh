@@ -17,9 +17,9 @@
 //
 // Tiles. NARROW (lane groups; EXACT layouts only): a tile is TR consecutive
 // rows, moved as one bulk copy when they are adjacent in memory, otherwise
-// one copy per row. WIDE (one block per row): a tile is one row; its
-// 16-byte-aligned interior moves as one bulk copy and the at most two
-// partial chunks at its ends are read element by element from global memory.
+// one copy per row. WIDE (one block per row): a tile is one row; its full
+// 16-byte chunks move as one bulk copy and its edge elements are read one by
+// one from global memory by their owners.
 //
 // Waits are bounded: a thread waiting for a stage gives up after
 // kWaitLimitNs, the block leaves its loop together (the decision is taken
@@ -124,14 +124,10 @@ __device__ __forceinline__ void issue_tile(const StagedParams& p, long long mine
   locate_tile(mine0, i, si, tile);
   const Segment& s = p.seg[si];
   if constexpr (WIDE) {
-    const T* xr = static_cast<const T*>(s.x) + tile * s.x_stride;
-    const int phase = (int)((reinterpret_cast<uintptr_t>(xr) & 15u) / sizeof(T));
-    const int first = phase ? 1 : 0;  // first full chunk
-    const int nch = (phase + s.dim + V - 1) / V;
-    const int last = ((phase + s.dim) % V == 0) ? nch : nch - 1;  // one past the last full
-    const uint32_t bytes = (uint32_t)(last - first) * 16u;
+    const Row<T> g = row_geometry<T, false>(s, tile);
+    const uint32_t bytes = (uint32_t)g.nfull * 16u;
     mbar_expect_tx(bar, bytes);
-    if (bytes) bulk_load(dst, xr - phase + first * V, bytes, bar);
+    if (bytes) bulk_load(dst, g.x_full, bytes, bar);
   } else {
     const long long r0 = tile * p.tile_rows[si];
     long long nr = s.rows - r0;
@@ -148,31 +144,13 @@ __device__ __forceinline__ void issue_tile(const StagedParams& p, long long mine
   }
 }
 
-// Chunk k of a WIDE row: full chunks from the stage (which holds the row's
-// interior, starting at its first full chunk), the partial chunks at the row
-// ends element by element from global memory.
-template <typename T, bool EXACT>
-__device__ __forceinline__ void stage_chunk(const Row<T>& g, const unsigned char* stage, int D,
-                                            int k, F2 (&f)[Elem<T>::P]) {
-  constexpr int V = Elem<T>::V;
-  constexpr int P = Elem<T>::P;
-  if (chunk_full<T, EXACT>(g, k)) {
-    const int j = k - (g.phase ? 1 : 0);
-    Elem<T>::unpack(*reinterpret_cast<const uint4*>(stage + 16 * j), f);
-  } else if constexpr (EXACT) {
-#pragma unroll
-    for (int q = 0; q < P; ++q) f[q] = zero2();
-  } else {
-    load_chunk<T, false>(g, D, k, f);
-  }
-}
-
 template <typename T, int OP, bool WIDE, bool EXACT, int NT, int VPT>
 __global__ void __launch_bounds__(NT, (NT >= 1024 ? 1 : 1024 / NT))
 rows_staged_kernel(const StagedParams p) {
   constexpr int P = Elem<T>::P;
   constexpr bool BIAS = OP == kOpLn;
   static_assert(WIDE || EXACT, "lane-group rows are staged only for 16-byte aligned layouts");
+  static_assert(!WIDE || NT >= 2 * (Elem<T>::V - 1), "every edge element needs its own thread");
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ __align__(8) uint64_t full[kMaxStagesDevice];
   __shared__ float red[2][NT / 32];
@@ -234,19 +212,29 @@ rows_staged_kernel(const StagedParams p) {
       const Row<T> g = row_geometry<T, EXACT>(s, tile);
       F2 v[VPT][P];
 #pragma unroll
-      for (int q = 0; q < VPT; ++q) stage_chunk<T, EXACT>(g, stage, D, tid + NT * q, v[q]);
+      for (int q = 0; q < VPT; ++q) {
+        const int f = tid + NT * q;
+        if (f < g.nfull) {
+          Elem<T>::unpack(*reinterpret_cast<const uint4*>(stage + 16 * f), v[q]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < P; ++j) v[q][j] = zero2();
+        }
+      }
       float K = 0.f;
       if (OP == kOpLn)
-        K = g.phase ? Elem<T>::get(g.x_al + g.phase)
-                    : Elem<T>::get(reinterpret_cast<const T*>(stage));
-      const bool edge = owns_partial<T, EXACT>(g, tid, NT);
+        K = (g.head || !g.nfull) ? Elem<T>::get(g.x_row)
+                                 : Elem<T>::get(reinterpret_cast<const T*>(stage));
+      const bool has_edge = !EXACT && tid < g.nedge;
+      float xe = load_edge<T, EXACT>(g, D, tid);
       float rstd, mean;
-      row_stats<T, OP, EXACT, VPT>(v, g, D, tid, NT, K, p.eps, edge, block_reduce, rstd, mean);
+      row_stats<T, OP, EXACT, VPT>(v, xe, g, D, tid, NT, K, p.eps, has_edge, block_reduce, rstd,
+                                   mean);
       if constexpr (EXACT) {
-        normalize_store<T, OP, EXACT, VPT>(s, g, v, direct, tid, NT, rstd, mean, edge);
+        normalize_store<T, OP, EXACT, VPT>(s, g, v, xe, direct, tid, NT, rstd, mean, has_edge);
       } else {
-        if (g.phase != cache.phase) cache.fill(s, g.phase, tid, NT);
-        normalize_store<T, OP, EXACT, VPT>(s, g, v, cache, tid, NT, rstd, mean, edge);
+        if (g.phase != cache.phase) cache.fill(s, g, tid, NT);
+        normalize_store<T, OP, EXACT, VPT>(s, g, v, xe, cache, tid, NT, rstd, mean, has_edge);
       }
     } else {
       const int G = s.lanes;
@@ -269,18 +257,19 @@ rows_staged_kernel(const StagedParams p) {
         F2 v[VPT][P];
 #pragma unroll
         for (int q = 0; q < VPT; ++q) {
-          const int k = gl + G * q;
-          if (k < g.nch) {
-            Elem<T>::unpack(*reinterpret_cast<const uint4*>(row + 16 * k), v[q]);
+          const int f = gl + G * q;
+          if (f < g.nfull) {
+            Elem<T>::unpack(*reinterpret_cast<const uint4*>(row + 16 * f), v[q]);
           } else {
 #pragma unroll
             for (int j = 0; j < P; ++j) v[q][j] = zero2();
           }
         }
         const float K = OP == kOpLn ? Elem<T>::get(reinterpret_cast<const T*>(row)) : 0.f;
-        float rstd, mean;
-        row_stats<T, OP, true, VPT>(v, g, D, gl, G, K, p.eps, false, group_reduce, rstd, mean);
-        normalize_store<T, OP, true, VPT>(s, g, v, direct, gl, G, rstd, mean, false);
+        float xe = 0.f, rstd, mean;
+        row_stats<T, OP, true, VPT>(v, xe, g, D, gl, G, K, p.eps, false, group_reduce, rstd,
+                                    mean);
+        normalize_store<T, OP, true, VPT>(s, g, v, xe, direct, gl, G, rstd, mean, false);
       }
     }
   }
