@@ -72,45 +72,23 @@ struct Segment {
 // column), so the packed instructions take their operands without any
 // register shuffling.
 
-struct F2 {
-  unsigned long long v;
-};
+using F2 = float2;
 
-__device__ __forceinline__ F2 make2(float lo, float hi) {
-  F2 d;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(d.v) : "f"(lo), "f"(hi));
-  return d;
-}
+__device__ __forceinline__ F2 make2(float lo, float hi) { return make_float2(lo, hi); }
 __device__ __forceinline__ F2 make2_bits(uint32_t lo, uint32_t hi) {
-  F2 d;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(d.v) : "r"(lo), "r"(hi));
-  return d;
+  return make_float2(__uint_as_float(lo), __uint_as_float(hi));
 }
 __device__ __forceinline__ void split2(F2 a, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(a.v));
+  lo = a.x;
+  hi = a.y;
 }
-__device__ __forceinline__ F2 zero2() { return F2{0ull}; }
-__device__ __forceinline__ F2 splat(float v) { return make2(v, v); }
-__device__ __forceinline__ F2 add2(F2 a, F2 b) {
-  F2 d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d.v) : "l"(a.v), "l"(b.v));
-  return d;
-}
-__device__ __forceinline__ F2 sub2(F2 a, F2 b) {
-  F2 d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d.v) : "l"(a.v), "l"(b.v));
-  return d;
-}
-__device__ __forceinline__ F2 mul2(F2 a, F2 b) {
-  F2 d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d.v) : "l"(a.v), "l"(b.v));
-  return d;
-}
-__device__ __forceinline__ F2 fma2(F2 a, F2 b, F2 c) {
-  F2 d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d.v) : "l"(a.v), "l"(b.v), "l"(c.v));
-  return d;
-}
+__device__ __forceinline__ F2 zero2() { return make_float2(0.f, 0.f); }
+__device__ __forceinline__ F2 splat(float v) { return make_float2(v, v); }
+__device__ __forceinline__ F2 add2(F2 a, F2 b) { return __fadd2_rn(a, b); }
+// a - b is a + (-b): negation is exact and the sum rounds as the difference.
+__device__ __forceinline__ F2 sub2(F2 a, F2 b) { return __fadd2_rn(a, make_float2(-b.x, -b.y)); }
+__device__ __forceinline__ F2 mul2(F2 a, F2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ F2 fma2(F2 a, F2 b, F2 c) { return __ffma2_rn(a, b, c); }
 // lo + hi, rounded once.
 __device__ __forceinline__ float hsum2(F2 a) {
   float lo, hi;
@@ -139,10 +117,8 @@ struct Elem<float> {
     f[1] = make2_bits(u.z, u.w);
   }
   static __device__ __forceinline__ uint4 pack(const F2 (&f)[2]) {
-    uint4 u;
-    asm("mov.b64 {%0, %1}, %2;" : "=r"(u.x), "=r"(u.y) : "l"(f[0].v));
-    asm("mov.b64 {%0, %1}, %2;" : "=r"(u.z), "=r"(u.w) : "l"(f[1].v));
-    return u;
+    return make_uint4(__float_as_uint(f[0].x), __float_as_uint(f[0].y), __float_as_uint(f[1].x),
+                      __float_as_uint(f[1].y));
   }
   static __device__ __forceinline__ uint4 assemble(const uint32_t (&e)[4]) {
     return make_uint4(e[0], e[1], e[2], e[3]);
@@ -191,6 +167,11 @@ struct Elem<__nv_bfloat16> {
 
 // ---------------------------------------------------------------------------
 // memory access
+
+// The block's dynamic shared memory (prefetch slots, weight/bias cache,
+// staged tiles), addressed by 16-byte word offsets so that the compiler uses
+// 32-bit shared-window addresses rather than generic pointers.
+extern __shared__ __align__(128) uint4 dyn_smem[];
 
 __device__ __forceinline__ uint4 load_stream(const void* p) {
   return __ldcs(reinterpret_cast<const uint4*>(p));
@@ -450,17 +431,21 @@ struct AffineDirect {
 // D and the phase). NULL weight = ones, NULL bias = zeros.
 template <typename T, int NSLOT, bool BIAS>
 struct AffineCache {
-  uint4* w;  // [NSLOT][blockDim.x]
-  uint4* b;  // [NSLOT][blockDim.x] (BIAS)
+  int base;  // first 16-byte word: weight [NSLOT][blockDim.x], then bias (BIAS)
   float we, be;
   int phase;
 
-  __device__ __forceinline__ void init(unsigned char* smem) {
-    w = reinterpret_cast<uint4*>(smem);
-    b = w + NSLOT * blockDim.x;
+  __device__ __forceinline__ void init(int word_offset) {
+    base = word_offset;
     we = 1.f;
     be = 0.f;
     phase = -1;
+  }
+  __device__ __forceinline__ uint4& wslot(int p) const {
+    return dyn_smem[base + p * blockDim.x + threadIdx.x];
+  }
+  __device__ __forceinline__ uint4& bslot(int p) const {
+    return dyn_smem[base + (NSLOT + p) * blockDim.x + threadIdx.x];
   }
 
   __device__ __forceinline__ void fill(const Segment& s, const Row<T>& g, int k0, int step) {
@@ -477,14 +462,14 @@ struct AffineCache {
         const int c = c0 + i;
         e[i] = (wv && (unsigned)c < (unsigned)D) ? Elem<T>::get_bits(wv + c) : Elem<T>::kOneBits;
       }
-      w[p * blockDim.x + threadIdx.x] = Elem<T>::assemble(e);
+      wslot(p) = Elem<T>::assemble(e);
       if constexpr (BIAS) {
 #pragma unroll
         for (int i = 0; i < V; ++i) {
           const int c = c0 + i;
           e[i] = (bv && (unsigned)c < (unsigned)D) ? Elem<T>::get_bits(bv + c) : 0u;
         }
-        b[p * blockDim.x + threadIdx.x] = Elem<T>::assemble(e);
+        bslot(p) = Elem<T>::assemble(e);
       }
     }
     if (k0 < g.nedge) {
@@ -497,8 +482,8 @@ struct AffineCache {
 
   __device__ __forceinline__ void get(int p, int /*f*/, F2 (&wf)[Elem<T>::P],
                                       F2 (&bf)[Elem<T>::P]) const {
-    Elem<T>::unpack(w[p * blockDim.x + threadIdx.x], wf);
-    if constexpr (BIAS) Elem<T>::unpack(b[p * blockDim.x + threadIdx.x], bf);
+    Elem<T>::unpack(wslot(p), wf);
+    if constexpr (BIAS) Elem<T>::unpack(bslot(p), bf);
   }
   __device__ __forceinline__ void edge(float& w_, float& b_) const {
     w_ = we;

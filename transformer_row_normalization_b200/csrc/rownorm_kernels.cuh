@@ -54,10 +54,9 @@ constexpr int kMinThreadsPerSm = 1024;
 // straight from global memory when they are taken.
 template <typename T, int NSLOT>
 struct Prefetch {
-  uint4* base;
   int on;
   __device__ __forceinline__ uint4* slot(int stage, int p) const {
-    return base + ((stage * NSLOT + p) * blockDim.x + threadIdx.x);
+    return &dyn_smem[(stage * NSLOT + p) * blockDim.x + threadIdx.x];
   }
   // Start the copies of the thread's full chunks of row g into `stage`.
   __device__ __forceinline__ void issue(const Row<T>& g, int k0, int step, int stage) const {
@@ -89,9 +88,10 @@ struct Prefetch {
   }
 };
 
+// 16-byte words of prefetch slots (two stages).
 template <int NSLOT>
-__host__ __device__ constexpr int prefetch_smem_bytes(int threads) {
-  return 2 * NSLOT * threads * 16;
+__host__ __device__ constexpr int prefetch_smem_words(int threads) {
+  return 2 * NSLOT * threads;
 }
 
 template <typename T, int OP, bool EXACT, int VPL>
@@ -99,8 +99,7 @@ __global__ void __launch_bounds__(kWarpBlock, kMinThreadsPerSmWarp / kWarpBlock)
 rows_warp_kernel(const Params p) {
   constexpr int P = Elem<T>::P;
   constexpr bool BIAS = OP == kOpLn;
-  extern __shared__ __align__(128) unsigned char smem[];
-  const Prefetch<T, VPL> pf{reinterpret_cast<uint4*>(smem), p.prefetch};
+  const Prefetch<T, VPL> pf{p.prefetch};
   const int lane = threadIdx.x & 31;
   const long long warp = (long long)blockIdx.x * (kWarpBlock / 32) + (threadIdx.x >> 5);
   const long long nwarps = (long long)gridDim.x * (kWarpBlock / 32);
@@ -116,14 +115,13 @@ rows_warp_kernel(const Params p) {
     const int D = s.dim;
     AffineCache<T, VPL, BIAS> cache;
     if constexpr (!EXACT)
-      cache.init(smem + (p.prefetch ? prefetch_smem_bytes<VPL>(kWarpBlock) : 0));
+      cache.init(p.prefetch ? prefetch_smem_words<VPL>(kWarpBlock) : 0);
     const AffineDirect<T, BIAS> direct{static_cast<const T*>(s.w), static_cast<const T*>(s.b)};
     auto reduce = [&](float t) { return group_sum(t, G, mask); };
     long long r = warp * per_warp + gi;
-    Row<T> gn;
     float Kn = 0.f, En = 0.f;
     if (r < s.rows) {
-      gn = row_geometry<T, EXACT>(s, r);
+      const Row<T> gn = row_geometry<T, EXACT>(s, r);
       pf.issue(gn, gl, G, 0);
       if (OP == kOpLn) Kn = Elem<T>::get(gn.x_row);
       En = load_edge<T, EXACT>(gn, D, gl);
@@ -131,18 +129,18 @@ rows_warp_kernel(const Params p) {
     cp_async_commit();
 #pragma unroll 1
     for (int i = 0; r < s.rows; ++i, r += ngroups) {
-      const Row<T> g = gn;
       const float K = Kn;
       float xe = En;
       const long long rn = r + ngroups;
       if (rn < s.rows) {
-        gn = row_geometry<T, EXACT>(s, rn);
+        const Row<T> gn = row_geometry<T, EXACT>(s, rn);
         pf.issue(gn, gl, G, (i + 1) & 1);
         if (OP == kOpLn) Kn = Elem<T>::get(gn.x_row);
         En = load_edge<T, EXACT>(gn, D, gl);
       }
       cp_async_commit();
       cp_async_wait<1>();
+      const Row<T> g = row_geometry<T, EXACT>(s, r);
       const bool has_edge = !EXACT && gl < g.nedge;
       F2 v[VPL][P];
       pf.take(g, gl, G, i & 1, v);
@@ -168,8 +166,7 @@ rows_cta_kernel(const Params p) {
   // Two alternating reduction buffers: a buffer is rewritten only after every
   // thread has passed the barrier of the reduction in between.
   __shared__ float red[2][NT / 32];
-  extern __shared__ __align__(128) unsigned char smem[];
-  const Prefetch<T, VPT> pf{reinterpret_cast<uint4*>(smem), p.prefetch};
+  const Prefetch<T, VPT> pf{p.prefetch};
   int slot = 0;
   const int tid = threadIdx.x;
   auto reduce = [&](float t) {
@@ -182,13 +179,12 @@ rows_cta_kernel(const Params p) {
     const Segment s = pick_segment(p.seg, si);
     const int D = s.dim;
     AffineCache<T, VPT, BIAS> cache;
-    if constexpr (!EXACT) cache.init(smem + (p.prefetch ? prefetch_smem_bytes<VPT>(NT) : 0));
+    if constexpr (!EXACT) cache.init(p.prefetch ? prefetch_smem_words<VPT>(NT) : 0);
     const AffineDirect<T, BIAS> direct{static_cast<const T*>(s.w), static_cast<const T*>(s.b)};
     long long r = blockIdx.x;
-    Row<T> gn;
     float Kn = 0.f, En = 0.f;
     if (r < s.rows) {
-      gn = row_geometry<T, EXACT>(s, r);
+      const Row<T> gn = row_geometry<T, EXACT>(s, r);
       pf.issue(gn, tid, NT, 0);
       if (OP == kOpLn) Kn = Elem<T>::get(gn.x_row);
       En = load_edge<T, EXACT>(gn, D, tid);
@@ -196,18 +192,18 @@ rows_cta_kernel(const Params p) {
     cp_async_commit();
 #pragma unroll 1
     for (int i = 0; r < s.rows; ++i, r += gridDim.x) {
-      const Row<T> g = gn;
       const float K = Kn;
       float xe = En;
       const long long rn = r + gridDim.x;
       if (rn < s.rows) {
-        gn = row_geometry<T, EXACT>(s, rn);
+        const Row<T> gn = row_geometry<T, EXACT>(s, rn);
         pf.issue(gn, tid, NT, (i + 1) & 1);
         if (OP == kOpLn) Kn = Elem<T>::get(gn.x_row);
         En = load_edge<T, EXACT>(gn, D, tid);
       }
       cp_async_commit();
       cp_async_wait<1>();
+      const Row<T> g = row_geometry<T, EXACT>(s, r);
       const bool has_edge = !EXACT && tid < g.nedge;
       F2 v[VPT][P];
       pf.take(g, tid, NT, i & 1, v);

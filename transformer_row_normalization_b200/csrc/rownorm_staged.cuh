@@ -151,7 +151,7 @@ rows_staged_kernel(const StagedParams p) {
   constexpr bool BIAS = OP == kOpLn;
   static_assert(WIDE || EXACT, "lane-group rows are staged only for 16-byte aligned layouts");
   static_assert(!WIDE || NT >= 2 * (Elem<T>::V - 1), "every edge element needs its own thread");
-  extern __shared__ __align__(128) unsigned char smem[];
+  unsigned char* const smem = reinterpret_cast<unsigned char*>(dyn_smem);
   __shared__ __align__(8) uint64_t full[kMaxStagesDevice];
   __shared__ float red[2][NT / 32];
   const int tid = threadIdx.x;
@@ -179,7 +179,7 @@ rows_staged_kernel(const StagedParams p) {
   };
   int cur_seg = -1;
   AffineCache<T, VPT, BIAS> cache;
-  if constexpr (!EXACT) cache.init(smem + p.cache_offset);
+  if constexpr (!EXACT) cache.init(p.cache_offset / 16);
   bool aborted = false;
 #pragma unroll 1
   for (long long i = 0; i < n; ++i) {
