@@ -173,8 +173,11 @@ typedef struct rn_launch_info {
     int32_t vector_y;       /* 1: y rows share x's 16-byte phase (16-byte   */
                             /* stores); 0: y written element by element     */
     int32_t phase_period;   /* distinct 16-byte phases among x's rows       */
-    int32_t exact;          /* 1: every row of x and y starts 16-byte       */
-                            /* aligned and dim fills whole 16-byte chunks   */
+    int32_t exact;          /* layout class: 0 any; 1 every row of x and y, */
+                            /* the weight and the bias start 16-byte        */
+                            /* aligned and dim fills whole 16-byte chunks;  */
+                            /* 2 as 1, and those chunks divide evenly over  */
+                            /* the row's threads (no slot is ever empty)    */
     int32_t staged;         /* 1: rows stream through shared memory by bulk */
                             /* copies (S stages); 0: loaded into registers  */
     int32_t stages;         /* staged: stages per block                     */

@@ -124,3 +124,28 @@ def test_staged_plans_for_the_large_workloads():
             assert p["staged"] == 1 and p["stages"] >= 2, (dim, p)
     finally:
         rn.set_path_override(0)
+
+
+@pytest.mark.parametrize("dim,layout", [(128, 2), (768, 2), (1000, 1), (1024, 2), (4096, 2),
+                                        (4097, 0), (5120, 1), (8192, 2), (16384, 2)])
+def test_layout_class_of_the_planned_launch(dim, layout):
+    # 2: every thread owns all its chunk slots in every row (no slot tests);
+    # 1: aligned rows with a ragged last round of slots, or more than four
+    # chunks per thread; 0: rows off the 16-byte grid.
+    x = torch.empty(4096, dim, dtype=torch.bfloat16, device="cuda")
+    w = torch.ones(dim, dtype=torch.bfloat16, device="cuda")
+    assert rn.plan(rn.RN_OP_LN, x, weight=w, bias=w)["exact"] == layout
+
+
+@pytest.mark.parametrize("dtype,dim", [(torch.bfloat16, 768), (torch.bfloat16, 8192),
+                                       (torch.bfloat16, 1000), (torch.float32, 2048)])
+def test_null_vectors_match_explicit_ones_and_zeros(dtype, dim):
+    # A NULL weight (bias) is all ones (zeros). The kernels run separate row
+    # loops for present and absent vectors; both must give the same bits.
+    x = wl.random_rows(999, dim, dtype, seed=dim + 5, mean=0.5, std=2.0).cuda()
+    ones = torch.ones(dim, dtype=dtype, device="cuda")
+    zeros = torch.zeros(dim, dtype=dtype, device="cuda")
+    b = wl.random_vector(dim, dtype, seed=6, mean=0.0, std=0.1).cuda()
+    assert torch.equal(rn.rms_norm(x, None, 1e-6), rn.rms_norm(x, ones, 1e-6))
+    assert torch.equal(rn.layer_norm(x, None, None, 1e-5), rn.layer_norm(x, ones, zeros, 1e-5))
+    assert torch.equal(rn.layer_norm(x, None, b, 1e-5), rn.layer_norm(x, ones, b, 1e-5))

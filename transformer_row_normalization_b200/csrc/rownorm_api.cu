@@ -136,6 +136,7 @@ struct SegPlan {
   int vector_y;      // y rows share x's 16-byte phase
   int phase_period;  // distinct 16-byte phases among the rows of x
   int exact;         // every x and y row 16-byte aligned, dim % V == 0
+  int full;          // exact, and dim / V == lanes * chunks (no slot ever empty)
 };
 
 // The lane count / block size is a function of (dtype, dim) and, for lane
@@ -185,16 +186,21 @@ SegPlan plan_segment(const rn_view* x, const rn_view* y, const void* w, const vo
   p.exact = rows_aligned && ya % 16 == 0 &&
             (y->rows <= 1 || (y->row_stride * es) % 16 == 0) &&
             reinterpret_cast<uintptr_t>(w) % 16 == 0 && reinterpret_cast<uintptr_t>(b) % 16 == 0;
+  p.full = p.exact && nfull == (int64_t)p.lanes * p.chunks && p.chunks <= rn::kFullMaxChunks;
   return p;
 }
 
+int layout_of(const SegPlan& p) {
+  return p.full ? rn::kLayoutFull : (p.exact ? rn::kLayoutExact : rn::kLayoutAny);
+}
+
 const void* kernel_for(int dtype, int op, const SegPlan& p) {
-  const bool ex = p.exact != 0;
+  const int lay = layout_of(p);
   if (p.family == 0)
-    return dtype == RN_F32 ? rn::warp_kernel_f32(op, ex, p.chunks)
-                           : rn::warp_kernel_bf16(op, ex, p.chunks);
-  return dtype == RN_F32 ? rn::cta_kernel_f32(op, ex, p.lanes, p.chunks)
-                         : rn::cta_kernel_bf16(op, ex, p.lanes, p.chunks);
+    return dtype == RN_F32 ? rn::warp_kernel_f32(op, lay, p.chunks)
+                           : rn::warp_kernel_bf16(op, lay, p.chunks);
+  return dtype == RN_F32 ? rn::cta_kernel_f32(op, lay, p.lanes, p.chunks)
+                         : rn::cta_kernel_bf16(op, lay, p.lanes, p.chunks);
 }
 
 struct DeviceInfo {
@@ -389,8 +395,10 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
   int64_t rows[2] = {xs[0]->rows, nseg > 1 ? xs[1]->rows : 0};
   SegPlan merged = plans[0];
   for (int i = 1; i < nseg; ++i) {
+    if (plans[i].chunks != merged.chunks) merged.full = 0;  // a segment would leave slots empty
     if (plans[i].chunks > merged.chunks) merged.chunks = plans[i].chunks;
     merged.exact = merged.exact && plans[i].exact;
+    merged.full = merged.full && plans[i].full;
   }
   const void* fn = kernel_for(dtype, op, merged);
   if (!fn) return fail(RN_ERR_UNSUPPORTED, "no compiled kernel for this shape");
@@ -450,7 +458,7 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
   in.blocks_per_sm = bps;
   in.vector_y = plans[0].vector_y;
   in.phase_period = plans[0].phase_period;
-  in.exact = merged.exact;
+  in.exact = layout_of(merged);
   return RN_OK;
 }
 

@@ -50,6 +50,15 @@ namespace rn {
 
 enum : int { kOpRms = 0, kOpLn = 1 };
 
+// Layout classes of a launch (what the planner guarantees for every row):
+//   kLayoutAny    any 16-byte phase, any D, any weight/bias alignment;
+//   kLayoutExact  EXACT: x and y rows, weight and bias start on 16-byte
+//                 boundaries and D is a multiple of V (no edge elements);
+//   kLayoutFull   EXACT, and the row's D / V chunks divide evenly over the
+//                 threads of the row: every thread owns all its slots in
+//                 every row, so no slot is ever tested.
+enum : int { kLayoutAny = 0, kLayoutExact = 1, kLayoutFull = 2 };
+
 // One row space (a tensor viewed as [rows, dim]); strides in elements.
 struct Segment {
   const void* x;
@@ -262,7 +271,7 @@ __device__ __forceinline__ float load_edge(const Row<T>& g, int D, int k0) {
 }
 
 // All of a thread's slots of one row from global memory (absent ones zero).
-template <typename T, int NSLOT>
+template <typename T, bool FULL, int NSLOT>
 __device__ __forceinline__ void load_row(const Row<T>& g, int k0, int step,
                                          F2 (&v)[NSLOT][Elem<T>::P]) {
   constexpr int V = Elem<T>::V;
@@ -270,7 +279,7 @@ __device__ __forceinline__ void load_row(const Row<T>& g, int k0, int step,
 #pragma unroll
   for (int p = 0; p < NSLOT; ++p) {
     const int f = k0 + step * p;
-    if (f < g.nfull) {
+    if (FULL || f < g.nfull) {
       Elem<T>::unpack(load_stream(g.x_full + (long long)f * V), v[p]);
     } else {
 #pragma unroll
@@ -303,7 +312,7 @@ __device__ __forceinline__ float sum_squares(const F2 (&v)[NSLOT][Elem<T>::P], f
 
 // LayerNorm pass 1: replaces x by d = x - K (slots and edge element) and
 // returns the thread's sum of d.
-template <typename T, bool EXACT, int NSLOT>
+template <typename T, bool EXACT, bool FULL, int NSLOT>
 __device__ __forceinline__ float shift_and_sum(F2 (&v)[NSLOT][Elem<T>::P], float& xe,
                                                const Row<T>& g, int k0, int step, float K,
                                                bool has_edge) {
@@ -312,7 +321,7 @@ __device__ __forceinline__ float shift_and_sum(F2 (&v)[NSLOT][Elem<T>::P], float
   F2 acc = zero2();
 #pragma unroll
   for (int p = 0; p < NSLOT; ++p) {
-    if (k0 + step * p < g.nfull) {
+    if (FULL || k0 + step * p < g.nfull) {
 #pragma unroll
       for (int j = 0; j < P; ++j) {
         v[p][j] = sub2(v[p][j], K2);
@@ -329,7 +338,7 @@ __device__ __forceinline__ float shift_and_sum(F2 (&v)[NSLOT][Elem<T>::P], float
 }
 
 // LayerNorm pass 2: the thread's sum of (d - mean)^2.
-template <typename T, bool EXACT, int NSLOT>
+template <typename T, bool EXACT, bool FULL, int NSLOT>
 __device__ __forceinline__ float sum_dev_squares(const F2 (&v)[NSLOT][Elem<T>::P], float xe,
                                                  const Row<T>& g, int k0, int step, float mean,
                                                  bool has_edge) {
@@ -338,7 +347,7 @@ __device__ __forceinline__ float sum_dev_squares(const F2 (&v)[NSLOT][Elem<T>::P
   F2 acc = zero2();
 #pragma unroll
   for (int p = 0; p < NSLOT; ++p) {
-    if (k0 + step * p < g.nfull) {
+    if (FULL || k0 + step * p < g.nfull) {
 #pragma unroll
       for (int j = 0; j < P; ++j) {
         const F2 t = sub2(v[p][j], M2);
@@ -392,8 +401,9 @@ __device__ __forceinline__ float block_sum(float x, float* red) {
 
 // EXACT rows: the weight/bias columns of chunk f are one aligned 16-byte
 // chunk of each vector (L1-resident after the first row). EXACT rows have
-// no edge elements.
-template <typename T, bool BIAS>
+// no edge elements. AFF: the weight (and bias) are known to be present, so
+// no per-chunk test of a NULL vector remains in the row loop.
+template <typename T, bool BIAS, bool AFF>
 struct AffineDirect {
   const T* w;
   const T* b;
@@ -401,14 +411,14 @@ struct AffineDirect {
                                       F2 (&bf)[Elem<T>::P]) const {
     constexpr int V = Elem<T>::V;
     constexpr int P = Elem<T>::P;
-    if (w) {
+    if (AFF || w) {
       Elem<T>::unpack(load_cached(w + f * V), wf);
     } else {
 #pragma unroll
       for (int j = 0; j < P; ++j) wf[j] = splat(1.f);
     }
     if constexpr (BIAS) {
-      if (b) {
+      if (AFF || b) {
         Elem<T>::unpack(load_cached(b + f * V), bf);
       } else {
 #pragma unroll
@@ -498,7 +508,7 @@ constexpr int affine_cache_bytes(int threads) {
 
 // Normalize the thread's chunks and edge element of one row, apply weight
 // (and bias), store.
-template <typename T, int OP, bool EXACT, int NSLOT, typename Src>
+template <typename T, int OP, bool EXACT, bool FULL, int NSLOT, typename Src>
 __device__ __forceinline__ void normalize_store(const Segment& s, const Row<T>& g,
                                                 const F2 (&v)[NSLOT][Elem<T>::P], float xe,
                                                 const Src& src, int k0, int step, float rstd,
@@ -510,7 +520,7 @@ __device__ __forceinline__ void normalize_store(const Segment& s, const Row<T>& 
 #pragma unroll
   for (int p = 0; p < NSLOT; ++p) {
     const int f = k0 + step * p;
-    if (f >= g.nfull) continue;
+    if (!FULL && f >= g.nfull) continue;
     F2 wf[P], bf[P], o[P];
     src.get(p, f, wf, bf);
 #pragma unroll
@@ -545,7 +555,7 @@ __device__ __forceinline__ void normalize_store(const Segment& s, const Row<T>& 
 
 // rstd (and mean) of one row from the thread's slots and edge element, with
 // `reduce` summing a per-thread partial over the threads of the row.
-template <typename T, int OP, bool EXACT, int NSLOT, typename Reduce>
+template <typename T, int OP, bool EXACT, bool FULL, int NSLOT, typename Reduce>
 __device__ __forceinline__ void row_stats(F2 (&v)[NSLOT][Elem<T>::P], float& xe,
                                           const Row<T>& g, int D, int k0, int step, float K,
                                           float eps, bool has_edge, Reduce reduce, float& rstd,
@@ -558,10 +568,10 @@ __device__ __forceinline__ void row_stats(F2 (&v)[NSLOT][Elem<T>::P], float& xe,
     mean = 0.f;
     rstd = rsqrtf(__fadd_rn(__fmul_rn(ss, inv_d), eps));
   } else {
-    const float s1 = reduce(shift_and_sum<T, EXACT, NSLOT>(v, xe, g, k0, step, K, has_edge));
+    const float s1 = reduce(shift_and_sum<T, EXACT, FULL, NSLOT>(v, xe, g, k0, step, K, has_edge));
     mean = __fmul_rn(s1, inv_d);
     const float s2 =
-        reduce(sum_dev_squares<T, EXACT, NSLOT>(v, xe, g, k0, step, mean, has_edge));
+        reduce(sum_dev_squares<T, EXACT, FULL, NSLOT>(v, xe, g, k0, step, mean, has_edge));
     rstd = rsqrtf(__fadd_rn(__fmul_rn(s2, inv_d), eps));
   }
 }

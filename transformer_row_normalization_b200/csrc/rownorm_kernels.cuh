@@ -59,26 +59,28 @@ struct Prefetch {
     return &dyn_smem[(stage * NSLOT + p) * blockDim.x + threadIdx.x];
   }
   // Start the copies of the thread's full chunks of row g into `stage`.
+  template <bool FULL>
   __device__ __forceinline__ void issue(const Row<T>& g, int k0, int step, int stage) const {
     constexpr int V = Elem<T>::V;
     if (!on) return;
 #pragma unroll
     for (int p = 0; p < NSLOT; ++p) {
       const int f = k0 + step * p;
-      if (f < g.nfull) cp_async16(slot(stage, p), g.x_full + (long long)f * V);
+      if (FULL || f < g.nfull) cp_async16(slot(stage, p), g.x_full + (long long)f * V);
     }
   }
   // The thread's slots of row g from `stage` (copies complete); absent ones zero.
+  template <bool FULL>
   __device__ __forceinline__ void take(const Row<T>& g, int k0, int step, int stage,
                                        F2 (&v)[NSLOT][Elem<T>::P]) const {
     constexpr int P = Elem<T>::P;
     if (!on) {
-      load_row<T, NSLOT>(g, k0, step, v);
+      load_row<T, FULL, NSLOT>(g, k0, step, v);
       return;
     }
 #pragma unroll
     for (int p = 0; p < NSLOT; ++p) {
-      if (k0 + step * p < g.nfull) {
+      if (FULL || k0 + step * p < g.nfull) {
         Elem<T>::unpack(*slot(stage, p), v[p]);
       } else {
 #pragma unroll
@@ -94,15 +96,89 @@ __host__ __device__ constexpr int prefetch_smem_words(int threads) {
   return 2 * NSLOT * threads;
 }
 
-template <typename T, int OP, bool EXACT, int VPL>
+// The rows r0, r0 + stride, ... of one segment, owned by one thread group (a
+// lane group, or a block) in which this thread is k0 of `step`. Each row's
+// chunks are prefetched one row ahead; `src` supplies weight and bias.
+template <typename T, int OP, bool EXACT, bool FULL, int NSLOT, typename Src, typename Reduce>
+__device__ __forceinline__ void segment_rows(const Segment& s, const Prefetch<T, NSLOT>& pf,
+                                             long long r0, long long stride, int k0, int step,
+                                             float eps, Reduce reduce, Src& src) {
+  constexpr int P = Elem<T>::P;
+  const int D = s.dim;
+  long long r = r0;
+  float Kn = 0.f, En = 0.f;
+  if (r < s.rows) {
+    const Row<T> gn = row_geometry<T, EXACT>(s, r);
+    pf.template issue<FULL>(gn, k0, step, 0);
+    if (OP == kOpLn) Kn = Elem<T>::get(gn.x_row);
+    En = load_edge<T, EXACT>(gn, D, k0);
+  }
+  cp_async_commit();
+#pragma unroll 1
+  for (int i = 0; r < s.rows; ++i, r += stride) {
+    const float K = Kn;
+    float xe = En;
+    const long long rn = r + stride;
+    if (rn < s.rows) {
+      const Row<T> gn = row_geometry<T, EXACT>(s, rn);
+      pf.template issue<FULL>(gn, k0, step, (i + 1) & 1);
+      if (OP == kOpLn) Kn = Elem<T>::get(gn.x_row);
+      En = load_edge<T, EXACT>(gn, D, k0);
+    }
+    cp_async_commit();
+    cp_async_wait<1>();
+    const Row<T> g = row_geometry<T, EXACT>(s, r);
+    const bool has_edge = !EXACT && k0 < g.nedge;
+    F2 v[NSLOT][P];
+    pf.template take<FULL>(g, k0, step, i & 1, v);
+    float rstd, mean;
+    row_stats<T, OP, EXACT, FULL, NSLOT>(v, xe, g, D, k0, step, K, eps, has_edge, reduce, rstd,
+                                         mean);
+    if constexpr (!EXACT) {
+      if (g.phase != src.phase) src.fill(s, g, k0, step);
+    }
+    normalize_store<T, OP, EXACT, FULL, NSLOT>(s, g, v, xe, src, k0, step, rstd, mean,
+                                               has_edge);
+  }
+  cp_async_wait<0>();
+}
+
+// One segment with the weight/bias source its layout calls for: for EXACT
+// layouts straight from the vectors (a loop without NULL tests when every
+// vector the op uses is present), otherwise the realigned per-thread cache
+// at 16-byte word `cache_word` of the dynamic shared memory.
+template <typename T, int OP, int LAYOUT, int NSLOT, typename Reduce>
+__device__ __forceinline__ void run_segment(const Segment& s, const Prefetch<T, NSLOT>& pf,
+                                            long long r0, long long stride, int k0, int step,
+                                            float eps, Reduce reduce, int cache_word) {
+  constexpr bool BIAS = OP == kOpLn;
+  constexpr bool EXACT = LAYOUT != kLayoutAny;
+  constexpr bool FULL = LAYOUT == kLayoutFull;
+  const T* w = static_cast<const T*>(s.w);
+  const T* b = static_cast<const T*>(s.b);
+  if constexpr (EXACT) {
+    if (w && (!BIAS || b)) {
+      AffineDirect<T, BIAS, true> src{w, b};
+      segment_rows<T, OP, true, FULL, NSLOT>(s, pf, r0, stride, k0, step, eps, reduce, src);
+    } else {
+      AffineDirect<T, BIAS, false> src{w, b};
+      segment_rows<T, OP, true, FULL, NSLOT>(s, pf, r0, stride, k0, step, eps, reduce, src);
+    }
+  } else {
+    AffineCache<T, NSLOT, BIAS> src;
+    src.init(cache_word);
+    segment_rows<T, OP, false, false, NSLOT>(s, pf, r0, stride, k0, step, eps, reduce, src);
+  }
+}
+
+template <typename T, int OP, int LAYOUT, int VPL>
 __global__ void __launch_bounds__(kWarpBlock, kMinThreadsPerSmWarp / kWarpBlock)
 rows_warp_kernel(const Params p) {
-  constexpr int P = Elem<T>::P;
-  constexpr bool BIAS = OP == kOpLn;
   const Prefetch<T, VPL> pf{p.prefetch};
   const int lane = threadIdx.x & 31;
   const long long warp = (long long)blockIdx.x * (kWarpBlock / 32) + (threadIdx.x >> 5);
   const long long nwarps = (long long)gridDim.x * (kWarpBlock / 32);
+  const int cache_word = p.prefetch ? prefetch_smem_words<VPL>(kWarpBlock) : 0;
 #pragma unroll 1
   for (int si = 0; si < p.nseg; ++si) {
     const Segment s = pick_segment(p.seg, si);
@@ -111,112 +187,32 @@ rows_warp_kernel(const Params p) {
     const int gl = lane & (G - 1);
     const int gi = lane / G;
     const unsigned mask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << (gi * G));
-    const long long ngroups = nwarps * per_warp;
-    const int D = s.dim;
-    AffineCache<T, VPL, BIAS> cache;
-    if constexpr (!EXACT)
-      cache.init(p.prefetch ? prefetch_smem_words<VPL>(kWarpBlock) : 0);
-    const AffineDirect<T, BIAS> direct{static_cast<const T*>(s.w), static_cast<const T*>(s.b)};
     auto reduce = [&](float t) { return group_sum(t, G, mask); };
-    long long r = warp * per_warp + gi;
-    float Kn = 0.f, En = 0.f;
-    if (r < s.rows) {
-      const Row<T> gn = row_geometry<T, EXACT>(s, r);
-      pf.issue(gn, gl, G, 0);
-      if (OP == kOpLn) Kn = Elem<T>::get(gn.x_row);
-      En = load_edge<T, EXACT>(gn, D, gl);
-    }
-    cp_async_commit();
-#pragma unroll 1
-    for (int i = 0; r < s.rows; ++i, r += ngroups) {
-      const float K = Kn;
-      float xe = En;
-      const long long rn = r + ngroups;
-      if (rn < s.rows) {
-        const Row<T> gn = row_geometry<T, EXACT>(s, rn);
-        pf.issue(gn, gl, G, (i + 1) & 1);
-        if (OP == kOpLn) Kn = Elem<T>::get(gn.x_row);
-        En = load_edge<T, EXACT>(gn, D, gl);
-      }
-      cp_async_commit();
-      cp_async_wait<1>();
-      const Row<T> g = row_geometry<T, EXACT>(s, r);
-      const bool has_edge = !EXACT && gl < g.nedge;
-      F2 v[VPL][P];
-      pf.take(g, gl, G, i & 1, v);
-      float rstd, mean;
-      row_stats<T, OP, EXACT, VPL>(v, xe, g, D, gl, G, K, p.eps, has_edge, reduce, rstd, mean);
-      if constexpr (EXACT) {
-        normalize_store<T, OP, EXACT, VPL>(s, g, v, xe, direct, gl, G, rstd, mean, has_edge);
-      } else {
-        if (g.phase != cache.phase) cache.fill(s, g, gl, G);
-        normalize_store<T, OP, EXACT, VPL>(s, g, v, xe, cache, gl, G, rstd, mean, has_edge);
-      }
-    }
-    cp_async_wait<0>();
+    run_segment<T, OP, LAYOUT, VPL>(s, pf, warp * per_warp + gi, nwarps * per_warp, gl, G,
+                                    p.eps, reduce, cache_word);
   }
 }
 
-template <typename T, int OP, bool EXACT, int NT, int VPT>
+template <typename T, int OP, int LAYOUT, int NT, int VPT>
 __global__ void __launch_bounds__(NT, kMinThreadsPerSm / NT)
 rows_cta_kernel(const Params p) {
-  constexpr int P = Elem<T>::P;
   static_assert(NT >= 2 * (Elem<T>::V - 1), "every edge element needs its own thread");
-  constexpr bool BIAS = OP == kOpLn;
   // Two alternating reduction buffers: a buffer is rewritten only after every
   // thread has passed the barrier of the reduction in between.
   __shared__ float red[2][NT / 32];
   const Prefetch<T, VPT> pf{p.prefetch};
   int slot = 0;
-  const int tid = threadIdx.x;
   auto reduce = [&](float t) {
     const float r = block_sum<NT>(t, red[slot]);
     slot ^= 1;
     return r;
   };
+  const int cache_word = p.prefetch ? prefetch_smem_words<VPT>(NT) : 0;
 #pragma unroll 1
   for (int si = 0; si < p.nseg; ++si) {
     const Segment s = pick_segment(p.seg, si);
-    const int D = s.dim;
-    AffineCache<T, VPT, BIAS> cache;
-    if constexpr (!EXACT) cache.init(p.prefetch ? prefetch_smem_words<VPT>(NT) : 0);
-    const AffineDirect<T, BIAS> direct{static_cast<const T*>(s.w), static_cast<const T*>(s.b)};
-    long long r = blockIdx.x;
-    float Kn = 0.f, En = 0.f;
-    if (r < s.rows) {
-      const Row<T> gn = row_geometry<T, EXACT>(s, r);
-      pf.issue(gn, tid, NT, 0);
-      if (OP == kOpLn) Kn = Elem<T>::get(gn.x_row);
-      En = load_edge<T, EXACT>(gn, D, tid);
-    }
-    cp_async_commit();
-#pragma unroll 1
-    for (int i = 0; r < s.rows; ++i, r += gridDim.x) {
-      const float K = Kn;
-      float xe = En;
-      const long long rn = r + gridDim.x;
-      if (rn < s.rows) {
-        const Row<T> gn = row_geometry<T, EXACT>(s, rn);
-        pf.issue(gn, tid, NT, (i + 1) & 1);
-        if (OP == kOpLn) Kn = Elem<T>::get(gn.x_row);
-        En = load_edge<T, EXACT>(gn, D, tid);
-      }
-      cp_async_commit();
-      cp_async_wait<1>();
-      const Row<T> g = row_geometry<T, EXACT>(s, r);
-      const bool has_edge = !EXACT && tid < g.nedge;
-      F2 v[VPT][P];
-      pf.take(g, tid, NT, i & 1, v);
-      float rstd, mean;
-      row_stats<T, OP, EXACT, VPT>(v, xe, g, D, tid, NT, K, p.eps, has_edge, reduce, rstd, mean);
-      if constexpr (EXACT) {
-        normalize_store<T, OP, EXACT, VPT>(s, g, v, xe, direct, tid, NT, rstd, mean, has_edge);
-      } else {
-        if (g.phase != cache.phase) cache.fill(s, g, tid, NT);
-        normalize_store<T, OP, EXACT, VPT>(s, g, v, xe, cache, tid, NT, rstd, mean, has_edge);
-      }
-    }
-    cp_async_wait<0>();
+    run_segment<T, OP, LAYOUT, VPT>(s, pf, blockIdx.x, gridDim.x, threadIdx.x, NT, p.eps,
+                                    reduce, cache_word);
   }
 }
 
