@@ -136,7 +136,8 @@ struct SegPlan {
   int vector_y;      // y rows share x's 16-byte phase
   int phase_period;  // distinct 16-byte phases among the rows of x
   int exact;         // every x and y row 16-byte aligned, dim % V == 0
-  int full;          // exact, and dim / V == lanes * chunks (no slot ever empty)
+  int64_t nfull_max; // full 16-byte chunks of a row: at most / at least
+  int64_t nfull_min;
 };
 
 // The lane count / block size is a function of (dtype, dim) and, for lane
@@ -186,21 +187,31 @@ SegPlan plan_segment(const rn_view* x, const rn_view* y, const void* w, const vo
   p.exact = rows_aligned && ya % 16 == 0 &&
             (y->rows <= 1 || (y->row_stride * es) % 16 == 0) &&
             reinterpret_cast<uintptr_t>(w) % 16 == 0 && reinterpret_cast<uintptr_t>(b) % 16 == 0;
-  p.full = p.exact && nfull == (int64_t)p.lanes * p.chunks && p.chunks <= rn::kFullMaxChunks;
+  p.nfull_max = nfull;
+  p.nfull_min = rows_aligned ? nfull : (nfull > 0 ? nfull - 1 : 0);
   return p;
 }
 
-int layout_of(const SegPlan& p) {
-  return p.full ? rn::kLayoutFull : (p.exact ? rn::kLayoutExact : rn::kLayoutAny);
+// The slots of a thread that every row of segment p fills when each thread
+// has `chunks` slots: all of them (rows divide evenly; EXACT only), all but
+// the last, or no guarantee.
+int slot_class(const SegPlan& p, int chunks) {
+  if (p.exact && p.nfull_max == (int64_t)p.lanes * chunks && chunks <= rn::kFullMaxChunks)
+    return rn::kSlotsFull;
+  // block-family kernels with more than kFullMaxChunks slots spill when
+  // specialized and measured faster testing every slot
+  if (p.family == 1 && chunks > rn::kFullMaxChunks) return rn::kSlotsTested;
+  if ((int64_t)(chunks - 1) * p.lanes <= p.nfull_min) return rn::kSlotsTail;
+  return rn::kSlotsTested;
 }
 
-const void* kernel_for(int dtype, int op, const SegPlan& p) {
-  const int lay = layout_of(p);
+const void* kernel_for(int dtype, int op, const SegPlan& p, int slots) {
+  const bool ex = p.exact != 0;
   if (p.family == 0)
-    return dtype == RN_F32 ? rn::warp_kernel_f32(op, lay, p.chunks)
-                           : rn::warp_kernel_bf16(op, lay, p.chunks);
-  return dtype == RN_F32 ? rn::cta_kernel_f32(op, lay, p.lanes, p.chunks)
-                         : rn::cta_kernel_bf16(op, lay, p.lanes, p.chunks);
+    return dtype == RN_F32 ? rn::warp_kernel_f32(op, ex, slots, p.chunks)
+                           : rn::warp_kernel_bf16(op, ex, slots, p.chunks);
+  return dtype == RN_F32 ? rn::cta_kernel_f32(op, ex, slots, p.lanes, p.chunks)
+                         : rn::cta_kernel_bf16(op, ex, slots, p.lanes, p.chunks);
 }
 
 struct DeviceInfo {
@@ -395,12 +406,17 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
   int64_t rows[2] = {xs[0]->rows, nseg > 1 ? xs[1]->rows : 0};
   SegPlan merged = plans[0];
   for (int i = 1; i < nseg; ++i) {
-    if (plans[i].chunks != merged.chunks) merged.full = 0;  // a segment would leave slots empty
     if (plans[i].chunks > merged.chunks) merged.chunks = plans[i].chunks;
     merged.exact = merged.exact && plans[i].exact;
-    merged.full = merged.full && plans[i].full;
   }
-  const void* fn = kernel_for(dtype, op, merged);
+  // every segment runs with the merged slot count
+  int slots = rn::kSlotsFull;
+  for (int i = 0; i < nseg; ++i) {
+    const int c = slot_class(plans[i], merged.chunks);
+    if (c < slots) slots = c;
+  }
+  if (!merged.exact && slots == rn::kSlotsFull) slots = rn::kSlotsTail;
+  const void* fn = kernel_for(dtype, op, merged, slots);
   if (!fn) return fail(RN_ERR_UNSUPPORTED, "no compiled kernel for this shape");
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -411,7 +427,9 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
   if (plan_staged(dtype, op, plans, xs, ws, bs, nseg, dev, sms, out)) return RN_OK;
   const int threads = merged.family == 0 ? rn::kWarpBlock : merged.lanes;
   const int cache = merged.exact ? 0 : rn::affine_cache_smem_bytes(op, threads, merged.chunks);
-  const int slots = rn::prefetch_slots_smem_bytes(threads, merged.chunks);
+  const int pf_bytes = rn::prefetch_slots_smem_bytes(
+      threads, merged.chunks,
+      merged.family == 0 ? rn::kWarpPrefetchStages : rn::kCtaPrefetchStages);
   // Next-row prefetch where it measured faster on B200: lane-group rows and
   // blocks of 256 or more threads (few blocks per SM, so few rows in
   // flight); blocks of 128 threads already keep 8+ rows per SM in flight and
@@ -421,8 +439,8 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
       g_path_override == 3 ||
       (g_path_override == 0 && (merged.family == 0 || merged.lanes >= 256));
   const int prefetch =
-      want_prefetch && cache + slots <= device_info(dev).smem_per_block - 1024 ? 1 : 0;
-  const int smem = cache + (prefetch ? slots : 0);
+      want_prefetch && cache + pf_bytes <= device_info(dev).smem_per_block - 1024 ? 1 : 0;
+  const int smem = cache + (prefetch ? pf_bytes : 0);
   st = blocks_per_sm(dev, fn, threads, smem, &bps);
   if (st) return st;
   int64_t needed = 1;
@@ -458,7 +476,7 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
   in.blocks_per_sm = bps;
   in.vector_y = plans[0].vector_y;
   in.phase_period = plans[0].phase_period;
-  in.exact = layout_of(merged);
+  in.exact = merged.exact ? (slots == rn::kSlotsFull ? 2 : 1) : 0;
   return RN_OK;
 }
 

@@ -50,14 +50,22 @@ namespace rn {
 
 enum : int { kOpRms = 0, kOpLn = 1 };
 
-// Layout classes of a launch (what the planner guarantees for every row):
-//   kLayoutAny    any 16-byte phase, any D, any weight/bias alignment;
-//   kLayoutExact  EXACT: x and y rows, weight and bias start on 16-byte
-//                 boundaries and D is a multiple of V (no edge elements);
-//   kLayoutFull   EXACT, and the row's D / V chunks divide evenly over the
-//                 threads of the row: every thread owns all its slots in
-//                 every row, so no slot is ever tested.
-enum : int { kLayoutAny = 0, kLayoutExact = 1, kLayoutFull = 2 };
+// Which of a thread's NSLOT chunk slots the planner guarantees present in
+// every row of a launch:
+//   kSlotsTested  none: each slot is tested against the row's chunk count;
+//   kSlotsTail    all but the last (tested): slot counts are ceil(chunks /
+//                 threads) and a row's chunk count varies by at most one
+//                 between 16-byte phases;
+//   kSlotsFull    all: the row's chunks divide evenly over its threads
+//                 (EXACT layouts only), so no slot is ever tested.
+enum : int { kSlotsTested = 0, kSlotsTail = 1, kSlotsFull = 2 };
+
+template <int SLOTS, int NSLOT>
+__device__ __forceinline__ bool slot_present(int p, int f, int nfull) {
+  if constexpr (SLOTS == kSlotsFull) return true;
+  if (SLOTS == kSlotsTail && p < NSLOT - 1) return true;
+  return f < nfull;
+}
 
 // One row space (a tensor viewed as [rows, dim]); strides in elements.
 struct Segment {
@@ -271,7 +279,7 @@ __device__ __forceinline__ float load_edge(const Row<T>& g, int D, int k0) {
 }
 
 // All of a thread's slots of one row from global memory (absent ones zero).
-template <typename T, bool FULL, int NSLOT>
+template <typename T, int SLOTS, int NSLOT>
 __device__ __forceinline__ void load_row(const Row<T>& g, int k0, int step,
                                          F2 (&v)[NSLOT][Elem<T>::P]) {
   constexpr int V = Elem<T>::V;
@@ -279,7 +287,7 @@ __device__ __forceinline__ void load_row(const Row<T>& g, int k0, int step,
 #pragma unroll
   for (int p = 0; p < NSLOT; ++p) {
     const int f = k0 + step * p;
-    if (FULL || f < g.nfull) {
+    if (slot_present<SLOTS, NSLOT>(p, f, g.nfull)) {
       Elem<T>::unpack(load_stream(g.x_full + (long long)f * V), v[p]);
     } else {
 #pragma unroll
@@ -312,7 +320,7 @@ __device__ __forceinline__ float sum_squares(const F2 (&v)[NSLOT][Elem<T>::P], f
 
 // LayerNorm pass 1: replaces x by d = x - K (slots and edge element) and
 // returns the thread's sum of d.
-template <typename T, bool EXACT, bool FULL, int NSLOT>
+template <typename T, bool EXACT, int SLOTS, int NSLOT>
 __device__ __forceinline__ float shift_and_sum(F2 (&v)[NSLOT][Elem<T>::P], float& xe,
                                                const Row<T>& g, int k0, int step, float K,
                                                bool has_edge) {
@@ -321,7 +329,7 @@ __device__ __forceinline__ float shift_and_sum(F2 (&v)[NSLOT][Elem<T>::P], float
   F2 acc = zero2();
 #pragma unroll
   for (int p = 0; p < NSLOT; ++p) {
-    if (FULL || k0 + step * p < g.nfull) {
+    if (slot_present<SLOTS, NSLOT>(p, k0 + step * p, g.nfull)) {
 #pragma unroll
       for (int j = 0; j < P; ++j) {
         v[p][j] = sub2(v[p][j], K2);
@@ -338,7 +346,7 @@ __device__ __forceinline__ float shift_and_sum(F2 (&v)[NSLOT][Elem<T>::P], float
 }
 
 // LayerNorm pass 2: the thread's sum of (d - mean)^2.
-template <typename T, bool EXACT, bool FULL, int NSLOT>
+template <typename T, bool EXACT, int SLOTS, int NSLOT>
 __device__ __forceinline__ float sum_dev_squares(const F2 (&v)[NSLOT][Elem<T>::P], float xe,
                                                  const Row<T>& g, int k0, int step, float mean,
                                                  bool has_edge) {
@@ -347,7 +355,7 @@ __device__ __forceinline__ float sum_dev_squares(const F2 (&v)[NSLOT][Elem<T>::P
   F2 acc = zero2();
 #pragma unroll
   for (int p = 0; p < NSLOT; ++p) {
-    if (FULL || k0 + step * p < g.nfull) {
+    if (slot_present<SLOTS, NSLOT>(p, k0 + step * p, g.nfull)) {
 #pragma unroll
       for (int j = 0; j < P; ++j) {
         const F2 t = sub2(v[p][j], M2);
@@ -508,7 +516,7 @@ constexpr int affine_cache_bytes(int threads) {
 
 // Normalize the thread's chunks and edge element of one row, apply weight
 // (and bias), store.
-template <typename T, int OP, bool EXACT, bool FULL, int NSLOT, typename Src>
+template <typename T, int OP, bool EXACT, int SLOTS, int NSLOT, typename Src>
 __device__ __forceinline__ void normalize_store(const Segment& s, const Row<T>& g,
                                                 const F2 (&v)[NSLOT][Elem<T>::P], float xe,
                                                 const Src& src, int k0, int step, float rstd,
@@ -520,7 +528,7 @@ __device__ __forceinline__ void normalize_store(const Segment& s, const Row<T>& 
 #pragma unroll
   for (int p = 0; p < NSLOT; ++p) {
     const int f = k0 + step * p;
-    if (!FULL && f >= g.nfull) continue;
+    if (!slot_present<SLOTS, NSLOT>(p, f, g.nfull)) continue;
     F2 wf[P], bf[P], o[P];
     src.get(p, f, wf, bf);
 #pragma unroll
@@ -555,7 +563,7 @@ __device__ __forceinline__ void normalize_store(const Segment& s, const Row<T>& 
 
 // rstd (and mean) of one row from the thread's slots and edge element, with
 // `reduce` summing a per-thread partial over the threads of the row.
-template <typename T, int OP, bool EXACT, bool FULL, int NSLOT, typename Reduce>
+template <typename T, int OP, bool EXACT, int SLOTS, int NSLOT, typename Reduce>
 __device__ __forceinline__ void row_stats(F2 (&v)[NSLOT][Elem<T>::P], float& xe,
                                           const Row<T>& g, int D, int k0, int step, float K,
                                           float eps, bool has_edge, Reduce reduce, float& rstd,
@@ -568,10 +576,10 @@ __device__ __forceinline__ void row_stats(F2 (&v)[NSLOT][Elem<T>::P], float& xe,
     mean = 0.f;
     rstd = rsqrtf(__fadd_rn(__fmul_rn(ss, inv_d), eps));
   } else {
-    const float s1 = reduce(shift_and_sum<T, EXACT, FULL, NSLOT>(v, xe, g, k0, step, K, has_edge));
+    const float s1 = reduce(shift_and_sum<T, EXACT, SLOTS, NSLOT>(v, xe, g, k0, step, K, has_edge));
     mean = __fmul_rn(s1, inv_d);
     const float s2 =
-        reduce(sum_dev_squares<T, EXACT, FULL, NSLOT>(v, xe, g, k0, step, mean, has_edge));
+        reduce(sum_dev_squares<T, EXACT, SLOTS, NSLOT>(v, xe, g, k0, step, mean, has_edge));
     rstd = rsqrtf(__fadd_rn(__fmul_rn(s2, inv_d), eps));
   }
 }

@@ -48,7 +48,7 @@ constexpr int kWarpBlock = 256;
 constexpr int kMinThreadsPerSmWarp = 768;
 constexpr int kMinThreadsPerSm = 1024;
 
-// Per-thread prefetch slots: [2 stages][NSLOT][blockDim.x] 16-byte words.
+// Per-thread prefetch slots: [stages][NSLOT][blockDim.x] 16-byte words.
 // When the slots do not fit in shared memory next to the weight cache (the
 // planner decides), `on` is 0: nothing is copied ahead and rows are loaded
 // straight from global memory when they are taken.
@@ -59,28 +59,29 @@ struct Prefetch {
     return &dyn_smem[(stage * NSLOT + p) * blockDim.x + threadIdx.x];
   }
   // Start the copies of the thread's full chunks of row g into `stage`.
-  template <bool FULL>
+  template <int SLOTS>
   __device__ __forceinline__ void issue(const Row<T>& g, int k0, int step, int stage) const {
     constexpr int V = Elem<T>::V;
     if (!on) return;
 #pragma unroll
     for (int p = 0; p < NSLOT; ++p) {
       const int f = k0 + step * p;
-      if (FULL || f < g.nfull) cp_async16(slot(stage, p), g.x_full + (long long)f * V);
+      if (slot_present<SLOTS, NSLOT>(p, f, g.nfull))
+        cp_async16(slot(stage, p), g.x_full + (long long)f * V);
     }
   }
   // The thread's slots of row g from `stage` (copies complete); absent ones zero.
-  template <bool FULL>
+  template <int SLOTS>
   __device__ __forceinline__ void take(const Row<T>& g, int k0, int step, int stage,
                                        F2 (&v)[NSLOT][Elem<T>::P]) const {
     constexpr int P = Elem<T>::P;
     if (!on) {
-      load_row<T, FULL, NSLOT>(g, k0, step, v);
+      load_row<T, SLOTS, NSLOT>(g, k0, step, v);
       return;
     }
 #pragma unroll
     for (int p = 0; p < NSLOT; ++p) {
-      if (FULL || k0 + step * p < g.nfull) {
+      if (slot_present<SLOTS, NSLOT>(p, k0 + step * p, g.nfull)) {
         Elem<T>::unpack(*slot(stage, p), v[p]);
       } else {
 #pragma unroll
@@ -90,55 +91,80 @@ struct Prefetch {
   }
 };
 
-// 16-byte words of prefetch slots (two stages).
-template <int NSLOT>
+// Prefetch stages (rows in flight per thread group: the one being normalized
+// and NST - 1 ahead). Measured on B200, a third stage gained nothing for lane
+// groups (LayerNorm 768, 1000, 1024; RMSNorm 512) and cost up to 8 % for
+// blocks, so both families keep one row ahead.
+constexpr int kWarpPrefetchStages = 2;
+constexpr int kCtaPrefetchStages = 2;
+
+// 16-byte words of prefetch slots.
+template <int NSLOT, int NST>
 __host__ __device__ constexpr int prefetch_smem_words(int threads) {
-  return 2 * NSLOT * threads;
+  return NST * NSLOT * threads;
 }
 
 // The rows r0, r0 + stride, ... of one segment, owned by one thread group (a
 // lane group, or a block) in which this thread is k0 of `step`. Each row's
-// chunks are prefetched one row ahead; `src` supplies weight and bias.
-template <typename T, int OP, bool EXACT, bool FULL, int NSLOT, typename Src, typename Reduce>
+// chunks are prefetched NST - 1 rows ahead, stage i % NST holding row i;
+// the shift K and the thread's edge element of the rows ahead wait in
+// register queues. `src` supplies weight and bias.
+template <typename T, int OP, bool EXACT, int SLOTS, int NSLOT, int NST, typename Src,
+          typename Reduce>
 __device__ __forceinline__ void segment_rows(const Segment& s, const Prefetch<T, NSLOT>& pf,
                                              long long r0, long long stride, int k0, int step,
                                              float eps, Reduce reduce, Src& src) {
+  static_assert(NST >= 2, "at least one row ahead");
   constexpr int P = Elem<T>::P;
   const int D = s.dim;
-  long long r = r0;
-  float Kn = 0.f, En = 0.f;
-  if (r < s.rows) {
-    const Row<T> gn = row_geometry<T, EXACT>(s, r);
-    pf.template issue<FULL>(gn, k0, step, 0);
-    if (OP == kOpLn) Kn = Elem<T>::get(gn.x_row);
-    En = load_edge<T, EXACT>(gn, D, k0);
-  }
-  cp_async_commit();
-#pragma unroll 1
-  for (int i = 0; r < s.rows; ++i, r += stride) {
-    const float K = Kn;
-    float xe = En;
-    const long long rn = r + stride;
-    if (rn < s.rows) {
-      const Row<T> gn = row_geometry<T, EXACT>(s, rn);
-      pf.template issue<FULL>(gn, k0, step, (i + 1) & 1);
-      if (OP == kOpLn) Kn = Elem<T>::get(gn.x_row);
-      En = load_edge<T, EXACT>(gn, D, k0);
+  float Kq[NST - 1], Eq[NST - 1];
+#pragma unroll
+  for (int j = 0; j < NST - 1; ++j) {
+    const long long rj = r0 + j * stride;
+    Kq[j] = 0.f;
+    Eq[j] = 0.f;
+    if (rj < s.rows) {
+      const Row<T> gj = row_geometry<T, EXACT>(s, rj);
+      pf.template issue<SLOTS>(gj, k0, step, j);
+      if (OP == kOpLn) Kq[j] = Elem<T>::get(gj.x_row);
+      Eq[j] = load_edge<T, EXACT>(gj, D, k0);
     }
     cp_async_commit();
-    cp_async_wait<1>();
+  }
+  int st = 0;  // stage of row r
+#pragma unroll 1
+  for (long long r = r0; r < s.rows; r += stride) {
+    const float K = Kq[0];
+    float xe = Eq[0];
+#pragma unroll
+    for (int j = 0; j + 1 < NST - 1; ++j) {
+      Kq[j] = Kq[j + 1];
+      Eq[j] = Eq[j + 1];
+    }
+    // the stage the previous row was taken from receives row r + (NST-1) stride
+    const int sa = st == 0 ? NST - 1 : st - 1;
+    const long long ra = r + (NST - 1) * stride;
+    if (ra < s.rows) {
+      const Row<T> ga = row_geometry<T, EXACT>(s, ra);
+      pf.template issue<SLOTS>(ga, k0, step, sa);
+      if (OP == kOpLn) Kq[NST - 2] = Elem<T>::get(ga.x_row);
+      Eq[NST - 2] = load_edge<T, EXACT>(ga, D, k0);
+    }
+    cp_async_commit();
+    cp_async_wait<NST - 1>();
     const Row<T> g = row_geometry<T, EXACT>(s, r);
     const bool has_edge = !EXACT && k0 < g.nedge;
     F2 v[NSLOT][P];
-    pf.template take<FULL>(g, k0, step, i & 1, v);
+    pf.template take<SLOTS>(g, k0, step, st, v);
     float rstd, mean;
-    row_stats<T, OP, EXACT, FULL, NSLOT>(v, xe, g, D, k0, step, K, eps, has_edge, reduce, rstd,
-                                         mean);
+    row_stats<T, OP, EXACT, SLOTS, NSLOT>(v, xe, g, D, k0, step, K, eps, has_edge, reduce, rstd,
+                                          mean);
     if constexpr (!EXACT) {
       if (g.phase != src.phase) src.fill(s, g, k0, step);
     }
-    normalize_store<T, OP, EXACT, FULL, NSLOT>(s, g, v, xe, src, k0, step, rstd, mean,
-                                               has_edge);
+    normalize_store<T, OP, EXACT, SLOTS, NSLOT>(s, g, v, xe, src, k0, step, rstd, mean,
+                                                has_edge);
+    st = st == NST - 1 ? 0 : st + 1;
   }
   cp_async_wait<0>();
 }
@@ -147,38 +173,37 @@ __device__ __forceinline__ void segment_rows(const Segment& s, const Prefetch<T,
 // layouts straight from the vectors (a loop without NULL tests when every
 // vector the op uses is present), otherwise the realigned per-thread cache
 // at 16-byte word `cache_word` of the dynamic shared memory.
-template <typename T, int OP, int LAYOUT, int NSLOT, typename Reduce>
+template <typename T, int OP, bool EXACT, int SLOTS, int NSLOT, int NST, typename Reduce>
 __device__ __forceinline__ void run_segment(const Segment& s, const Prefetch<T, NSLOT>& pf,
                                             long long r0, long long stride, int k0, int step,
                                             float eps, Reduce reduce, int cache_word) {
   constexpr bool BIAS = OP == kOpLn;
-  constexpr bool EXACT = LAYOUT != kLayoutAny;
-  constexpr bool FULL = LAYOUT == kLayoutFull;
+  static_assert(EXACT || SLOTS != kSlotsFull, "only EXACT rows divide evenly");
   const T* w = static_cast<const T*>(s.w);
   const T* b = static_cast<const T*>(s.b);
   if constexpr (EXACT) {
     if (w && (!BIAS || b)) {
       AffineDirect<T, BIAS, true> src{w, b};
-      segment_rows<T, OP, true, FULL, NSLOT>(s, pf, r0, stride, k0, step, eps, reduce, src);
+      segment_rows<T, OP, true, SLOTS, NSLOT, NST>(s, pf, r0, stride, k0, step, eps, reduce, src);
     } else {
       AffineDirect<T, BIAS, false> src{w, b};
-      segment_rows<T, OP, true, FULL, NSLOT>(s, pf, r0, stride, k0, step, eps, reduce, src);
+      segment_rows<T, OP, true, SLOTS, NSLOT, NST>(s, pf, r0, stride, k0, step, eps, reduce, src);
     }
   } else {
     AffineCache<T, NSLOT, BIAS> src;
     src.init(cache_word);
-    segment_rows<T, OP, false, false, NSLOT>(s, pf, r0, stride, k0, step, eps, reduce, src);
+    segment_rows<T, OP, false, SLOTS, NSLOT, NST>(s, pf, r0, stride, k0, step, eps, reduce, src);
   }
 }
 
-template <typename T, int OP, int LAYOUT, int VPL>
+template <typename T, int OP, bool EXACT, int SLOTS, int VPL>
 __global__ void __launch_bounds__(kWarpBlock, kMinThreadsPerSmWarp / kWarpBlock)
 rows_warp_kernel(const Params p) {
   const Prefetch<T, VPL> pf{p.prefetch};
   const int lane = threadIdx.x & 31;
   const long long warp = (long long)blockIdx.x * (kWarpBlock / 32) + (threadIdx.x >> 5);
   const long long nwarps = (long long)gridDim.x * (kWarpBlock / 32);
-  const int cache_word = p.prefetch ? prefetch_smem_words<VPL>(kWarpBlock) : 0;
+  const int cache_word = p.prefetch ? prefetch_smem_words<VPL, kWarpPrefetchStages>(kWarpBlock) : 0;
 #pragma unroll 1
   for (int si = 0; si < p.nseg; ++si) {
     const Segment s = pick_segment(p.seg, si);
@@ -188,12 +213,12 @@ rows_warp_kernel(const Params p) {
     const int gi = lane / G;
     const unsigned mask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << (gi * G));
     auto reduce = [&](float t) { return group_sum(t, G, mask); };
-    run_segment<T, OP, LAYOUT, VPL>(s, pf, warp * per_warp + gi, nwarps * per_warp, gl, G,
+    run_segment<T, OP, EXACT, SLOTS, VPL, kWarpPrefetchStages>(s, pf, warp * per_warp + gi, nwarps * per_warp, gl, G,
                                     p.eps, reduce, cache_word);
   }
 }
 
-template <typename T, int OP, int LAYOUT, int NT, int VPT>
+template <typename T, int OP, bool EXACT, int SLOTS, int NT, int VPT>
 __global__ void __launch_bounds__(NT, kMinThreadsPerSm / NT)
 rows_cta_kernel(const Params p) {
   static_assert(NT >= 2 * (Elem<T>::V - 1), "every edge element needs its own thread");
@@ -207,11 +232,11 @@ rows_cta_kernel(const Params p) {
     slot ^= 1;
     return r;
   };
-  const int cache_word = p.prefetch ? prefetch_smem_words<VPT>(NT) : 0;
+  const int cache_word = p.prefetch ? prefetch_smem_words<VPT, kCtaPrefetchStages>(NT) : 0;
 #pragma unroll 1
   for (int si = 0; si < p.nseg; ++si) {
     const Segment s = pick_segment(p.seg, si);
-    run_segment<T, OP, LAYOUT, VPT>(s, pf, blockIdx.x, gridDim.x, threadIdx.x, NT, p.eps,
+    run_segment<T, OP, EXACT, SLOTS, VPT, kCtaPrefetchStages>(s, pf, blockIdx.x, gridDim.x, threadIdx.x, NT, p.eps,
                                     reduce, cache_word);
   }
 }

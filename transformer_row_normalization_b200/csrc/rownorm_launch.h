@@ -6,12 +6,12 @@ namespace rn {
 
 constexpr int kWarpFamilyMaxChunksF32 = 8;   // dim <= 1024: at most dim / V full chunks
 constexpr int kWarpFamilyMaxChunksBf16 = 4;  // over lanes >= dim / (4 V)
-constexpr int kCtaMinChunks = 2;             // chunks per thread, block family
+constexpr int kCtaMinChunks = 1;             // chunks per thread, block family
 constexpr int kCtaMaxChunks = 5;
 constexpr int kTargetChunksPerThread = 4;    // 64 bytes of loads in flight per thread
-// Most chunks per thread of a kLayoutFull kernel: at 5 its block-family
-// instantiations spill under the 64-register budget and measured slower on
-// B200 than the tested loop.
+// Most chunks per thread of a kSlotsFull kernel, and of a block-family
+// kSlotsTail kernel: at 5 those instantiations spill under the 64-register
+// budget and measured slower on B200 than the loop that tests every slot.
 constexpr int kFullMaxChunks = 4;
 
 // Shared memory of the realigned weight/bias cache (layouts that are not
@@ -19,18 +19,18 @@ constexpr int kFullMaxChunks = 4;
 constexpr int affine_cache_smem_bytes(int op, int threads, int chunks) {
   return threads * chunks * 16 * (op == 1 ? 2 : 1);
 }
-// Shared memory of the register kernels' prefetch slots (two stages of each
-// thread's chunk slots).
-constexpr int prefetch_slots_smem_bytes(int threads, int chunks) {
-  return 2 * chunks * threads * 16;
+// Shared memory of the register kernels' prefetch slots (`stages` stages of
+// each thread's chunk slots).
+constexpr int prefetch_slots_smem_bytes(int threads, int chunks, int stages) {
+  return stages * chunks * threads * 16;
 }
 
-// layout: kLayoutAny / kLayoutExact / kLayoutFull (0 / 1 / 2)
-constexpr int warp_key(int op, int layout, int chunks) {
-  return (op * 3 + layout) * 16 + chunks;
+// slots: kSlotsTested / kSlotsTail / kSlotsFull (0 / 1 / 2)
+constexpr int warp_key(int op, bool exact, int slots, int chunks) {
+  return ((op * 2 + (exact ? 1 : 0)) * 3 + slots) * 16 + chunks;
 }
-constexpr int cta_key(int op, int layout, int threads, int chunks) {
-  return ((op * 3 + layout) * 2048 + threads) * 8 + chunks;
+constexpr int cta_key(int op, bool exact, int slots, int threads, int chunks) {
+  return (((op * 2 + (exact ? 1 : 0)) * 3 + slots) * 2048 + threads) * 8 + chunks;
 }
 
 constexpr int staged_key(int op, bool wide, bool exact, int threads, int chunks) {
@@ -41,12 +41,12 @@ constexpr int staged_key(int op, bool wide, bool exact, int threads, int chunks)
 // if that configuration is not compiled. op: 0 RMSNorm, 1 LayerNorm. exact:
 // every row of x and y starts 16-byte aligned, dim is a multiple of the
 // 16-byte vector width, and the weight and bias start 16-byte aligned.
-const void* warp_kernel_f32(int op, int layout, int chunks);
-const void* warp_kernel_bf16(int op, int layout, int chunks);
+const void* warp_kernel_f32(int op, bool exact, int slots, int chunks);
+const void* warp_kernel_bf16(int op, bool exact, int slots, int chunks);
 // Kernel entry for (op, exact, threads per block, chunks per thread) in the
 // block family; nullptr if not compiled.
-const void* cta_kernel_f32(int op, int layout, int threads, int chunks);
-const void* cta_kernel_bf16(int op, int layout, int threads, int chunks);
+const void* cta_kernel_f32(int op, bool exact, int slots, int threads, int chunks);
+const void* cta_kernel_bf16(int op, bool exact, int slots, int threads, int chunks);
 // Bulk-copy staged kernels: wide (one block per row) or narrow (lane groups,
 // rows 16-byte aligned); nullptr if not compiled.
 const void* staged_kernel_f32(int op, bool wide, bool exact, int threads, int chunks);

@@ -228,14 +228,14 @@ rows_staged_kernel(const StagedParams p) {
       const bool has_edge = !EXACT && tid < g.nedge;
       float xe = load_edge<T, EXACT>(g, D, tid);
       float rstd, mean;
-      row_stats<T, OP, EXACT, false, VPT>(v, xe, g, D, tid, NT, K, p.eps, has_edge, block_reduce,
+      row_stats<T, OP, EXACT, kSlotsTested, VPT>(v, xe, g, D, tid, NT, K, p.eps, has_edge, block_reduce,
                                           rstd, mean);
       if constexpr (EXACT) {
-        normalize_store<T, OP, EXACT, false, VPT>(s, g, v, xe, direct, tid, NT, rstd, mean,
+        normalize_store<T, OP, EXACT, kSlotsTested, VPT>(s, g, v, xe, direct, tid, NT, rstd, mean,
                                                   has_edge);
       } else {
         if (g.phase != cache.phase) cache.fill(s, g, tid, NT);
-        normalize_store<T, OP, EXACT, false, VPT>(s, g, v, xe, cache, tid, NT, rstd, mean,
+        normalize_store<T, OP, EXACT, kSlotsTested, VPT>(s, g, v, xe, cache, tid, NT, rstd, mean,
                                                   has_edge);
       }
     } else {
@@ -269,9 +269,9 @@ rows_staged_kernel(const StagedParams p) {
         }
         const float K = OP == kOpLn ? Elem<T>::get(reinterpret_cast<const T*>(row)) : 0.f;
         float xe = 0.f, rstd, mean;
-        row_stats<T, OP, true, false, VPT>(v, xe, g, D, gl, G, K, p.eps, false, group_reduce, rstd,
+        row_stats<T, OP, true, kSlotsTested, VPT>(v, xe, g, D, gl, G, K, p.eps, false, group_reduce, rstd,
                                     mean);
-        normalize_store<T, OP, true, false, VPT>(s, g, v, xe, direct, gl, G, rstd, mean, false);
+        normalize_store<T, OP, true, kSlotsTested, VPT>(s, g, v, xe, direct, gl, G, rstd, mean, false);
       }
     }
   }
