@@ -4,7 +4,8 @@ TEST INFRASTRUCTURE. Only the test suite, the entry module's ``smoke()`` and
 the benchmark's CPU-baseline leg use this package. It shares no code with the
 CUDA library (it neither imports it nor is imported by it); the arithmetic
 lives in ``rownorm_oracle.c``, which states what each function follows on the
-pages ("Fused transformer kernels on Emily", "Emily.Fast", "norm_fusion.rs").
+pages ("Fused transformer kernels on Emily", "Emily.Fast", "norm_fusion.rs"),
+including the residual-add and gated RMSNorm fusions of "norm_fusion.rs".
 
 Inputs are numpy arrays (or CPU torch tensors) holding the exact bytes the
 GPU sees: float32 values, or bfloat16 as raw uint16/int16 bit patterns.
@@ -85,9 +86,14 @@ class Oracle:
         lib.oracle_dual_head_rms_norm.argtypes = [
             vp, i64, i64, i64, vp, i64, i64, i64, ctypes.c_int, vp, vp,
             ctypes.c_float, vp, vp, ctypes.c_int]
+        lib.oracle_add_rms_norm.argtypes = [vp, vp, ctypes.c_int, i64, i64, i64, i64,
+                                            vp, ctypes.c_float, vp, vp, ctypes.c_int]
+        lib.oracle_gated_rms_norm.argtypes = [vp, vp, ctypes.c_int, i64, i64, i64, i64,
+                                              vp, ctypes.c_float, vp, ctypes.c_int]
         lib.oracle_decode.argtypes = [vp, ctypes.c_int, i64, vp]
         for fn in (lib.oracle_rms_norm, lib.oracle_layer_norm,
-                   lib.oracle_dual_head_rms_norm):
+                   lib.oracle_dual_head_rms_norm, lib.oracle_add_rms_norm,
+                   lib.oracle_gated_rms_norm):
             fn.restype = ctypes.c_int
         lib.oracle_decode.restype = None
         self._lib = lib
@@ -136,6 +142,39 @@ class Oracle:
             raise ValueError(f"oracle_dual_head_rms_norm rejected its arguments ({st})")
         return yq, yk
 
+    def add_rms_norm(self, x, residual, weight, eps, nthreads=1):
+        """(y, h): h = x + residual stored in the input type (as fp64), and
+        y = RMSNorm(h) * weight, in fp64; both float64 [rows, dim]."""
+        x, rows, dim, xs = _view(x)
+        r, rr, rd, rs = _view(residual)
+        code = _dtype_code(x)
+        if (rr, rd) != (rows, dim) or _dtype_code(r) != code:
+            raise ValueError("x and residual must share shape and dtype")
+        w = _vector(weight, dim, code)
+        y = np.empty((rows, dim), dtype=np.float64)
+        h = np.empty((rows, dim), dtype=np.float64)
+        st = self._lib.oracle_add_rms_norm(_ptr(x), _ptr(r), code, rows, dim, xs, rs,
+                                           _ptr(w), float(eps), _ptr(y), _ptr(h),
+                                           int(nthreads))
+        if st:
+            raise ValueError(f"oracle_add_rms_norm rejected its arguments (status {st})")
+        return y, h
+
+    def gated_rms_norm(self, x, gate, weight, eps, nthreads=1):
+        """RMSNorm(x) * weight * silu(gate) in fp64; float64 [rows, dim]."""
+        x, rows, dim, xs = _view(x)
+        z, zr, zd, zs = _view(gate)
+        code = _dtype_code(x)
+        if (zr, zd) != (rows, dim) or _dtype_code(z) != code:
+            raise ValueError("x and gate must share shape and dtype")
+        w = _vector(weight, dim, code)
+        y = np.empty((rows, dim), dtype=np.float64)
+        st = self._lib.oracle_gated_rms_norm(_ptr(x), _ptr(z), code, rows, dim, xs, zs,
+                                             _ptr(w), float(eps), _ptr(y), int(nthreads))
+        if st:
+            raise ValueError(f"oracle_gated_rms_norm rejected its arguments (status {st})")
+        return y
+
     def decode(self, a):
         """Exact fp64 values of a float32 or bfloat16-bits array."""
         a = np.ascontiguousarray(_as_numpy(a))
@@ -164,6 +203,14 @@ def layer_norm(x, weight, bias, eps, nthreads=1):
 
 def dual_head_rms_norm(q, k, wq, wk, eps, nthreads=1):
     return default().dual_head_rms_norm(q, k, wq, wk, eps, nthreads)
+
+
+def add_rms_norm(x, residual, weight, eps, nthreads=1):
+    return default().add_rms_norm(x, residual, weight, eps, nthreads)
+
+
+def gated_rms_norm(x, gate, weight, eps, nthreads=1):
+    return default().gated_rms_norm(x, gate, weight, eps, nthreads)
 
 
 def decode(a):

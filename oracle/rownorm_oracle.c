@@ -28,11 +28,28 @@
  *                RMSNorm of the key rows with the key weight, one eps shared,
  *                returned queries first, keys second.
  *
+ *   Residual add + RMSNorm -- the elementwise-producer fusion that
+ *                "norm_fusion.rs" (module doc comment) leaves composed until
+ *                a kernel pins the summation order. The composed path adds
+ *                the residual, stores the sum in the tensor's type, then
+ *                normalizes what it stored:
+ *                  h_j = round_T(x_j + r_j)
+ *                  y_j = h_j / sqrt( (1/D) * sum_i h_i^2 + eps ) * w_j
+ *
+ *   Gated RMSNorm -- "norm_fusion.rs" (module doc comment): the output RMS
+ *                normalization chained into the SwiGLU epilogue, i.e. the
+ *                normalized row times the SiLU of the gate:
+ *                  y_j = x_j / sqrt( (1/D) * sum_i x_i^2 + eps ) * w_j
+ *                        * silu(z_j),   silu(t) = t / (1 + exp(-t))
+ *
  * Readings where the pages are silent (each is listed in the design doc):
  *   - the variance divisor is D (population variance);
  *   - eps travels as a binary32 value (norm_fusion.rs keeps it as f32 bits)
  *     and is promoted exactly to fp64 here;
- *   - a null weight means all ones, a null bias all zeros.
+ *   - a null weight means all ones, a null bias all zeros;
+ *   - round_T is round-to-nearest-even to the storage type (binary32, or
+ *     bfloat16: the upper 16 bits of the binary32 value, rounded on the
+ *     16 bits dropped).
  *
  * Inputs are [rows, dim] views whose last axis is contiguous and whose rows
  * start row_stride elements apart. Element type 0 = binary32, 1 = bfloat16
@@ -153,6 +170,103 @@ int oracle_dual_head_rms_norm(const void *q, int64_t q_rows, int64_t q_dim,
     if (status) return status;
     return oracle_rms_norm(k, dtype, k_rows, k_dim, k_stride, wk, eps, yk,
                            nthreads);
+}
+
+/* x + r as the composed path stores it: rounded to nearest, ties to even,
+ * to the storage type. (double)->(float) rounds to nearest-even (the C
+ * default rounding mode); for two binary32 or two bfloat16 operands the
+ * binary32 value is the exact sum rounded once, and bfloat16 rounding then
+ * acts on the 16 low bits the narrower format drops. */
+static double store_round(double s, int dtype) {
+    float f = (float)s;
+    if (dtype == ORACLE_F32) return (double)f;
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7f800000u) == 0x7f800000u) {
+        /* infinity keeps its pattern; NaN stays NaN (quiet bit set) */
+        if (u & 0x007fffffu) u |= 0x00400000u;
+        u &= 0xffff0000u;
+    } else {
+        const uint32_t dropped = u & 0xffffu;
+        const uint32_t kept_lsb = (u >> 16) & 1u;
+        u &= 0xffff0000u;
+        if (dropped > 0x8000u || (dropped == 0x8000u && kept_lsb)) u += 0x10000u;
+    }
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* One residual-add + RMSNorm row: the stored sum, then RMSNorm of it. */
+static void add_rms_norm_row(const void *x, const void *r, int dtype, int64_t row,
+                             int64_t dim, int64_t x_stride, int64_t r_stride,
+                             const void *w, double eps, double *y_row,
+                             double *h_row) {
+    for (int64_t i = 0; i < dim; ++i) {
+        double s = decode_element(x, dtype, row * x_stride + i) +
+                   decode_element(r, dtype, row * r_stride + i);
+        h_row[i] = store_round(s, dtype);
+    }
+    double sum_h2 = 0.0;
+    for (int64_t i = 0; i < dim; ++i) sum_h2 += h_row[i] * h_row[i];
+    double mean_h2 = sum_h2 / (double)dim;
+    double rms_h = sqrt(mean_h2 + eps);
+    for (int64_t j = 0; j < dim; ++j) {
+        double weight = (w != NULL) ? decode_element(w, dtype, j) : 1.0;
+        y_row[j] = h_row[j] / rms_h * weight;
+    }
+}
+
+/* One gated RMSNorm row: RMSNorm, weight, then times silu of the gate. */
+static void gated_rms_norm_row(const void *x, const void *z, int dtype, int64_t row,
+                               int64_t dim, int64_t x_stride, int64_t z_stride,
+                               const void *w, double eps, double *y_row) {
+    double sum_x2 = 0.0;
+    for (int64_t i = 0; i < dim; ++i) {
+        double xv = decode_element(x, dtype, row * x_stride + i);
+        sum_x2 += xv * xv;
+    }
+    double mean_x2 = sum_x2 / (double)dim;
+    double rms_x = sqrt(mean_x2 + eps);
+    for (int64_t j = 0; j < dim; ++j) {
+        double xv = decode_element(x, dtype, row * x_stride + j);
+        double weight = (w != NULL) ? decode_element(w, dtype, j) : 1.0;
+        double gate = decode_element(z, dtype, row * z_stride + j);
+        double silu = gate / (1.0 + exp(-gate));
+        y_row[j] = xv / rms_x * weight * silu;
+    }
+}
+
+int oracle_add_rms_norm(const void *x, const void *r, int dtype, int64_t rows,
+                        int64_t dim, int64_t x_stride, int64_t r_stride,
+                        const void *w, float eps, double *y, double *h,
+                        int nthreads) {
+    int status = check_view(x, dtype, rows, dim, x_stride);
+    if (!status) status = check_view(r, dtype, rows, dim, r_stride);
+    if (status) return status;
+    if (rows > 0 && (y == NULL || h == NULL)) return 1;
+    const double eps64 = (double)eps;
+    (void)nthreads;
+#pragma omp parallel for schedule(static) num_threads(nthreads > 0 ? nthreads : 1)
+    for (int64_t i = 0; i < rows; ++i)
+        add_rms_norm_row(x, r, dtype, i, dim, x_stride, r_stride, w, eps64,
+                         y + i * dim, h + i * dim);
+    return 0;
+}
+
+int oracle_gated_rms_norm(const void *x, const void *z, int dtype, int64_t rows,
+                          int64_t dim, int64_t x_stride, int64_t z_stride,
+                          const void *w, float eps, double *y, int nthreads) {
+    int status = check_view(x, dtype, rows, dim, x_stride);
+    if (!status) status = check_view(z, dtype, rows, dim, z_stride);
+    if (status) return status;
+    if (rows > 0 && y == NULL) return 1;
+    const double eps64 = (double)eps;
+    (void)nthreads;
+#pragma omp parallel for schedule(static) num_threads(nthreads > 0 ? nthreads : 1)
+    for (int64_t i = 0; i < rows; ++i)
+        gated_rms_norm_row(x, z, dtype, i, dim, x_stride, z_stride, w, eps64,
+                           y + i * dim);
+    return 0;
 }
 
 /* Exposed so the test suite can pin the element decoding on its own. */

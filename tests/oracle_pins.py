@@ -14,8 +14,15 @@ Kinds of pin used here:
   invariants       -- unit output RMS, zero mean / unit variance, constant
                       rows give the bias, scale and shift invariance,
                       permutation equivariance, weight/bias linearity;
-  library routines -- torch.nn.functional.layer_norm / rms_norm in fp64;
+  library routines -- torch.nn.functional.layer_norm / rms_norm / silu in
+                      fp64; torch's binary32 -> bfloat16 cast for the
+                      stored residual sum;
   brute force      -- exact rational mean and variance on rows of 1..5.
+
+The residual-add and gated RMSNorm fusions ("norm_fusion.rs", module doc
+comment) are pinned the same ways: the stored sum against a library cast
+(ties included), the normalized output against library routines, a zero gate,
+a closed form with silu(1), and the identity silu(t) - silu(-t) = t.
 """
 import json
 import math
@@ -398,6 +405,128 @@ def pin_bf16_decoding(orc):
     assert np.array_equal(got[~nan], ref[~nan])
     f = np.random.default_rng(41).normal(0, 1e3, 1000).astype(np.float32)
     assert np.array_equal(orc.decode(f), f.astype(np.float64))
+
+
+def _bits_to_bf16(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(bits.astype(np.int16)).view(torch.bfloat16)
+
+
+def pin_add_rms_stored_sum_is_library_cast(orc):
+    # bf16: h = bfloat16(float32(x) + float32(r)) by torch's cast (round to
+    # nearest even), on random rows and on sums built to land exactly on a
+    # bfloat16 midpoint with an even and with an odd kept bit.
+    g = np.random.default_rng(71)
+    x = torch.from_numpy(g.normal(0, 2, (6, 40)).astype(np.float32)).to(torch.bfloat16)
+    r = torch.from_numpy(g.normal(0, 2, (6, 40)).astype(np.float32)).to(torch.bfloat16)
+    # 1 + 2^-8 (tie, kept bit even -> rounds down to 1) and 1 + 3 * 2^-8
+    # (tie, kept bit odd -> rounds up to 1 + 2^-6): x = 1, r = 2^-8 or 3 * 2^-8
+    x[0, :4] = 1.0
+    r[0, 0], r[0, 1] = 2.0 ** -8, 3 * 2.0 ** -8
+    r[0, 2], r[0, 3] = -(2.0 ** -9), 2.0 ** -9 + 2.0 ** -16
+    _, h = orc.add_rms_norm(_bf16_bits(x), _bf16_bits(r), None, 1e-6)
+    want = (x.float() + r.float()).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(h, want), "stored bf16 sum != library cast"
+    assert h[0, 0] == 1.0 and h[0, 1] == 1.0 + 2.0 ** -6, (h[0, 0], h[0, 1])
+    # f32: h = float32 addition
+    xf = g.normal(0, 3, (5, 33)).astype(np.float32)
+    rf = g.normal(0, 3, (5, 33)).astype(np.float32)
+    _, hf = orc.add_rms_norm(xf, rf, None, 1e-6)
+    assert np.array_equal(hf, (xf + rf).astype(np.float64)), "stored f32 sum != f32 add"
+
+
+def pin_add_rms_matches_torch(orc):
+    for dtype in ("f32", "bf16"):
+        x = _rows(72, 7, 96, dtype)
+        r = _rows(73, 7, 96, dtype)
+        w = _rows(74, 1, 96, dtype, mean=1.0, std=0.1).reshape(-1)
+        y, h = orc.add_rms_norm(x, r, w, 1e-5)
+        xt = torch.from_numpy(orc.decode(x))
+        rt = torch.from_numpy(orc.decode(r))
+        ht = (xt.float() + rt.float())
+        if dtype == "bf16":
+            ht = ht.to(torch.bfloat16)
+        ht = ht.double()
+        want = torch.nn.functional.rms_norm(ht, (96,), eps=f32(1e-5)) * \
+            torch.from_numpy(orc.decode(w))
+        _close(y, want.numpy(), 1e-12, 1e-14, f"add_rms vs torch ({dtype})")
+
+
+def pin_add_rms_zero_residual(orc):
+    x = _rows(75, 4, 50, "bf16")
+    y, h = orc.add_rms_norm(x, np.zeros_like(x), None, 1e-6)
+    xt = torch.from_numpy(orc.decode(x))
+    assert np.array_equal(h, xt.numpy()), "x + 0 must store x"
+    want = torch.nn.functional.rms_norm(xt, (50,), eps=f32(1e-6))
+    _close(y, want.numpy(), 1e-12, 1e-14, "add_rms with r = 0")
+
+
+def pin_add_rms_strided_residual(orc):
+    # the residual's rows are read with the residual's own row stride
+    x = _rows(85, 4, 16, "bf16")
+    wide = _rows(86, 4, 27, "bf16")
+    r = wide[:, 5:21]
+    y, h = orc.add_rms_norm(x, r, None, 1e-6)
+    xt = torch.from_numpy(orc.decode(x)).float()
+    rt = torch.from_numpy(orc.decode(np.ascontiguousarray(r))).float()
+    ht = (xt + rt).to(torch.bfloat16).double()
+    assert np.array_equal(h, ht.numpy()), "strided residual: stored sum"
+    want = torch.nn.functional.rms_norm(ht, (16,), eps=f32(1e-6))
+    _close(y, want.numpy(), 1e-12, 1e-14, "add_rms strided residual")
+
+
+def pin_gated_zero_gate(orc):
+    x = _rows(76, 3, 24)
+    y = orc.gated_rms_norm(x, np.zeros_like(x), None, 1e-6)
+    assert np.all(y == 0.0), "silu(0) = 0 must zero the output"
+
+
+def pin_gated_closed_form(orc):
+    # "Emily.Fast" doctest row [1, 2, 3, 4], weight 1, gate 1 everywhere:
+    # y_j = x_j / sqrt(15/2 + eps) * silu(1), silu(1) = 1 / (1 + e^-1).
+    x = np.array([[1, 2, 3, 4]], dtype=np.float32)
+    z = np.ones_like(x)
+    y = orc.gated_rms_norm(x, z, None, 1e-5)
+    silu1 = Decimal(1) / (Decimal(1) + (-Decimal(1)).exp())
+    den = (Decimal(15) / Decimal(2) + Decimal(f32(1e-5))).sqrt()
+    want = [float(Decimal(v) / den * silu1) for v in (1, 2, 3, 4)]
+    _close(y[0], want, 1e-14, 0.0, "gated closed form")
+
+
+def pin_gated_odd_part_is_gate(orc):
+    # silu(t) - silu(-t) = t, so y(z) - y(-z) = RMSNorm(x) * w * z.
+    x = _rows(77, 5, 64)
+    z = _rows(78, 5, 64, std=3.0)
+    w = _rows(79, 1, 64, mean=1.0, std=0.1).reshape(-1)
+    d = orc.gated_rms_norm(x, z, w, 1e-6) - orc.gated_rms_norm(x, -z, w, 1e-6)
+    n = torch.nn.functional.rms_norm(torch.from_numpy(x.astype(np.float64)), (64,),
+                                     eps=f32(1e-6)).numpy()
+    _close(d, n * w.astype(np.float64) * z.astype(np.float64), 1e-12, 1e-14,
+           "gated odd part")
+
+
+def pin_gated_matches_torch(orc):
+    for dtype in ("f32", "bf16"):
+        x = _rows(80, 6, 128, dtype)
+        z = _rows(81, 6, 128, dtype, std=2.0)
+        w = _rows(82, 1, 128, dtype, mean=1.0, std=0.1).reshape(-1)
+        y = orc.gated_rms_norm(x, z, w, 1e-6)
+        xt, zt = torch.from_numpy(orc.decode(x)), torch.from_numpy(orc.decode(z))
+        want = torch.nn.functional.rms_norm(xt, (128,), eps=f32(1e-6)) * \
+            torch.from_numpy(orc.decode(w)) * torch.nn.functional.silu(zt)
+        _close(y, want.numpy(), 1e-12, 1e-14, f"gated vs torch ({dtype})")
+
+
+def pin_gated_strided_gate(orc):
+    # the gate's rows are read with the gate's own row stride
+    x = _rows(83, 4, 16)
+    wide = _rows(84, 4, 24, std=2.0)
+    got = orc.gated_rms_norm(x, wide[:, 3:19], None, 1e-6)
+    want = orc.gated_rms_norm(x, np.ascontiguousarray(wide[:, 3:19]), None, 1e-6)
+    assert np.array_equal(got, want)
+    xt = torch.from_numpy(x.astype(np.float64))
+    zt = torch.from_numpy(np.ascontiguousarray(wide[:, 3:19]).astype(np.float64))
+    ref = torch.nn.functional.rms_norm(xt, (16,), eps=f32(1e-6)) * torch.nn.functional.silu(zt)
+    _close(got, ref.numpy(), 1e-12, 1e-14, "gated strided gate")
 
 
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

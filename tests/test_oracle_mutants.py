@@ -57,6 +57,34 @@ MUTANTS = {
         "oracle_rms_norm(q, dtype, q_rows, q_dim, q_stride, wq, eps, yq,",
         "oracle_rms_norm(q, dtype, q_rows, q_dim, q_stride, wk, eps, yq,"),
     "bf16 decoded with wrong shift": ("(uint32_t)half << 16", "(uint32_t)half << 15"),
+    "add stores the unrounded sum": ("h_row[i] = store_round(s, dtype);", "h_row[i] = s;"),
+    "add ignores the residual": (
+        "double s = decode_element(x, dtype, row * x_stride + i) +\n"
+        "                   decode_element(r, dtype, row * r_stride + i);",
+        "double s = decode_element(x, dtype, row * x_stride + i);"),
+    "add subtracts the residual": (
+        "double s = decode_element(x, dtype, row * x_stride + i) +\n",
+        "double s = decode_element(x, dtype, row * x_stride + i) -\n"),
+    "add residual read with x stride": ("decode_element(r, dtype, row * r_stride + i)",
+                                        "decode_element(r, dtype, row * x_stride + i)"),
+    "bf16 store truncates": (
+        "if (dropped > 0x8000u || (dropped == 0x8000u && kept_lsb)) u += 0x10000u;", ""),
+    "bf16 store ties away from zero": (
+        "if (dropped > 0x8000u || (dropped == 0x8000u && kept_lsb)) u += 0x10000u;",
+        "if (dropped >= 0x8000u) u += 0x10000u;"),
+    "add rms divisor D-1": ("double mean_h2 = sum_h2 / (double)dim;",
+                            "double mean_h2 = sum_h2 / (double)(dim - 1);"),
+    "add rms drops weight": ("y_row[j] = h_row[j] / rms_h * weight;",
+                             "y_row[j] = h_row[j] / rms_h;"),
+    "gated silu sign": ("double silu = gate / (1.0 + exp(-gate));",
+                        "double silu = gate / (1.0 + exp(gate));"),
+    "gated sigmoid only": ("double silu = gate / (1.0 + exp(-gate));",
+                           "double silu = 1.0 / (1.0 + exp(-gate));"),
+    "gated drops eps": ("double rms_x = sqrt(mean_x2 + eps);", "double rms_x = sqrt(mean_x2);"),
+    "gated gate read with x stride": ("decode_element(z, dtype, row * z_stride + j)",
+                                      "decode_element(z, dtype, row * x_stride + j)"),
+    "gated drops weight": ("y_row[j] = xv / rms_x * weight * silu;",
+                           "y_row[j] = xv / rms_x * silu;"),
 }
 
 
