@@ -65,7 +65,7 @@ extern "C" {
 #define RN_API
 #endif
 
-#define RN_ABI_VERSION 1
+#define RN_ABI_VERSION 2
 
 /* Largest supported dim. Rows are held on chip (registers) between reading
  * and writing, so x is read from HBM exactly once; wider rows are rejected
@@ -145,6 +145,44 @@ RN_API int rn_dual_head_rms_norm(const rn_view *q, const rn_view *k,
                                  const rn_view *yq, const rn_view *yk,
                                  void *stream);
 
+/*
+ * Residual add + RMSNorm in one pass ("norm_fusion.rs", module doc comment:
+ * the elementwise-producer fusion kept composed until a kernel pins the
+ * summation order; this library's order is fixed and documented):
+ *   h[r, j] = x[r, j] + residual[r, j], rounded once (nearest, ties to even)
+ *             to the element type and STORED;
+ *   y[r, j] = h[r, j] * rsqrt(mean_i(h[r, i]^2) + eps) * w[j]
+ * The row statistics use the stored h, so y equals rn_rms_norm applied to
+ * h bit for bit (one pass instead of an add kernel, a store and a reload).
+ *   x, residual  input views of one shape and dtype.
+ *   weight       device pointer to dim elements, or NULL (all ones).
+ *   y            output view like x; may be x itself (then not also h).
+ *   h            output view like x for the stored sum; may be x or the
+ *                residual exactly (an in-place residual stream).
+ * Every row of residual and h must start at the same 16-byte phase as the
+ * matching row of x (true for equal shapes and strides); otherwise
+ * RN_ERR_ALIGN. Any other overlap is RN_ERR_OVERLAP. Other errors as
+ * rn_rms_norm; nothing is enqueued on error.
+ */
+RN_API int rn_add_rms_norm(const rn_view *x, const rn_view *residual,
+                           const void *weight, float eps, const rn_view *y,
+                           const rn_view *h, void *stream);
+
+/*
+ * Gated RMSNorm: the output RMS normalization chained into the SwiGLU-style
+ * gate ("norm_fusion.rs", module doc comment), in one pass:
+ *   y[r, j] = ((x[r, j] * rsqrt(mean_i(x[r, i]^2) + eps)) * w[j]) * silu(z[r, j])
+ *   silu(t) = t / (1 + exp(-t)), in binary32, rounded once to the output.
+ *   x, z    input views of one shape and dtype; every row of z starts at the
+ *           same 16-byte phase as the matching row of x (else RN_ERR_ALIGN).
+ *   weight  device pointer to dim elements, or NULL (all ones).
+ *   y       output view like x; may be x itself, must not overlap z.
+ * Other arguments and errors as rn_rms_norm.
+ */
+RN_API int rn_gated_rms_norm(const rn_view *x, const rn_view *z,
+                             const void *weight, float eps, const rn_view *y,
+                             void *stream);
+
 /* Static text for an rn_status value ("unknown status" otherwise). */
 RN_API const char *rn_status_string(int status);
 
@@ -184,12 +222,14 @@ typedef struct rn_launch_info {
     int32_t stage_bytes;    /* staged: bytes per stage                      */
 } rn_launch_info;
 
-enum { RN_OP_RMS = 0, RN_OP_LN = 1, RN_OP_DUAL = 2 };
+enum { RN_OP_RMS = 0, RN_OP_LN = 1, RN_OP_DUAL = 2, RN_OP_ADD_RMS = 3, RN_OP_GATED_RMS = 4 };
 
 /*
  * The launch the library would make for op (RN_OP_*) on these arguments,
  * without launching. For RN_OP_DUAL, x/y are q/yq and x2/y2 are k/yk (the
- * weight and bias arguments are wq and wk); otherwise x2/y2 are ignored.
+ * weight and bias arguments are wq and wk); for RN_OP_ADD_RMS x2/y2 are the
+ * residual and h; for RN_OP_GATED_RMS x2 is the gate; otherwise x2/y2 are
+ * ignored.
  * Queries the current device (SM count, occupancy), so it needs a GPU.
  */
 RN_API int rn_plan(int op, const rn_view *x, const rn_view *y,

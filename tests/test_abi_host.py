@@ -51,7 +51,7 @@ def test_only_declared_symbols_are_exported(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.rn_abi_version() == 1
+    assert lib.rn_abi_version() == 2
     assert lib.rn_status_string(0) == b"ok"
     for st in range(1, 9):
         assert lib.rn_status_string(st) not in (b"ok", b"unknown status")
@@ -198,3 +198,56 @@ def test_cpu_tensors_are_rejected_loudly():
     x = torch.zeros(2, 8)
     with pytest.raises(TypeError, match="CUDA"):
         rn.rms_norm(x, None, 1e-6)
+
+
+def add_rms(lib, x, r, y, h, w=None, eps=1e-6):
+    return lib.rn_add_rms_norm(ctypes.byref(x), ctypes.byref(r) if r is not None else None, w,
+                               eps, ctypes.byref(y), ctypes.byref(h) if h is not None else None,
+                               None)
+
+
+def gated(lib, x, z, y, w=None, eps=1e-6):
+    return lib.rn_gated_rms_norm(ctypes.byref(x), ctypes.byref(z) if z is not None else None, w,
+                                 eps, ctypes.byref(y), None)
+
+
+MB = 1 << 20
+
+
+def test_add_rms_validation(lib):
+    x, r = V(), V(data=FAKE + MB)
+    y, h = V(data=FAKE + 2 * MB), V(data=FAKE + 3 * MB)
+    assert add_rms(lib, x, None, y, h) == 1
+    assert add_rms(lib, x, r, y, None) == 1
+    assert add_rms(lib, x, V(data=FAKE + MB, rows=5), y, h) == 2
+    assert add_rms(lib, x, V(data=FAKE + MB, dtype=0), y, h) == 3
+    assert add_rms(lib, x, r, y, h, eps=float("nan")) == 4
+    # the residual and h must share x's 16-byte phase on every row
+    assert add_rms(lib, x, V(data=FAKE + MB + 2), y, h) == 5
+    assert b"residual" in lib.rn_last_error()
+    assert add_rms(lib, x, r, y, V(data=FAKE + 3 * MB + 8)) == 5
+    assert add_rms(lib, x, V(data=FAKE + MB, stride=65), y, h) == 5
+    # overlaps: y over h, y over the residual, h partly over x or the residual
+    assert add_rms(lib, x, r, V(data=FAKE + 3 * MB), h) == 6
+    assert add_rms(lib, x, r, V(data=FAKE + MB + 64), h) == 6
+    assert add_rms(lib, x, r, y, V(data=FAKE + 64)) == 6
+    assert add_rms(lib, x, r, y, V(data=FAKE + MB + 64)) == 6
+    assert add_rms(lib, x, r, y, h, w=ctypes.c_void_p(FAKE + 3 * MB + 16)) == 6
+    # h may be x or the residual exactly; y may be x unless h is
+    z = dict(rows=0)
+    assert add_rms(lib, V(**z), V(data=FAKE + MB, **z), V(data=FAKE + 2 * MB, **z), V(**z)) == 0
+    assert add_rms(lib, V(**z), V(data=FAKE + MB, **z), V(data=FAKE + 2 * MB, **z),
+                   V(data=FAKE + MB, **z)) == 0
+    assert add_rms(lib, V(**z), V(data=FAKE + MB, **z), V(**z), V(data=FAKE + 3 * MB, **z)) == 0
+
+
+def test_gated_rms_validation(lib):
+    x, zv, y = V(), V(data=FAKE + MB), V(data=FAKE + 2 * MB)
+    assert gated(lib, x, None, y) == 1
+    assert gated(lib, x, V(data=FAKE + MB, dim=32), y) == 2
+    assert gated(lib, x, zv, y, eps=-1.0) == 4
+    assert gated(lib, x, V(data=FAKE + MB + 4), y) == 5
+    assert gated(lib, x, zv, V(data=FAKE + MB)) == 6   # y over the gate
+    assert gated(lib, x, zv, V(data=FAKE + 32)) == 6   # y partly over x
+    z = dict(rows=0)
+    assert gated(lib, V(**z), V(data=FAKE + MB, **z), V(**z)) == 0  # y == x

@@ -11,6 +11,11 @@ LayerNorm adds the bias after the product n*w; where n*w and b nearly cancel
 the exact result is tiny while the binary32 error scales with |n*w| + |b|,
 so LayerNorm also allows an absolute floor 1e-5 * (|n*w| + |b| + 1) (that is
 ~170 binary32 ulps of the operands, far below one bf16 ulp of them).
+
+Gated RMSNorm in fp32 (``scaled=True``): its outputs reach |y| ~ 40 (the gate's
+silu grows like the gate), where a fixed 1e-5 is below the binary32 error of
+the product chain itself (four roundings, expf within 2 ulps, a divide:
+about 1e-6 relative). Its bound is 1e-5 * (1 + |y|), ten times that error.
 """
 import numpy as np
 import torch
@@ -27,14 +32,18 @@ def to_f64(t):
     return t.detach().to("cpu").double().numpy()
 
 
-def check(gpu, ref, dtype, bias=None, what=""):
+def check(gpu, ref, dtype, bias=None, what="", scaled=False):
     """Assert parity; returns (max_abs_err, max_err_in_ulps or None)."""
     got = to_f64(gpu).reshape(ref.shape)
     err = np.abs(got - ref)
     assert np.all(np.isfinite(got) == np.isfinite(ref)), f"{what}: finiteness differs"
     if dtype == torch.float32:
         worst = float(err.max()) if err.size else 0.0
-        assert worst <= 1e-5, f"{what}: max abs err {worst:.3e} > 1e-5"
+        if scaled:
+            bad = err > 1e-5 * (1.0 + np.abs(ref))
+            assert not bad.any(), f"{what}: {int(bad.sum())} elements beyond 1e-5 * (1 + |y|)"
+        else:
+            assert worst <= 1e-5, f"{what}: max abs err {worst:.3e} > 1e-5"
         return worst, None
     ulp = bf16_ulp(ref)
     bound = ulp.copy()

@@ -28,7 +28,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "librownorm.so")
 
 RN_F32, RN_BF16 = 0, 1
-RN_OP_RMS, RN_OP_LN, RN_OP_DUAL = 0, 1, 2
+RN_OP_RMS, RN_OP_LN, RN_OP_DUAL, RN_OP_ADD_RMS, RN_OP_GATED_RMS = 0, 1, 2, 3, 4
 STATUS_NAMES = {0: "RN_OK", 1: "RN_ERR_NULL", 2: "RN_ERR_SHAPE", 3: "RN_ERR_DTYPE",
                 4: "RN_ERR_EPS", 5: "RN_ERR_ALIGN", 6: "RN_ERR_OVERLAP",
                 7: "RN_ERR_UNSUPPORTED", 8: "RN_ERR_CUDA"}
@@ -74,6 +74,8 @@ def load_library():
         lib.rn_rms_norm.argtypes = [pv, vp, f32, pv, vp]
         lib.rn_layer_norm.argtypes = [pv, vp, vp, f32, pv, vp]
         lib.rn_dual_head_rms_norm.argtypes = [pv, pv, vp, vp, f32, pv, pv, vp]
+        lib.rn_add_rms_norm.argtypes = [pv, pv, vp, f32, pv, pv, vp]
+        lib.rn_gated_rms_norm.argtypes = [pv, pv, vp, f32, pv, vp]
         lib.rn_plan.argtypes = [ctypes.c_int, pv, pv, pv, pv, vp, vp,
                                 ctypes.POINTER(rn_launch_info)]
         lib.rn_set_grid_override.argtypes = [ctypes.c_int]
@@ -84,7 +86,7 @@ def load_library():
         lib.rn_last_error.argtypes = []
         lib.rn_last_error.restype = ctypes.c_char_p
         for fn in (lib.rn_rms_norm, lib.rn_layer_norm, lib.rn_dual_head_rms_norm,
-                   lib.rn_plan, lib.rn_set_grid_override, lib.rn_abi_version,
+                   lib.rn_add_rms_norm, lib.rn_gated_rms_norm, lib.rn_plan, lib.rn_set_grid_override, lib.rn_abi_version,
                    lib.rn_set_path_override, lib.rn_device_error_count):
             fn.restype = ctypes.c_int
         _lib = lib
@@ -206,13 +208,47 @@ def rn_dual_head_rms_norm(q, k, wq, wk, eps=1e-6, out_q=None, out_k=None, stream
     return out_q, out_k
 
 
+def rn_add_rms_norm(x, residual, weight, eps=1e-6, out=None, out_h=None, stream=None):
+    """(y, h): h = x + residual stored in x's dtype, y = RMSNorm(h) * weight, in
+    one pass. ``out_h`` may be ``x`` or ``residual`` (in-place residual stream)."""
+    import torch
+    _require_cuda(x, residual, weight, out, out_h)
+    out = torch.empty_like(x) if out is None else out
+    out_h = torch.empty_like(x) if out_h is None else out_h
+    xv, rv, yv, hv = _view(x), _view(residual), _view(out), _view(out_h)
+    lib = load_library()
+    with torch.cuda.device(x.device):
+        _check(lib.rn_add_rms_norm(ctypes.byref(xv), ctypes.byref(rv),
+                                   _vector(weight, xv.dim, x), float(eps), ctypes.byref(yv),
+                                   ctypes.byref(hv), _stream(x, stream)))
+    return out, out_h
+
+
+def rn_gated_rms_norm(x, z, weight, eps=1e-6, out=None, stream=None):
+    """RMSNorm(x) * weight * silu(z) over the last axis, in one pass."""
+    import torch
+    _require_cuda(x, z, weight, out)
+    out = torch.empty_like(x) if out is None else out
+    xv, zv, yv = _view(x), _view(z), _view(out)
+    lib = load_library()
+    with torch.cuda.device(x.device):
+        _check(lib.rn_gated_rms_norm(ctypes.byref(xv), ctypes.byref(zv),
+                                     _vector(weight, xv.dim, x), float(eps), ctypes.byref(yv),
+                                     _stream(x, stream)))
+    return out
+
+
 rms_norm = rn_rms_norm
 layer_norm = rn_layer_norm
 dual_head_rms_norm = rn_dual_head_rms_norm
+add_rms_norm = rn_add_rms_norm
+gated_rms_norm = rn_gated_rms_norm
 
 
 def plan(op, x, out=None, weight=None, bias=None, k=None, out_k=None):
-    """The launch configuration the library picks (see rn_launch_info)."""
+    """The launch configuration the library picks (see rn_launch_info). For
+    RN_OP_ADD_RMS ``k`` is the residual and ``out_k`` the stored sum h; for
+    RN_OP_GATED_RMS ``k`` is the gate."""
     import torch
     out = torch.empty_like(x) if out is None else out
     xv, yv = _view(x), _view(out)
@@ -225,6 +261,12 @@ def plan(op, x, out=None, weight=None, bias=None, k=None, out_k=None):
             _check(lib.rn_plan(op, ctypes.byref(xv), ctypes.byref(yv), ctypes.byref(kv),
                                ctypes.byref(ykv), _vector(weight, xv.dim, x),
                                _vector(bias, kv.dim, k), ctypes.byref(info)))
+        elif op in (RN_OP_ADD_RMS, RN_OP_GATED_RMS):
+            out_k = torch.empty_like(x) if out_k is None else out_k
+            kv, ykv = _view(k), _view(out_k)
+            _check(lib.rn_plan(op, ctypes.byref(xv), ctypes.byref(yv), ctypes.byref(kv),
+                               ctypes.byref(ykv), _vector(weight, xv.dim, x), None,
+                               ctypes.byref(info)))
         else:
             _check(lib.rn_plan(op, ctypes.byref(xv), ctypes.byref(yv), None, None,
                                _vector(weight, xv.dim, x), _vector(bias, xv.dim, x),

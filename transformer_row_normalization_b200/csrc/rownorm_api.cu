@@ -318,7 +318,7 @@ bool plan_staged(int dtype, int op, const SegPlan* plans, const rn_view* const* 
   // HBM bandwidth than this staged pipeline at every shape tried (the staged
   // kernel keeps more bytes in flight but runs fewer warps per SM and pays a
   // block barrier per tile). The staged kernel stays selectable.
-  if (g_path_override != 2) return false;
+  if (g_path_override != 2 || rn::op_has_second(op)) return false;
   const int es = elem_size(dtype);
   const bool wide = plans[0].family == 1;
   for (int i = 0; i < nseg; ++i) {
@@ -428,8 +428,9 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
   const int threads = merged.family == 0 ? rn::kWarpBlock : merged.lanes;
   const int cache = merged.exact ? 0 : rn::affine_cache_smem_bytes(op, threads, merged.chunks);
   const int pf_bytes = rn::prefetch_slots_smem_bytes(
-      threads, merged.chunks,
-      merged.family == 0 ? rn::kWarpPrefetchStages : rn::kCtaPrefetchStages);
+                           threads, merged.chunks,
+                           merged.family == 0 ? rn::kWarpPrefetchStages : rn::kCtaPrefetchStages) *
+                       (rn::op_has_second(op) ? 2 : 1);
   // Next-row prefetch where it measured faster on B200: lane-group rows and
   // blocks of 256 or more threads (few blocks per SM, so few rows in
   // flight); blocks of 128 threads already keep 8+ rows per SM in flight and
@@ -493,6 +494,8 @@ rn::Segment make_segment(const rn_view* x, const rn_view* y, const void* w, cons
   s.dim = (int)x->dim;
   s.lanes = p.lanes;
   s.vector_y = p.vector_y;
+  s.x2 = nullptr;
+  s.h = nullptr;
   return s;
 }
 
@@ -606,6 +609,74 @@ int run_dual(const rn_view* q, const rn_view* k, const void* wq, const void* wk,
   return launch(l, params, stream);
 }
 
+// Every row of `v` starts at the same 16-byte phase as the matching row of x.
+bool same_phase(const rn_view* x, const rn_view* v) {
+  const int es = elem_size(x->dtype);
+  const uintptr_t xa = reinterpret_cast<uintptr_t>(x->data);
+  const uintptr_t va = reinterpret_cast<uintptr_t>(v->data);
+  return ((va - xa) % 16 == 0) &&
+         (x->rows <= 1 || (((v->row_stride - x->row_stride) * es) % 16 == 0));
+}
+
+// Residual add + RMSNorm (op kOpAddRms: x2 = residual, h = stored sum) and
+// gated RMSNorm (kOpGatedRms: x2 = gate, h unused).
+int run_second(int op, const rn_view* x, const rn_view* x2, const void* w, float eps,
+               const rn_view* y, const rn_view* h, void* stream, rn_launch_info* plan_only) {
+  const bool add = op == rn::kOpAddRms;
+  const char* x2n = add ? "residual" : "z";
+  int st;
+  if ((st = check_view(x, "x"))) return st;
+  if ((st = check_view(x2, x2n))) return st;
+  if ((st = check_view(y, "y"))) return st;
+  if (add && (st = check_view(h, "h"))) return st;
+  if ((st = check_pair(x, x2, "x", x2n))) return st;
+  if ((st = check_pair(x, y, "x", "y"))) return st;
+  if (add && (st = check_pair(x, h, "x", "h"))) return st;
+  if ((st = check_eps(eps))) return st;
+  if ((st = check_vector(w, x->dtype, "weight"))) return st;
+  if (!same_phase(x, x2))
+    return fail(RN_ERR_ALIGN, "%s rows must share x's 16-byte alignment", x2n);
+  if (add && !same_phase(x, h))
+    return fail(RN_ERR_ALIGN, "h rows must share x's 16-byte alignment");
+  const void* vecs[1] = {w};
+  const int64_t dims[1] = {x->dim};
+  // y may be x itself; it must not touch the second input, h or the weight
+  const rn_view* not_y[2] = {x2, h};
+  if ((st = check_output(y, x, not_y, add ? 2 : 1, vecs, dims, 1, "y"))) return st;
+  if (add) {
+    // h may be x or the residual exactly (an in-place residual stream)
+    const Span sh = span_of(h);
+    if (intersects(sh, span_of(x)) && !same_view(h, x))
+      return fail(RN_ERR_OVERLAP, "h partially overlaps x");
+    if (intersects(sh, span_of(x2)) && !same_view(h, x2))
+      return fail(RN_ERR_OVERLAP, "h partially overlaps the residual");
+    if (w && intersects(sh, span_of_vector(w, x->dim, x->dtype)))
+      return fail(RN_ERR_OVERLAP, "h overlaps the weight");
+  }
+  if (x->rows == 0 && !plan_only) return RN_OK;
+  const SegPlan p = plan_segment(x, y, w, nullptr);
+  Launch l{};
+  const rn_view* xs[1] = {x};
+  const void* ws[1] = {w};
+  const void* bs[1] = {nullptr};
+  if ((st = plan_launch(x->dtype, op, &p, xs, ws, bs, 1, &l))) return st;
+  if (plan_only) {
+    *plan_only = l.info;
+    return RN_OK;
+  }
+  rn::Params params{};
+  params.seg[0] = make_segment(x, y, w, nullptr, p);
+  params.seg[0].x2 = x2->data;
+  params.seg[0].x2_stride = x2->rows > 1 ? x2->row_stride : x2->dim;
+  if (add) {
+    params.seg[0].h = h->data;
+    params.seg[0].h_stride = h->rows > 1 ? h->row_stride : h->dim;
+  }
+  params.nseg = 1;
+  params.eps = eps;
+  return launch(l, params, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -618,6 +689,16 @@ RN_API int rn_rms_norm(const rn_view* x, const void* weight, float eps, const rn
 RN_API int rn_layer_norm(const rn_view* x, const void* weight, const void* bias, float eps,
                          const rn_view* y, void* stream) {
   return run_single(rn::kOpLn, x, weight, bias, eps, y, stream, nullptr);
+}
+
+RN_API int rn_add_rms_norm(const rn_view* x, const rn_view* residual, const void* weight,
+                           float eps, const rn_view* y, const rn_view* h, void* stream) {
+  return run_second(rn::kOpAddRms, x, residual, weight, eps, y, h, stream, nullptr);
+}
+
+RN_API int rn_gated_rms_norm(const rn_view* x, const rn_view* z, const void* weight, float eps,
+                             const rn_view* y, void* stream) {
+  return run_second(rn::kOpGatedRms, x, z, weight, eps, y, nullptr, stream, nullptr);
 }
 
 RN_API int rn_dual_head_rms_norm(const rn_view* q, const rn_view* k, const void* wq,
@@ -652,6 +733,10 @@ RN_API int rn_plan(int op, const rn_view* x, const rn_view* y, const rn_view* x2
   if (op == RN_OP_DUAL) return run_dual(x, x2, weight, bias, 1e-6f, y, y2, nullptr, info);
   if (op == RN_OP_RMS) return run_single(rn::kOpRms, x, weight, nullptr, 1e-6f, y, nullptr, info);
   if (op == RN_OP_LN) return run_single(rn::kOpLn, x, weight, bias, 1e-6f, y, nullptr, info);
+  if (op == RN_OP_ADD_RMS)
+    return run_second(rn::kOpAddRms, x, x2, weight, 1e-6f, y, y2, nullptr, info);
+  if (op == RN_OP_GATED_RMS)
+    return run_second(rn::kOpGatedRms, x, x2, weight, 1e-6f, y, nullptr, nullptr, info);
   return fail(RN_ERR_UNSUPPORTED, "unknown op %d", op);
 }
 

@@ -15,6 +15,13 @@
 //   The page calls its LayerNorm statistic "Welford-style"; the two passes
 //   here run over a row already on chip, so they cost no extra HBM traffic
 //   and give the same population mean and variance.
+//   Residual add + RMSNorm and gated RMSNorm ("norm_fusion.rs", module doc
+//   comment: the elementwise fusions kept composed until a kernel pins the
+//   summation order, which this one does):
+//               h_j  = round_T(x_j + r_j)        (stored; the row statistics
+//               y_j  = (h_j * rstd) * w_j          use the stored values)
+//               y_j  = ((x_j * rstd) * w_j) * silu(z_j),
+//               silu(t) = t / (1 + exp(-t))       (binary32, expf called)
 //
 // Row layout. A row is moved as 16-byte chunks on the 16-byte address grid:
 // the columns between the first and the last 16-byte boundary inside the row
@@ -48,7 +55,13 @@
 
 namespace rn {
 
-enum : int { kOpRms = 0, kOpLn = 1 };
+enum : int { kOpRms = 0, kOpLn = 1, kOpAddRms = 2, kOpGatedRms = 3 };
+
+// A second input row space read beside x: the residual (kOpAddRms) or the
+// gate (kOpGatedRms).
+__host__ __device__ constexpr bool op_has_second(int op) {
+  return op == kOpAddRms || op == kOpGatedRms;
+}
 
 // Which of a thread's NSLOT chunk slots the planner guarantees present in
 // every row of a launch:
@@ -80,6 +93,12 @@ struct Segment {
   int lanes;       // threads per row in the lane-group kernels (power of two <= 32)
   int vector_y;    // 1: every y row has its x row's 16-byte phase
   int pad_;
+  // second input and stored sum (kOpAddRms: residual r and h = x + r;
+  // kOpGatedRms: gate z); every row shares its x row's 16-byte phase
+  const void* x2;
+  void* h;
+  long long x2_stride;
+  long long h_stride;
 };
 
 // ---------------------------------------------------------------------------
@@ -113,6 +132,13 @@ __device__ __forceinline__ float hsum2(F2 a) {
   return __fadd_rn(lo, hi);
 }
 
+// silu(t) = t / (1 + exp(-t)) in binary32, with CUDA's expf and a correctly
+// rounded divide.
+__device__ __forceinline__ float silu(float t) {
+  return __fdiv_rn(t, __fadd_rn(1.f, expf(-t)));
+}
+__device__ __forceinline__ F2 silu2(F2 t) { return make2(silu(t.x), silu(t.y)); }
+
 // ---------------------------------------------------------------------------
 // element types: a 16-byte chunk <-> P = V/2 binary32 pairs
 
@@ -129,6 +155,8 @@ struct Elem<float> {
     return __float_as_uint(*p);
   }
   static __device__ __forceinline__ void put(float* p, float v) { *p = v; }
+  // v as stored: binary32 already is
+  static __device__ __forceinline__ float stored(float v) { return v; }
   static __device__ __forceinline__ void unpack(const uint4& u, F2 (&f)[2]) {
     f[0] = make2_bits(u.x, u.y);
     f[1] = make2_bits(u.z, u.w);
@@ -155,6 +183,10 @@ struct Elem<__nv_bfloat16> {
   }
   static __device__ __forceinline__ void put(__nv_bfloat16* p, float v) {
     *p = __float2bfloat16_rn(v);
+  }
+  // v rounded to bfloat16 (nearest, ties to even), widened back exactly
+  static __device__ __forceinline__ float stored(float v) {
+    return __bfloat162float(__float2bfloat16_rn(v));
   }
   // bfloat16 is the upper half of a binary32 pattern: widening is exact bit
   // placement (low element: shift up; high element: clear the low half).
@@ -514,13 +546,22 @@ constexpr int affine_cache_bytes(int threads) {
   return threads * NSLOT * 16 * (BIAS ? 2 : 1);
 }
 
+// No gate (every op but kOpGatedRms).
+struct NoGate {
+  template <int P>
+  __device__ __forceinline__ void get(int, int, F2 (&)[P]) const {}
+  __device__ __forceinline__ float edge() const { return 0.f; }
+};
+
 // Normalize the thread's chunks and edge element of one row, apply weight
-// (and bias), store.
-template <typename T, int OP, bool EXACT, int SLOTS, int NSLOT, typename Src>
+// (and bias, or the gate's silu), store.
+template <typename T, int OP, bool EXACT, int SLOTS, int NSLOT, typename Src,
+          typename Gate = NoGate>
 __device__ __forceinline__ void normalize_store(const Segment& s, const Row<T>& g,
                                                 const F2 (&v)[NSLOT][Elem<T>::P], float xe,
                                                 const Src& src, int k0, int step, float rstd,
-                                                float mean, bool has_edge) {
+                                                float mean, bool has_edge,
+                                                const Gate& gate = Gate()) {
   constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
   const F2 R2 = splat(rstd);
@@ -533,10 +574,16 @@ __device__ __forceinline__ void normalize_store(const Segment& s, const Row<T>& 
     src.get(p, f, wf, bf);
 #pragma unroll
     for (int j = 0; j < P; ++j) {
-      if constexpr (OP == kOpRms)
-        o[j] = mul2(mul2(v[p][j], R2), wf[j]);
-      else
+      if constexpr (OP == kOpLn)
         o[j] = fma2(mul2(sub2(v[p][j], M2), R2), wf[j], bf[j]);
+      else
+        o[j] = mul2(mul2(v[p][j], R2), wf[j]);
+    }
+    if constexpr (OP == kOpGatedRms) {
+      F2 zf[P];
+      gate.template get<P>(p, f, zf);
+#pragma unroll
+      for (int j = 0; j < P; ++j) o[j] = mul2(o[j], silu2(zf[j]));
     }
     T* yc = g.y_row + g.head + (long long)f * V;
     if (EXACT || s.vector_y) {
@@ -554,9 +601,9 @@ __device__ __forceinline__ void normalize_store(const Segment& s, const Row<T>& 
   if (!EXACT && has_edge) {
     float we, be;
     src.edge(we, be);
-    const float o = OP == kOpRms
-                        ? __fmul_rn(__fmul_rn(xe, rstd), we)
-                        : __fmaf_rn(__fmul_rn(__fsub_rn(xe, mean), rstd), we, be);
+    float o = OP == kOpLn ? __fmaf_rn(__fmul_rn(__fsub_rn(xe, mean), rstd), we, be)
+                          : __fmul_rn(__fmul_rn(xe, rstd), we);
+    if constexpr (OP == kOpGatedRms) o = __fmul_rn(o, silu(gate.edge()));
     Elem<T>::put(g.y_row + edge_column(g, s.dim, k0), o);
   }
 }
@@ -571,7 +618,7 @@ __device__ __forceinline__ void row_stats(F2 (&v)[NSLOT][Elem<T>::P], float& xe,
   // Means are sums times 1/D rounded to binary32 (one multiply instead of a
   // divide per row; exact for power-of-two D, within 2 ulps otherwise).
   const float inv_d = __frcp_rn((float)D);
-  if (OP == kOpRms) {
+  if (OP != kOpLn) {
     const float ss = reduce(sum_squares<T, EXACT, NSLOT>(v, xe, has_edge));
     mean = 0.f;
     rstd = rsqrtf(__fadd_rn(__fmul_rn(ss, inv_d), eps));

@@ -48,41 +48,49 @@ constexpr int kWarpBlock = 256;
 constexpr int kMinThreadsPerSmWarp = 768;
 constexpr int kMinThreadsPerSm = 1024;
 
-// Per-thread prefetch slots: [stages][NSLOT][blockDim.x] 16-byte words.
-// When the slots do not fit in shared memory next to the weight cache (the
-// planner decides), `on` is 0: nothing is copied ahead and rows are loaded
-// straight from global memory when they are taken.
+// Per-thread prefetch slots: [stages][NSLOT][blockDim.x] 16-byte words
+// from 16-byte word `base` of the dynamic shared memory (a second bank
+// follows the first for ops with a second input). When the slots do not fit
+// in shared memory next to the weight cache (the planner decides), `on` is
+// 0: nothing is copied ahead and rows are loaded straight from global memory
+// when they are taken.
 template <typename T, int NSLOT>
 struct Prefetch {
   int on;
+  int base;
   __device__ __forceinline__ uint4* slot(int stage, int p) const {
-    return &dyn_smem[(stage * NSLOT + p) * blockDim.x + threadIdx.x];
+    return &dyn_smem[base + (stage * NSLOT + p) * blockDim.x + threadIdx.x];
   }
-  // Start the copies of the thread's full chunks of row g into `stage`.
+  // Start the copies of the thread's full chunks of a row (first full chunk
+  // at `full`) into `stage`.
   template <int SLOTS>
-  __device__ __forceinline__ void issue(const Row<T>& g, int k0, int step, int stage) const {
+  __device__ __forceinline__ void issue(const T* full, int nfull, int k0, int step,
+                                        int stage) const {
     constexpr int V = Elem<T>::V;
     if (!on) return;
 #pragma unroll
     for (int p = 0; p < NSLOT; ++p) {
       const int f = k0 + step * p;
-      if (slot_present<SLOTS, NSLOT>(p, f, g.nfull))
-        cp_async16(slot(stage, p), g.x_full + (long long)f * V);
+      if (slot_present<SLOTS, NSLOT>(p, f, nfull))
+        cp_async16(slot(stage, p), full + (long long)f * V);
     }
   }
-  // The thread's slots of row g from `stage` (copies complete); absent ones zero.
+  // Slot p of the row in `stage` (copy complete), or straight from global
+  // memory when nothing was copied ahead.
+  __device__ __forceinline__ uint4 chunk(const T* full, int f, int stage, int p) const {
+    constexpr int V = Elem<T>::V;
+    return on ? *slot(stage, p) : load_stream(full + (long long)f * V);
+  }
+  // The thread's slots of a row; absent ones zero.
   template <int SLOTS>
-  __device__ __forceinline__ void take(const Row<T>& g, int k0, int step, int stage,
+  __device__ __forceinline__ void take(const T* full, int nfull, int k0, int step, int stage,
                                        F2 (&v)[NSLOT][Elem<T>::P]) const {
     constexpr int P = Elem<T>::P;
-    if (!on) {
-      load_row<T, SLOTS, NSLOT>(g, k0, step, v);
-      return;
-    }
 #pragma unroll
     for (int p = 0; p < NSLOT; ++p) {
-      if (slot_present<SLOTS, NSLOT>(p, k0 + step * p, g.nfull)) {
-        Elem<T>::unpack(*slot(stage, p), v[p]);
+      const int f = k0 + step * p;
+      if (slot_present<SLOTS, NSLOT>(p, f, nfull)) {
+        Elem<T>::unpack(chunk(full, f, stage, p), v[p]);
       } else {
 #pragma unroll
         for (int j = 0; j < P; ++j) v[p][j] = zero2();
@@ -98,37 +106,76 @@ struct Prefetch {
 constexpr int kWarpPrefetchStages = 2;
 constexpr int kCtaPrefetchStages = 2;
 
-// 16-byte words of prefetch slots.
+// 16-byte words of prefetch slots of one bank.
 template <int NSLOT, int NST>
 __host__ __device__ constexpr int prefetch_smem_words(int threads) {
   return NST * NSLOT * threads;
 }
 
+template <typename T>
+__device__ __forceinline__ const T* x2_row_of(const Segment& s, long long r) {
+  return static_cast<const T*>(s.x2) + r * s.x2_stride;
+}
+
+// The edge element of thread k0 in a row of a second row space that shares
+// x's 16-byte phase (0 when it owns none).
+template <typename T, bool EXACT>
+__device__ __forceinline__ float load_edge_at(const T* row, const Row<T>& g, int D, int k0) {
+  if constexpr (EXACT) return 0.f;
+  return k0 < g.nedge ? Elem<T>::get(row + edge_column(g, D, k0)) : 0.f;
+}
+
+// The gate's chunks for the store (kOpGatedRms): from the second prefetch
+// bank, or global memory, and its edge element.
+template <typename T, int NSLOT>
+struct GateSrc {
+  const Prefetch<T, NSLOT>* pf;
+  const T* full;
+  int stage;
+  float ze;
+  template <int P>
+  __device__ __forceinline__ void get(int p, int f, F2 (&zf)[P]) const {
+    Elem<T>::unpack(pf->chunk(full, f, stage, p), zf);
+  }
+  __device__ __forceinline__ float edge() const { return ze; }
+};
+
 // The rows r0, r0 + stride, ... of one segment, owned by one thread group (a
 // lane group, or a block) in which this thread is k0 of `step`. Each row's
-// chunks are prefetched NST - 1 rows ahead, stage i % NST holding row i;
-// the shift K and the thread's edge element of the rows ahead wait in
-// register queues. `src` supplies weight and bias.
+// chunks (and those of the second input) are prefetched NST - 1 rows ahead,
+// stage i % NST holding row i; the shift K and the thread's edge elements of
+// the rows ahead wait in register queues. `src` supplies weight and bias.
 template <typename T, int OP, bool EXACT, int SLOTS, int NSLOT, int NST, typename Src,
           typename Reduce>
 __device__ __forceinline__ void segment_rows(const Segment& s, const Prefetch<T, NSLOT>& pf,
-                                             long long r0, long long stride, int k0, int step,
-                                             float eps, Reduce reduce, Src& src) {
+                                             const Prefetch<T, NSLOT>& pf2, long long r0,
+                                             long long stride, int k0, int step, float eps,
+                                             Reduce reduce, Src& src) {
   static_assert(NST >= 2, "at least one row ahead");
+  constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
+  constexpr bool SECOND = op_has_second(OP);
   const int D = s.dim;
-  float Kq[NST - 1], Eq[NST - 1];
+  float Kq[NST - 1], Eq[NST - 1], E2q[NST - 1];
+  // queue the loads of row ra into stage `stage`
+  auto ahead = [&](long long ra, int stage, int j) {
+    const Row<T> ga = row_geometry<T, EXACT>(s, ra);
+    pf.template issue<SLOTS>(ga.x_full, ga.nfull, k0, step, stage);
+    if (OP == kOpLn) Kq[j] = Elem<T>::get(ga.x_row);
+    Eq[j] = load_edge<T, EXACT>(ga, D, k0);
+    if constexpr (SECOND) {
+      const T* row2 = x2_row_of<T>(s, ra);
+      pf2.template issue<SLOTS>(row2 + ga.head, ga.nfull, k0, step, stage);
+      E2q[j] = load_edge_at<T, EXACT>(row2, ga, D, k0);
+    }
+  };
 #pragma unroll
   for (int j = 0; j < NST - 1; ++j) {
     const long long rj = r0 + j * stride;
     Kq[j] = 0.f;
     Eq[j] = 0.f;
-    if (rj < s.rows) {
-      const Row<T> gj = row_geometry<T, EXACT>(s, rj);
-      pf.template issue<SLOTS>(gj, k0, step, j);
-      if (OP == kOpLn) Kq[j] = Elem<T>::get(gj.x_row);
-      Eq[j] = load_edge<T, EXACT>(gj, D, k0);
-    }
+    E2q[j] = 0.f;
+    if (rj < s.rows) ahead(rj, j, j);
     cp_async_commit();
   }
   int st = 0;  // stage of row r
@@ -136,34 +183,64 @@ __device__ __forceinline__ void segment_rows(const Segment& s, const Prefetch<T,
   for (long long r = r0; r < s.rows; r += stride) {
     const float K = Kq[0];
     float xe = Eq[0];
+    const float x2e = E2q[0];
 #pragma unroll
     for (int j = 0; j + 1 < NST - 1; ++j) {
       Kq[j] = Kq[j + 1];
       Eq[j] = Eq[j + 1];
+      E2q[j] = E2q[j + 1];
     }
     // the stage the previous row was taken from receives row r + (NST-1) stride
     const int sa = st == 0 ? NST - 1 : st - 1;
     const long long ra = r + (NST - 1) * stride;
-    if (ra < s.rows) {
-      const Row<T> ga = row_geometry<T, EXACT>(s, ra);
-      pf.template issue<SLOTS>(ga, k0, step, sa);
-      if (OP == kOpLn) Kq[NST - 2] = Elem<T>::get(ga.x_row);
-      Eq[NST - 2] = load_edge<T, EXACT>(ga, D, k0);
-    }
+    if (ra < s.rows) ahead(ra, sa, NST - 2);
     cp_async_commit();
     cp_async_wait<NST - 1>();
     const Row<T> g = row_geometry<T, EXACT>(s, r);
     const bool has_edge = !EXACT && k0 < g.nedge;
     F2 v[NSLOT][P];
-    pf.template take<SLOTS>(g, k0, step, st, v);
+    if constexpr (OP == kOpAddRms) {
+      // h = x + r rounded to T: stored, and what the row statistics see
+      const T* full2 = x2_row_of<T>(s, r) + g.head;
+      T* hrow = static_cast<T*>(s.h) + r * s.h_stride;
+#pragma unroll
+      for (int p = 0; p < NSLOT; ++p) {
+        const int f = k0 + step * p;
+        if (slot_present<SLOTS, NSLOT>(p, f, g.nfull)) {
+          F2 a[P], b[P];
+          Elem<T>::unpack(pf.chunk(g.x_full, f, st, p), a);
+          Elem<T>::unpack(pf2.chunk(full2, f, st, p), b);
+#pragma unroll
+          for (int j = 0; j < P; ++j) a[j] = add2(a[j], b[j]);
+          const uint4 hv = Elem<T>::pack(a);
+          store_stream(hrow + g.head + (long long)f * V, hv);
+          Elem<T>::unpack(hv, v[p]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < P; ++j) v[p][j] = zero2();
+        }
+      }
+      if (has_edge) {
+        xe = Elem<T>::stored(__fadd_rn(xe, x2e));
+        Elem<T>::put(hrow + edge_column(g, D, k0), xe);
+      }
+    } else {
+      pf.template take<SLOTS>(g.x_full, g.nfull, k0, step, st, v);
+    }
     float rstd, mean;
     row_stats<T, OP, EXACT, SLOTS, NSLOT>(v, xe, g, D, k0, step, K, eps, has_edge, reduce, rstd,
                                           mean);
     if constexpr (!EXACT) {
       if (g.phase != src.phase) src.fill(s, g, k0, step);
     }
-    normalize_store<T, OP, EXACT, SLOTS, NSLOT>(s, g, v, xe, src, k0, step, rstd, mean,
-                                                has_edge);
+    if constexpr (OP == kOpGatedRms) {
+      const GateSrc<T, NSLOT> gate{&pf2, x2_row_of<T>(s, r) + g.head, st, x2e};
+      normalize_store<T, OP, EXACT, SLOTS, NSLOT>(s, g, v, xe, src, k0, step, rstd, mean,
+                                                  has_edge, gate);
+    } else {
+      normalize_store<T, OP, EXACT, SLOTS, NSLOT>(s, g, v, xe, src, k0, step, rstd, mean,
+                                                  has_edge);
+    }
     st = st == NST - 1 ? 0 : st + 1;
   }
   cp_async_wait<0>();
@@ -175,8 +252,9 @@ __device__ __forceinline__ void segment_rows(const Segment& s, const Prefetch<T,
 // at 16-byte word `cache_word` of the dynamic shared memory.
 template <typename T, int OP, bool EXACT, int SLOTS, int NSLOT, int NST, typename Reduce>
 __device__ __forceinline__ void run_segment(const Segment& s, const Prefetch<T, NSLOT>& pf,
-                                            long long r0, long long stride, int k0, int step,
-                                            float eps, Reduce reduce, int cache_word) {
+                                            const Prefetch<T, NSLOT>& pf2, long long r0,
+                                            long long stride, int k0, int step, float eps,
+                                            Reduce reduce, int cache_word) {
   constexpr bool BIAS = OP == kOpLn;
   static_assert(EXACT || SLOTS != kSlotsFull, "only EXACT rows divide evenly");
   const T* w = static_cast<const T*>(s.w);
@@ -184,26 +262,31 @@ __device__ __forceinline__ void run_segment(const Segment& s, const Prefetch<T, 
   if constexpr (EXACT) {
     if (w && (!BIAS || b)) {
       AffineDirect<T, BIAS, true> src{w, b};
-      segment_rows<T, OP, true, SLOTS, NSLOT, NST>(s, pf, r0, stride, k0, step, eps, reduce, src);
+      segment_rows<T, OP, true, SLOTS, NSLOT, NST>(s, pf, pf2, r0, stride, k0, step, eps, reduce,
+                                                   src);
     } else {
       AffineDirect<T, BIAS, false> src{w, b};
-      segment_rows<T, OP, true, SLOTS, NSLOT, NST>(s, pf, r0, stride, k0, step, eps, reduce, src);
+      segment_rows<T, OP, true, SLOTS, NSLOT, NST>(s, pf, pf2, r0, stride, k0, step, eps, reduce,
+                                                   src);
     }
   } else {
     AffineCache<T, NSLOT, BIAS> src;
     src.init(cache_word);
-    segment_rows<T, OP, false, SLOTS, NSLOT, NST>(s, pf, r0, stride, k0, step, eps, reduce, src);
+    segment_rows<T, OP, false, SLOTS, NSLOT, NST>(s, pf, pf2, r0, stride, k0, step, eps, reduce,
+                                                  src);
   }
 }
 
 template <typename T, int OP, bool EXACT, int SLOTS, int VPL>
 __global__ void __launch_bounds__(kWarpBlock, kMinThreadsPerSmWarp / kWarpBlock)
 rows_warp_kernel(const Params p) {
-  const Prefetch<T, VPL> pf{p.prefetch};
+  constexpr int BANK = prefetch_smem_words<VPL, kWarpPrefetchStages>(kWarpBlock);
+  const Prefetch<T, VPL> pf{p.prefetch, 0};
+  const Prefetch<T, VPL> pf2{p.prefetch, BANK};
   const int lane = threadIdx.x & 31;
   const long long warp = (long long)blockIdx.x * (kWarpBlock / 32) + (threadIdx.x >> 5);
   const long long nwarps = (long long)gridDim.x * (kWarpBlock / 32);
-  const int cache_word = p.prefetch ? prefetch_smem_words<VPL, kWarpPrefetchStages>(kWarpBlock) : 0;
+  const int cache_word = p.prefetch ? BANK * (op_has_second(OP) ? 2 : 1) : 0;
 #pragma unroll 1
   for (int si = 0; si < p.nseg; ++si) {
     const Segment s = pick_segment(p.seg, si);
@@ -213,8 +296,8 @@ rows_warp_kernel(const Params p) {
     const int gi = lane / G;
     const unsigned mask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << (gi * G));
     auto reduce = [&](float t) { return group_sum(t, G, mask); };
-    run_segment<T, OP, EXACT, SLOTS, VPL, kWarpPrefetchStages>(s, pf, warp * per_warp + gi, nwarps * per_warp, gl, G,
-                                    p.eps, reduce, cache_word);
+    run_segment<T, OP, EXACT, SLOTS, VPL, kWarpPrefetchStages>(
+        s, pf, pf2, warp * per_warp + gi, nwarps * per_warp, gl, G, p.eps, reduce, cache_word);
   }
 }
 
@@ -225,19 +308,21 @@ rows_cta_kernel(const Params p) {
   // Two alternating reduction buffers: a buffer is rewritten only after every
   // thread has passed the barrier of the reduction in between.
   __shared__ float red[2][NT / 32];
-  const Prefetch<T, VPT> pf{p.prefetch};
+  constexpr int BANK = prefetch_smem_words<VPT, kCtaPrefetchStages>(NT);
+  const Prefetch<T, VPT> pf{p.prefetch, 0};
+  const Prefetch<T, VPT> pf2{p.prefetch, BANK};
   int slot = 0;
   auto reduce = [&](float t) {
     const float r = block_sum<NT>(t, red[slot]);
     slot ^= 1;
     return r;
   };
-  const int cache_word = p.prefetch ? prefetch_smem_words<VPT, kCtaPrefetchStages>(NT) : 0;
+  const int cache_word = p.prefetch ? BANK * (op_has_second(OP) ? 2 : 1) : 0;
 #pragma unroll 1
   for (int si = 0; si < p.nseg; ++si) {
     const Segment s = pick_segment(p.seg, si);
-    run_segment<T, OP, EXACT, SLOTS, VPT, kCtaPrefetchStages>(s, pf, blockIdx.x, gridDim.x, threadIdx.x, NT, p.eps,
-                                    reduce, cache_word);
+    run_segment<T, OP, EXACT, SLOTS, VPT, kCtaPrefetchStages>(
+        s, pf, pf2, blockIdx.x, gridDim.x, threadIdx.x, NT, p.eps, reduce, cache_word);
   }
 }
 

@@ -21,6 +21,15 @@ Workloads (shapes follow the pages' examples):
   dual_bf16_decode        the same heads at one token (decode).
   rms_bf16_16x4096x4096   RMSNorm bf16, N(0,1) with 1 % of entries x50.
   ln_bf16_65536x{D}       LayerNorm bf16, N(0.5, 2), every 64th row constant.
+
+Fused extensions (the elementwise fusions of "norm_fusion.rs", module doc
+comment), at the shapes of the rows they fuse with:
+  add_rms_bf16_16x4096x4096   residual add + RMSNorm at the hidden-state shape
+                              above: x, residual N(0,1), w N(1, 0.1).
+  gated_rms_bf16_8192x32x128  gated output RMSNorm over 128-wide heads at the
+                              prefill token count: x, z N(0,1), w N(1, 0.1).
+  add_rms_f32_4x128x1024,     the same two ops at the small f32 shape of the
+  gated_rms_f32_4x128x1024    Part 1 Correctness cell (x, r/z U(-1,1)).
 """
 from dataclasses import dataclass, field
 from typing import Dict, Optional, Tuple
@@ -34,7 +43,7 @@ CONSTANT_ROW_PERIOD = 64
 @dataclass(frozen=True)
 class Workload:
     name: str
-    op: str                      # "rms", "ln" or "dual"
+    op: str                      # "rms", "ln", "dual", "add_rms" or "gated_rms"
     dtype: torch.dtype
     shape: Tuple[int, ...]       # x (or q) shape; last axis is the row
     eps: float
@@ -77,6 +86,10 @@ class Workload:
             kd = self.k_shape[-1]
             return (2 * self.rows * self.dim * s + self.dim * s
                     + 2 * self.k_rows * kd * s + kd * s)
+        if self.op == "add_rms":   # read x, r; write y, h
+            return 4 * self.rows * self.dim * s + self.dim * s
+        if self.op == "gated_rms":  # read x, z; write y
+            return 3 * self.rows * self.dim * s + self.dim * s
         vectors = 2 if self.op == "ln" else 1
         return 2 * self.rows * self.dim * s + vectors * self.dim * s
 
@@ -99,10 +112,20 @@ _register(Workload("rms_bf16_16x4096x4096", "rms", torch.bfloat16, (16, 4096, 40
 for _k, _d in enumerate(LN_WIDTHS):
     _register(Workload(f"ln_bf16_65536x{_d}", "ln", torch.bfloat16, (65536, _d), 1e-5, 50 + _k))
 
+_register(Workload("add_rms_bf16_16x4096x4096", "add_rms", torch.bfloat16, (16, 4096, 4096),
+                   1e-5, 60))
+_register(Workload("gated_rms_bf16_8192x32x128", "gated_rms", torch.bfloat16, (8192, 32, 128),
+                   1e-6, 61))
+_register(Workload("add_rms_f32_4x128x1024", "add_rms", torch.float32, (4, 128, 1024), 1e-6, 62))
+_register(Workload("gated_rms_f32_4x128x1024", "gated_rms", torch.float32, (4, 128, 1024),
+                   1e-6, 63))
+
 # The large bf16 workloads: one pass over each is one benchmark step.
 LARGE_SUITE = ("dual_bf16_prefill", "rms_bf16_16x4096x4096") + tuple(
     f"ln_bf16_65536x{d}" for d in LN_WIDTHS)
 SMALL_SUITE = ("rms_f32_4x128x1024", "ln_f32_1x1024x768", "dual_bf16_decode")
+# The fused extensions, measured beside (not inside) the benchmark step.
+FUSED_SUITE = ("add_rms_bf16_16x4096x4096", "gated_rms_bf16_8192x32x128")
 
 
 def _gen(device, seed):
@@ -150,6 +173,16 @@ def make_inputs(w: Workload, device="cpu") -> Dict[str, torch.Tensor]:
         values = _normal((const_rows.numel(), 1), 0.5, 2.0, g, device)
         x[const_rows] = values.expand(-1, w.dim)
         out["x"] = x
+    elif w.op in ("add_rms", "gated_rms") and w.dtype == torch.float32:
+        second = "r" if w.op == "add_rms" else "z"
+        out["x"] = _uniform(w.shape, -1.0, 1.0, g, device)
+        out[second] = _uniform(w.shape, -1.0, 1.0, g, device)
+        out["w"] = _uniform((w.dim,), 0.5, 1.5, g, device)
+    elif w.op in ("add_rms", "gated_rms"):
+        second = "r" if w.op == "add_rms" else "z"
+        out["x"] = _normal(w.shape, 0.0, 1.0, g, device)
+        out[second] = _normal(w.shape, 0.0, 1.0, g, device)
+        out["w"] = _normal((w.dim,), 1.0, 0.1, g, device)
     else:
         raise KeyError(w.name)
     return {k: v.to(w.dtype) for k, v in out.items()}
