@@ -14,8 +14,9 @@ so LayerNorm also allows an absolute floor 1e-5 * (|n*w| + |b| + 1) (that is
 
 Gated RMSNorm in fp32 (``scaled=True``): its outputs reach |y| ~ 40 (the gate's
 silu grows like the gate), where a fixed 1e-5 is below the binary32 error of
-the product chain itself (four roundings, expf within 2 ulps, a divide:
-about 1e-6 relative). Its bound is 1e-5 * (1 + |y|), ten times that error.
+the product chain itself (four roundings; __expf within 2 + 1.2 |t| ulps and
+__fdividef within 2 ulps: about 1e-6 relative for |t| < 20). Its bound is
+1e-5 * (1 + |y|), ten times that error.
 """
 import numpy as np
 import torch
