@@ -314,6 +314,63 @@ def cpu_baseline(step, chunk_rows=2048):
                       f"{busy:.1f} s of oracle time"}
 
 
+def time_fused(device, rank, dist, peak, reps=30, oracle_rows=2048):
+    """The fused extensions (residual-add RMSNorm, gated RMSNorm), measured
+    beside the step: the median CUDA-event time of single launches on the
+    launching stream, each after a 256 MB read that evicts L2 (max over
+    ranks), and on rank 0 the fp64 oracle's rows/s on the first
+    `oracle_rows` rows on all host cores."""
+    import transformer_row_normalization_b200 as rn
+    evict = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=device)
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    out = []
+    for name in wl.FUSED_SUITE:
+        w = wl.WORKLOADS[name]
+        rw = wl.Workload(w.name, w.op, w.dtype, w.shape, w.eps, rank_seed(w.seed, rank))
+        a = wl.make_inputs(rw, device=device)
+        second = a["r"] if w.op == "add_rms" else a["z"]
+        y, h = torch.empty_like(a["x"]), torch.empty_like(a["x"])
+
+        def launch():
+            if w.op == "add_rms":
+                rn.add_rms_norm(a["x"], second, a["w"], w.eps, out=y, out_h=h)
+            else:
+                rn.gated_rms_norm(a["x"], second, a["w"], w.eps, out=y)
+
+        for _ in range(3):
+            launch()
+        times = []
+        for _ in range(reps):
+            evict.sum()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            launch()
+            e.record()
+            e.synchronize()
+            times.append(s.elapsed_time(e))
+        t = max_over_ranks(sorted(times)[len(times) // 2], dist, device)
+        g = w.algorithmic_bytes() / (t * 1e-3) / 1e9
+        item = {"workload": name, "us": round(t * 1e3, 2),
+                "rows_per_s": round(w.rows / (t * 1e-3)), "gbs": round(g, 1),
+                "frac": round(g / peak, 4), "algorithmic_bytes": w.algorithmic_bytes()}
+        if rank == 0:
+            import oracle
+            x = a["x"].reshape(-1, w.dim)[:oracle_rows].cpu()
+            x2 = second.reshape(-1, w.dim)[:oracle_rows].cpu()
+            wt = a["w"].cpu()
+            fn = oracle.add_rms_norm if w.op == "add_rms" else oracle.gated_rms_norm
+            fn(x[:64], x2[:64], wt, w.eps, nthreads=cores)  # warm-up
+            t0 = time.perf_counter()
+            fn(x, x2, wt, w.eps, nthreads=cores)
+            busy = time.perf_counter() - t0
+            item["oracle_rows_per_s"] = round(x.shape[0] / busy, 1)
+        out.append(item)
+    return {"workloads": out, "cores": cores,
+            "timing": f"median of {reps} single launches, each after a 256 MB read "
+                      "that evicts L2; oracle on the first "
+                      f"{oracle_rows} rows, fp64, {cores} threads"}
+
+
 # ---------------------------------------------------------------------------
 
 
@@ -384,6 +441,7 @@ def run_ours(args):
     e2e = {"value": world * rows * e2e_steps / (e2e_ms / 1e3), "unit": "rows/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
+    fused = time_fused(device, rank, dist, peak)
     base = cpu_baseline(step) if (rank == 0 and world == 1) else None
     if dist is not None:
         barrier(dist, device)
@@ -399,6 +457,7 @@ def run_ours(args):
                     "peak_source": peak_kind},
             "roofline": roofline, "cpu_baseline": base, "e2e": e2e,
             "gpu_launches": 7 * args.steps, "clocks": clk, "per_config": per_config,
+            "fused": fused,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

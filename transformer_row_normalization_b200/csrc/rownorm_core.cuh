@@ -314,24 +314,6 @@ __device__ __forceinline__ float load_edge(const Row<T>& g, int D, int k0) {
   return k0 < g.nedge ? Elem<T>::get(g.x_row + edge_column(g, D, k0)) : 0.f;
 }
 
-// All of a thread's slots of one row from global memory (absent ones zero).
-template <typename T, int SLOTS, int NSLOT>
-__device__ __forceinline__ void load_row(const Row<T>& g, int k0, int step,
-                                         F2 (&v)[NSLOT][Elem<T>::P]) {
-  constexpr int V = Elem<T>::V;
-  constexpr int P = Elem<T>::P;
-#pragma unroll
-  for (int p = 0; p < NSLOT; ++p) {
-    const int f = k0 + step * p;
-    if (slot_present<SLOTS, NSLOT>(p, f, g.nfull)) {
-      Elem<T>::unpack(load_stream(g.x_full + (long long)f * V), v[p]);
-    } else {
-#pragma unroll
-      for (int j = 0; j < P; ++j) v[p][j] = zero2();
-    }
-  }
-}
-
 // ---------------------------------------------------------------------------
 // per-thread partial sums over the slots and the edge element of one row
 //

@@ -81,19 +81,33 @@ struct Prefetch {
     constexpr int V = Elem<T>::V;
     return on ? *slot(stage, p) : load_stream(full + (long long)f * V);
   }
-  // The thread's slots of a row; absent ones zero.
+  // The thread's slots of a row; absent ones zero. (The test of `on` stays
+  // outside the slot loop: one uniform branch per row.)
   template <int SLOTS>
   __device__ __forceinline__ void take(const T* full, int nfull, int k0, int step, int stage,
                                        F2 (&v)[NSLOT][Elem<T>::P]) const {
+    constexpr int V = Elem<T>::V;
     constexpr int P = Elem<T>::P;
+    if (on) {
 #pragma unroll
-    for (int p = 0; p < NSLOT; ++p) {
-      const int f = k0 + step * p;
-      if (slot_present<SLOTS, NSLOT>(p, f, nfull)) {
-        Elem<T>::unpack(chunk(full, f, stage, p), v[p]);
-      } else {
+      for (int p = 0; p < NSLOT; ++p) {
+        if (slot_present<SLOTS, NSLOT>(p, k0 + step * p, nfull)) {
+          Elem<T>::unpack(*slot(stage, p), v[p]);
+        } else {
 #pragma unroll
-        for (int j = 0; j < P; ++j) v[p][j] = zero2();
+          for (int j = 0; j < P; ++j) v[p][j] = zero2();
+        }
+      }
+    } else {
+#pragma unroll
+      for (int p = 0; p < NSLOT; ++p) {
+        const int f = k0 + step * p;
+        if (slot_present<SLOTS, NSLOT>(p, f, nfull)) {
+          Elem<T>::unpack(load_stream(full + (long long)f * V), v[p]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < P; ++j) v[p][j] = zero2();
+        }
       }
     }
   }
