@@ -90,10 +90,14 @@ class Oracle:
                                             vp, ctypes.c_float, vp, vp, ctypes.c_int]
         lib.oracle_gated_rms_norm.argtypes = [vp, vp, ctypes.c_int, i64, i64, i64, i64,
                                               vp, ctypes.c_float, vp, ctypes.c_int]
+        lib.oracle_dual_head_rms_norm_rope.argtypes = [
+            vp, i64, i64, i64, vp, i64, i64, i64, ctypes.c_int, vp, vp, ctypes.c_float,
+            i64, i64, i64, i64, ctypes.c_int, ctypes.c_float, ctypes.c_float, vp, vp, vp,
+            ctypes.c_int]
         lib.oracle_decode.argtypes = [vp, ctypes.c_int, i64, vp]
         for fn in (lib.oracle_rms_norm, lib.oracle_layer_norm,
                    lib.oracle_dual_head_rms_norm, lib.oracle_add_rms_norm,
-                   lib.oracle_gated_rms_norm):
+                   lib.oracle_gated_rms_norm, lib.oracle_dual_head_rms_norm_rope):
             fn.restype = ctypes.c_int
         lib.oracle_decode.restype = None
         self._lib = lib
@@ -175,6 +179,35 @@ class Oracle:
             raise ValueError(f"oracle_gated_rms_norm rejected its arguments (status {st})")
         return y
 
+    def dual_head_rms_norm_rope(self, q, k, wq, wk, eps, heads_q, heads_k, offset, dims,
+                                traditional=False, base=10000.0, scale=1.0, inv_freq=None,
+                                nthreads=1):
+        """(RoPE(RMSNorm(q, wq)), RoPE(RMSNorm(k, wk))) in fp64, queries first.
+        Rows are head rows, token-major: row r is token r // heads. ``base``
+        and ``scale`` travel as binary32; ``inv_freq`` (dims/2 float32) replaces
+        base^(-2i/dims)."""
+        q, qr, qd, qs = _view(q)
+        k, kr, kd, ks = _view(k)
+        code = _dtype_code(q)
+        if _dtype_code(k) != code:
+            raise TypeError("q and k must share a dtype")
+        wq_ = _vector(wq, qd, code)
+        wk_ = _vector(wk, kd, code)
+        f = None
+        if inv_freq is not None:
+            f = np.ascontiguousarray(_as_numpy(inv_freq), dtype=np.float32).reshape(-1)
+            if f.size != dims // 2:
+                raise ValueError("inv_freq must hold dims / 2 values")
+        yq = np.empty((qr, qd), dtype=np.float64)
+        yk = np.empty((kr, kd), dtype=np.float64)
+        st = self._lib.oracle_dual_head_rms_norm_rope(
+            _ptr(q), qr, qd, qs, _ptr(k), kr, kd, ks, code, _ptr(wq_), _ptr(wk_), float(eps),
+            int(heads_q), int(heads_k), int(offset), int(dims), int(bool(traditional)),
+            float(base), float(scale), _ptr(f), _ptr(yq), _ptr(yk), int(nthreads))
+        if st:
+            raise ValueError(f"oracle_dual_head_rms_norm_rope rejected its arguments ({st})")
+        return yq, yk
+
     def decode(self, a):
         """Exact fp64 values of a float32 or bfloat16-bits array."""
         a = np.ascontiguousarray(_as_numpy(a))
@@ -211,6 +244,13 @@ def add_rms_norm(x, residual, weight, eps, nthreads=1):
 
 def gated_rms_norm(x, gate, weight, eps, nthreads=1):
     return default().gated_rms_norm(x, gate, weight, eps, nthreads)
+
+
+def dual_head_rms_norm_rope(q, k, wq, wk, eps, heads_q, heads_k, offset, dims,
+                            traditional=False, base=10000.0, scale=1.0, inv_freq=None,
+                            nthreads=1):
+    return default().dual_head_rms_norm_rope(q, k, wq, wk, eps, heads_q, heads_k, offset, dims,
+                                             traditional, base, scale, inv_freq, nthreads)
 
 
 def decode(a):

@@ -42,6 +42,18 @@
  *                  y_j = x_j / sqrt( (1/D) * sum_i x_i^2 + eps ) * w_j
  *                        * silu(z_j),   silu(t) = t / (1 + exp(-t))
  *
+ *   Dual q/k head RMSNorm + RoPE -- the dual head norm above, each normalized
+ *                head row then rotated as "Emily.Fast", `rope/3` and
+ *                `rope_with_freqs/4` describe: with pos = offset + token
+ *                (token = row / heads) and, for plane i < dims/2,
+ *                  theta_i = pos * scale * f_i,
+ *                  f_i = base^(-2i/dims), or the given inverse frequency,
+ *                the plane (a, b) = (i, i + dims/2) (split-half) or
+ *                (2i, 2i + 1) (traditional) becomes
+ *                  y_a = n_a cos theta_i - n_b sin theta_i
+ *                  y_b = n_b cos theta_i + n_a sin theta_i
+ *                and columns from dims on are n unchanged.
+ *
  * Readings where the pages are silent (each is listed in the design doc):
  *   - the variance divisor is D (population variance);
  *   - eps travels as a binary32 value (norm_fusion.rs keeps it as f32 bits)
@@ -58,6 +70,7 @@
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #define ORACLE_F32 0
@@ -267,6 +280,69 @@ int oracle_gated_rms_norm(const void *x, const void *z, int dtype, int64_t rows,
         gated_rms_norm_row(x, z, dtype, i, dim, x_stride, z_stride, w, eps64,
                            y + i * dim);
     return 0;
+}
+
+/* RMSNorm of one row into n_row (fp64), then RoPE of its first dims columns
+ * at position pos, into y_row. */
+static void rms_rope_row(const void *x, int dtype, int64_t row, int64_t dim,
+                         int64_t row_stride, const void *w, double eps, double pos,
+                         int64_t dims, int traditional, double base, double scale,
+                         const float *inv_freq, double *n_row, double *y_row) {
+    rms_norm_row(x, dtype, row, dim, row_stride, w, eps, n_row);
+    for (int64_t j = 0; j < dim; ++j) y_row[j] = n_row[j];
+    const int64_t half = dims / 2;
+    for (int64_t i = 0; i < half; ++i) {
+        double f = (inv_freq != NULL) ? (double)inv_freq[i]
+                                      : pow(base, -2.0 * (double)i / (double)dims);
+        double theta = pos * scale * f;
+        double c = cos(theta), s = sin(theta);
+        int64_t a = traditional ? 2 * i : i;
+        int64_t b = traditional ? 2 * i + 1 : i + half;
+        y_row[a] = n_row[a] * c - n_row[b] * s;
+        y_row[b] = n_row[b] * c + n_row[a] * s;
+    }
+}
+
+static int rms_rope_rows(const void *x, int dtype, int64_t rows, int64_t dim,
+                         int64_t stride, const void *w, double eps, int64_t heads,
+                         int64_t offset, int64_t dims, int traditional, double base,
+                         double scale, const float *inv_freq, double *y, int nthreads) {
+    int status = check_view(x, dtype, rows, dim, stride);
+    if (status) return status;
+    if (rows > 0 && y == NULL) return 1;
+    if (heads < 1 || rows % heads != 0 || dims < 0 || dims % 2 != 0 || dims > dim) return 3;
+    (void)nthreads;
+#pragma omp parallel num_threads(nthreads > 0 ? nthreads : 1)
+    {
+        double *n_row = (double *)malloc((size_t)dim * sizeof(double));
+#pragma omp for schedule(static)
+        for (int64_t r = 0; r < rows; ++r) {
+            double pos = (double)(offset + r / heads);
+            rms_rope_row(x, dtype, r, dim, stride, w, eps, pos, dims, traditional, base,
+                         scale, inv_freq, n_row, y + r * dim);
+        }
+        free(n_row);
+    }
+    return 0;
+}
+
+/* Queries first, keys second; one eps, one position schedule. */
+int oracle_dual_head_rms_norm_rope(const void *q, int64_t q_rows, int64_t q_dim,
+                                   int64_t q_stride, const void *k, int64_t k_rows,
+                                   int64_t k_dim, int64_t k_stride, int dtype,
+                                   const void *wq, const void *wk, float eps,
+                                   int64_t heads_q, int64_t heads_k, int64_t offset,
+                                   int64_t dims, int traditional, float base, float scale,
+                                   const float *inv_freq, double *yq, double *yk,
+                                   int nthreads) {
+    if (heads_q < 1 || heads_k < 1 || q_rows / heads_q != k_rows / heads_k) return 3;
+    int status = rms_rope_rows(q, dtype, q_rows, q_dim, q_stride, wq, (double)eps, heads_q,
+                               offset, dims, traditional, (double)base, (double)scale,
+                               inv_freq, yq, nthreads);
+    if (status) return status;
+    return rms_rope_rows(k, dtype, k_rows, k_dim, k_stride, wk, (double)eps, heads_k,
+                         offset, dims, traditional, (double)base, (double)scale, inv_freq,
+                         yk, nthreads);
 }
 
 /* Exposed so the test suite can pin the element decoding on its own. */

@@ -529,4 +529,103 @@ def pin_gated_strided_gate(orc):
     _close(got, ref.numpy(), 1e-12, 1e-14, "gated strided gate")
 
 
+# --------------------------------------------------------------------------
+# dual q/k head RMSNorm + RoPE ("Emily.Fast", rope/3 and rope_with_freqs/4)
+
+
+def _rope_complex(n, pos, dims, traditional, freqs):
+    """RoPE as complex multiplication: each plane (a, b) is the complex number
+    a + ib times exp(i * pos * f) (numpy's complex exponential)."""
+    y = n.copy()
+    half = dims // 2
+    for i in range(half):
+        a, b = (2 * i, 2 * i + 1) if traditional else (i, i + half)
+        z = (n[:, a] + 1j * n[:, b]) * np.exp(1j * pos * freqs[i])
+        y[:, a], y[:, b] = z.real, z.imag
+    return y
+
+
+def _torch_rms(x, w, eps):
+    xt = torch.from_numpy(np.asarray(x, dtype=np.float64))
+    n = torch.nn.functional.rms_norm(xt, (xt.shape[-1],), eps=f32(eps)).numpy()
+    return n if w is None else n * np.asarray(w, dtype=np.float64)
+
+
+def pin_rope_is_complex_rotation(orc):
+    # 3 tokens x 4 query heads and 2 key heads, head dim 16, partial rotary
+    # (dims 12), offset 5, base 10000 (binary32), both plane layouts
+    q = _rows(90, 12, 16)
+    k = _rows(91, 6, 16)
+    wq = _rows(92, 1, 16, mean=1.0, std=0.1).reshape(-1)
+    wk = _rows(93, 1, 16, mean=1.0, std=0.1).reshape(-1)
+    freqs = [f32(10000.0) ** (-2.0 * i / 12) for i in range(6)]
+    for trad in (False, True):
+        yq, yk = orc.dual_head_rms_norm_rope(q, k, wq, wk, 1e-6, 4, 2, 5, 12, traditional=trad)
+        for y, x, w, heads in ((yq, q, wq, 4), (yk, k, wk, 2)):
+            n = _torch_rms(x, w, 1e-6)
+            pos = (5 + np.arange(x.shape[0]) // heads).astype(np.float64)
+            want = _rope_complex(n, pos, 12, trad, freqs)
+            _close(y, want, 1e-13, 1e-14, f"rope complex (traditional={trad})")
+
+
+def pin_rope_page_freqs_example(orc):
+    # "Emily.Fast", rope_with_freqs/4 example: x = iota {1, 1, 4, 8} (4
+    # positions of one 8-wide head), offset 0, freqs [1, 0.1, 0.01, 0.001]
+    x = np.arange(32, dtype=np.float32).reshape(4, 8)
+    freqs = np.array([1.0, 0.1, 0.01, 0.001], dtype=np.float32)
+    yq, _ = orc.dual_head_rms_norm_rope(x, x, None, None, 1e-6, 1, 1, 0, 8, inv_freq=freqs)
+    n = _torch_rms(x, None, 1e-6)
+    want = _rope_complex(n, np.arange(4, dtype=np.float64), 8, False,
+                         [float(f) for f in freqs])
+    _close(yq, want, 1e-13, 1e-14, "rope page freqs example")
+    # with base 10000 and dims 8 the inverse frequencies are 1, 0.1, 0.01, 0.001
+    yb, _ = orc.dual_head_rms_norm_rope(x, x, None, None, 1e-6, 1, 1, 0, 8)
+    _close(yb, yq, 1e-7, 1e-9, "base 1e4 vs its frequency table")
+
+
+def pin_rope_preserves_plane_norms_and_tail(orc):
+    q = _rows(94, 8, 24)
+    yq, _ = orc.dual_head_rms_norm_rope(q, q, None, None, 1e-6, 2, 2, 1000, 16)
+    n = _torch_rms(q, None, 1e-6)
+    for i in range(8):
+        _close(yq[:, i] ** 2 + yq[:, i + 8] ** 2, n[:, i] ** 2 + n[:, i + 8] ** 2, 1e-13,
+               1e-15, "plane norm")
+    _close(yq[:, 16:], n[:, 16:], 1e-14, 1e-15, "columns past dims pass through")
+
+
+def pin_rope_position_zero_is_plain_norm(orc):
+    q = _rows(95, 6, 32, "bf16")
+    wq = _rows(96, 1, 32, "bf16", mean=1.0, std=0.1).reshape(-1)
+    yq, _ = orc.dual_head_rms_norm_rope(q, q, wq, wq, 1e-6, 6, 6, 0, 32)
+    n = _torch_rms(orc.decode(q), orc.decode(wq), 1e-6)
+    _close(yq, n, 1e-14, 1e-15, "token 0 at offset 0 is not rotated")
+    y0, _ = orc.dual_head_rms_norm_rope(q, q, wq, wq, 1e-6, 1, 1, 77, 32, scale=0.0)
+    _close(y0, n, 1e-14, 1e-15, "scale 0 does not rotate")
+
+
+def pin_rope_relative_position(orc):
+    # q . k after RoPE depends only on the positions' difference: shifting
+    # the offset leaves every query/key dot product of a token unchanged
+    q = _rows(97, 3, 16)
+    k = _rows(98, 3, 16)
+    dots = []
+    for off in (0, 37, 4096):
+        yq, yk = orc.dual_head_rms_norm_rope(q, k, None, None, 1e-6, 1, 1, off, 16)
+        dots.append(yq @ yk.T)
+    _close(dots[1], dots[0], 1e-11, 1e-12, "relative position (37)")
+    _close(dots[2], dots[0], 1e-10, 1e-11, "relative position (4096)")
+
+
+def pin_rope_layouts_are_a_column_permutation(orc):
+    # interleaving the columns turns split-half planes into traditional ones
+    d = 16
+    perm = np.empty(d, dtype=np.int64)
+    perm[0::2], perm[1::2] = np.arange(d // 2), np.arange(d // 2) + d // 2
+    q = _rows(99, 5, d)
+    ys, _ = orc.dual_head_rms_norm_rope(q, q, None, None, 1e-6, 1, 1, 3, d)
+    yt, _ = orc.dual_head_rms_norm_rope(np.ascontiguousarray(q[:, perm]), q, None, None, 1e-6,
+                                        1, 1, 3, d, traditional=True)
+    _close(yt, ys[:, perm], 1e-13, 1e-15, "traditional = permuted split-half")
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -85,6 +85,32 @@ MUTANTS = {
                                       "decode_element(z, dtype, row * x_stride + j)"),
     "gated drops weight": ("y_row[j] = xv / rms_x * weight * silu;",
                            "y_row[j] = xv / rms_x * silu;"),
+    "rope sign flipped": ("y_row[a] = n_row[a] * c - n_row[b] * s;",
+                          "y_row[a] = n_row[a] * c + n_row[b] * s;"),
+    "rope cos and sin swapped": ("double c = cos(theta), s = sin(theta);",
+                                 "double c = sin(theta), s = cos(theta);"),
+    "rope exponent without 2": ("pow(base, -2.0 * (double)i / (double)dims)",
+                                "pow(base, -(double)i / (double)dims)"),
+    "rope position per row not token": ("double pos = (double)(offset + r / heads);",
+                                        "double pos = (double)(offset + r);"),
+    "rope ignores offset": ("double pos = (double)(offset + r / heads);",
+                            "double pos = (double)(r / heads);"),
+    "rope ignores scale": ("double theta = pos * scale * f;", "double theta = pos * f;"),
+    "rope partner off by one": ("int64_t b = traditional ? 2 * i + 1 : i + half;",
+                                "int64_t b = traditional ? 2 * i + 1 : i + half - 1;"),
+    "rope ignores the layout flag": ("int64_t a = traditional ? 2 * i : i;\n"
+                                     "        int64_t b = traditional ? 2 * i + 1 : i + half;",
+                                     "int64_t a = i;\n        int64_t b = i + half;"),
+    "rope rotates the whole row": ("const int64_t half = dims / 2;",
+                                   "const int64_t half = dim / 2;"),
+    "rope ignores the frequency table": (
+        "double f = (inv_freq != NULL) ? (double)inv_freq[i]\n"
+        "                                      : pow(",
+        "double f = (inv_freq != NULL && 0) ? (double)inv_freq[i]\n"
+        "                                      : pow("),
+    "rope key rows use query heads": (
+        "return rms_rope_rows(k, dtype, k_rows, k_dim, k_stride, wk, (double)eps, heads_k,",
+        "return rms_rope_rows(k, dtype, k_rows, k_dim, k_stride, wk, (double)eps, heads_q,"),
 }
 
 
