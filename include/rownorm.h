@@ -183,6 +183,57 @@ RN_API int rn_gated_rms_norm(const rn_view *x, const rn_view *z,
                              const void *weight, float eps, const rn_view *y,
                              void *stream);
 
+/*
+ * RoPE schedule for rn_dual_head_rms_norm_rope ("Emily.Fast", rope/3 and
+ * rope_with_freqs/4). Head rows are token-major: row r of q is token
+ * r / heads_q (likewise k), at position offset + token. For plane i <
+ * dims / 2 the rotation angle is theta_i(pos); the planes are (i, i + dims/2)
+ * (split-half) or (2i, 2i + 1) (traditional, interleaved). Columns from dims
+ * on pass through unrotated.
+ */
+typedef struct rn_rope {
+    const float *table;   /* device, [n_pos][dims] binary32: cos theta_i(pos) */
+                          /* at [pos][i], sin theta_i(pos) at [pos][dims/2+i] */
+                          /* (build it with rn_rope_table); caller-owned       */
+    int64_t n_pos;        /* rows of the table (positions 0 .. n_pos - 1)      */
+    int64_t offset;       /* position of token 0 (0 for a prompt, the cache    */
+                          /* length in decode); offset + tokens <= n_pos       */
+    int32_t dims;         /* rotated columns: even, <= both head dims          */
+    int32_t traditional;  /* 1: planes (2i, 2i + 1); 0: (i, i + dims / 2)     */
+    int32_t heads_q;      /* q rows per token                                  */
+    int32_t heads_k;      /* k rows per token                                  */
+} rn_rope;
+
+/*
+ * Fill a HOST buffer `table` ([n_pos][dims] binary32) with the cos / sin of
+ * theta_i(pos) = pos * scale * f_i for every position and plane, where
+ * f_i = base^(-2i / dims), or inv_freq[i] when inv_freq (host, dims / 2
+ * binary32 values) is not NULL (rope_with_freqs/4: Llama-3, LongRoPE, linear
+ * or dynamic schedules precomputed by the caller). Angles are formed and
+ * evaluated in double and rounded once, so large positions keep full
+ * binary32 accuracy. Copy the table to the device once per model.
+ * Returns RN_OK, RN_ERR_SHAPE (odd dims, n_pos < 0), RN_ERR_NULL, RN_ERR_EPS
+ * (base <= 0 or non-finite base / scale).
+ */
+RN_API int rn_rope_table(int32_t dims, float base, float scale,
+                         const float *inv_freq, int64_t n_pos, float *table);
+
+/*
+ * Dual q/k head RMSNorm followed by RoPE, in ONE launch (the dual head norm
+ * of "norm_fusion.rs" with the rotary embedding that follows it in these
+ * models):
+ *   o = rms_norm(q, wq, eps) (binary32, not rounded), yq = rope(o); the same
+ *   for k with wk; y_a = o_a cos - o_b sin, y_b = o_b cos + o_a sin per plane.
+ * Arguments as rn_dual_head_rms_norm, plus the schedule `rope`. q and k must
+ * hold the same number of tokens. Errors: RN_ERR_NULL (rope or its table),
+ * RN_ERR_SHAPE (heads, tokens, dims or positions), RN_ERR_ALIGN (table),
+ * RN_ERR_OVERLAP (an output over the table); others as the dual head norm.
+ */
+RN_API int rn_dual_head_rms_norm_rope(const rn_view *q, const rn_view *k,
+                                      const void *wq, const void *wk, float eps,
+                                      const rn_rope *rope, const rn_view *yq,
+                                      const rn_view *yk, void *stream);
+
 /* Static text for an rn_status value ("unknown status" otherwise). */
 RN_API const char *rn_status_string(int status);
 

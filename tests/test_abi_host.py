@@ -3,6 +3,8 @@ point the header declares, and validates arguments before any CUDA call.
 Only invalid calls and rows == 0 calls are made here; they return before the
 library touches the CUDA runtime, so no GPU is needed."""
 import ctypes
+
+import numpy as np
 import os
 import re
 
@@ -251,3 +253,59 @@ def test_gated_rms_validation(lib):
     assert gated(lib, x, zv, V(data=FAKE + 32)) == 6   # y partly over x
     z = dict(rows=0)
     assert gated(lib, V(**z), V(data=FAKE + MB, **z), V(**z)) == 0  # y == x
+
+
+# ---------------------------------------------------------------------------
+# RoPE: the host table builder, and validation of the fused entry
+
+
+def test_rope_table_matches_the_math_library():
+    import math
+    t = rn.rope_table(8, 5, base=10000.0, scale=0.5)
+    for p in range(5):
+        for i in range(4):
+            theta = p * 0.5 * (10000.0 ** (-2.0 * i / 8))
+            assert t[p, i].item() == float(np.float32(math.cos(theta)))
+            assert t[p, 4 + i].item() == float(np.float32(math.sin(theta)))
+    f = [1.0, 0.25]
+    t = rn.rope_table(4, 3000, inv_freq=f)
+    assert t[2999, 0].item() == float(np.float32(math.cos(2999.0)))
+    assert t[2999, 3].item() == float(np.float32(math.sin(2999.0 * 0.25)))
+
+
+def test_rope_table_rejects_bad_schedules(lib):
+    buf = (ctypes.c_float * 64)()
+    assert lib.rn_rope_table(7, 10000.0, 1.0, None, 4, buf) == 2
+    assert lib.rn_rope_table(8, 10000.0, 1.0, None, -1, buf) == 2
+    assert lib.rn_rope_table(8, 10000.0, 1.0, None, 4, None) == 1
+    assert lib.rn_rope_table(8, 0.0, 1.0, None, 4, buf) == 4
+    assert lib.rn_rope_table(8, 10000.0, float("inf"), None, 4, buf) == 4
+
+
+def rope_call(lib, q, k, yq, yk, rope, wq=FAKE + (3 << 20), wk=FAKE + (3 << 20) + 4096):
+    return lib.rn_dual_head_rms_norm_rope(
+        ctypes.byref(q), ctypes.byref(k), ctypes.c_void_p(wq), ctypes.c_void_p(wk), 1e-6,
+        ctypes.byref(rope) if rope is not None else None, ctypes.byref(yq), ctypes.byref(yk), None)
+
+
+def test_rope_validation(lib):
+    table = FAKE + (5 << 20)
+    R = lambda **kw: rn.rn_rope(**{**dict(table=table, n_pos=4096, offset=0, dims=64,
+                                           traditional=0, heads_q=4, heads_k=2), **kw})
+    q, k = V(rows=8, dim=64), V(data=FAKE + MB, rows=4, dim=64)
+    yq, yk = V(data=FAKE + 2 * MB, rows=8, dim=64), V(data=FAKE + 3 * MB, rows=4, dim=64)
+    assert rope_call(lib, q, k, yq, yk, None) == 1
+    assert rope_call(lib, q, k, yq, yk, R(heads_q=0)) == 2
+    assert rope_call(lib, q, k, yq, yk, R(heads_q=3)) == 2          # 8 rows, 3 heads
+    assert rope_call(lib, q, k, yq, yk, R(heads_k=4)) == 2          # 2 tokens vs 1
+    assert rope_call(lib, q, k, yq, yk, R(dims=63)) == 2
+    assert rope_call(lib, q, k, yq, yk, R(dims=66)) == 2
+    assert rope_call(lib, q, k, yq, yk, R(offset=4095)) == 2        # needs 2 positions
+    assert b"positions" in lib.rn_last_error()
+    assert rope_call(lib, q, k, yq, yk, R(table=None)) == 1
+    assert rope_call(lib, q, k, yq, yk, R(table=table + 2)) == 5
+    # an output over the table
+    assert rope_call(lib, q, k, V(data=table + 256, rows=8, dim=64), yk, R()) == 6
+    z = dict(rows=0, dim=64)
+    assert rope_call(lib, V(**z), V(data=FAKE + MB, **z), V(data=FAKE + 2 * MB, **z),
+                     V(data=FAKE + 3 * MB, **z), R()) == 0

@@ -17,6 +17,13 @@ silu grows like the gate), where a fixed 1e-5 is below the binary32 error of
 the product chain itself (four roundings; __expf within 2 + 1.2 |t| ulps and
 __fdividef within 2 ulps: about 1e-6 relative for |t| < 20). Its bound is
 1e-5 * (1 + |y|), ten times that error.
+
+RMSNorm + RoPE (``rope=(dims, traditional)``): each rotated output mixes the
+two values of its plane, y_a = o_a cos - o_b sin. Where the two terms cancel,
+the exact result is far below the plane's size, while the binary32 error of
+the chain (about 4e-7 relative) scales with the plane norm
+sqrt(y_a^2 + y_b^2) (rotation keeps it). So bf16 also allows an absolute
+floor of 1e-5 times the plane norm, 25 times that error.
 """
 import numpy as np
 import torch
@@ -33,7 +40,19 @@ def to_f64(t):
     return t.detach().to("cpu").double().numpy()
 
 
-def check(gpu, ref, dtype, bias=None, what="", scaled=False):
+def plane_norms(ref, dims, traditional):
+    """sqrt(y_a^2 + y_b^2) of each element's RoPE plane (|y| past dims)."""
+    ref = np.asarray(ref, dtype=np.float64)
+    out = np.abs(ref).copy()
+    half = dims // 2
+    for i in range(half):
+        a, b = (2 * i, 2 * i + 1) if traditional else (i, i + half)
+        n = np.sqrt(ref[:, a] ** 2 + ref[:, b] ** 2)
+        out[:, a] = out[:, b] = n
+    return out
+
+
+def check(gpu, ref, dtype, bias=None, what="", scaled=False, rope=None):
     """Assert parity; returns (max_abs_err, max_err_in_ulps or None)."""
     got = to_f64(gpu).reshape(ref.shape)
     err = np.abs(got - ref)
@@ -48,6 +67,8 @@ def check(gpu, ref, dtype, bias=None, what="", scaled=False):
         return worst, None
     ulp = bf16_ulp(ref)
     bound = ulp.copy()
+    if rope is not None:
+        bound = np.maximum(bound, 1e-5 * plane_norms(ref, *rope))
     if bias is not None:
         b = np.broadcast_to(to_f64(bias), ref.shape)
         floor = 1e-5 * (np.abs(ref - b) + np.abs(b) + 1.0)

@@ -46,6 +46,13 @@ class rn_view(ctypes.Structure):
                 ("dtype", ctypes.c_int32)]
 
 
+class rn_rope(ctypes.Structure):
+    _fields_ = [("table", ctypes.c_void_p), ("n_pos", ctypes.c_int64),
+                ("offset", ctypes.c_int64), ("dims", ctypes.c_int32),
+                ("traditional", ctypes.c_int32), ("heads_q", ctypes.c_int32),
+                ("heads_k", ctypes.c_int32)]
+
+
 class rn_launch_info(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "family", "threads_per_row", "chunks_per_thread", "smem_bytes", "block_threads",
@@ -76,6 +83,9 @@ def load_library():
         lib.rn_dual_head_rms_norm.argtypes = [pv, pv, vp, vp, f32, pv, pv, vp]
         lib.rn_add_rms_norm.argtypes = [pv, pv, vp, f32, pv, pv, vp]
         lib.rn_gated_rms_norm.argtypes = [pv, pv, vp, f32, pv, vp]
+        lib.rn_dual_head_rms_norm_rope.argtypes = [pv, pv, vp, vp, f32,
+                                                   ctypes.POINTER(rn_rope), pv, pv, vp]
+        lib.rn_rope_table.argtypes = [ctypes.c_int32, f32, f32, vp, ctypes.c_int64, vp]
         lib.rn_plan.argtypes = [ctypes.c_int, pv, pv, pv, pv, vp, vp,
                                 ctypes.POINTER(rn_launch_info)]
         lib.rn_set_grid_override.argtypes = [ctypes.c_int]
@@ -86,7 +96,8 @@ def load_library():
         lib.rn_last_error.argtypes = []
         lib.rn_last_error.restype = ctypes.c_char_p
         for fn in (lib.rn_rms_norm, lib.rn_layer_norm, lib.rn_dual_head_rms_norm,
-                   lib.rn_add_rms_norm, lib.rn_gated_rms_norm, lib.rn_plan, lib.rn_set_grid_override, lib.rn_abi_version,
+                   lib.rn_add_rms_norm, lib.rn_gated_rms_norm, lib.rn_plan,
+                   lib.rn_dual_head_rms_norm_rope, lib.rn_rope_table, lib.rn_set_grid_override, lib.rn_abi_version,
                    lib.rn_set_path_override, lib.rn_device_error_count):
             fn.restype = ctypes.c_int
         _lib = lib
@@ -238,8 +249,59 @@ def rn_gated_rms_norm(x, z, weight, eps=1e-6, out=None, stream=None):
     return out
 
 
+def rope_table(dims, n_pos, base=10000.0, scale=1.0, inv_freq=None, device=None):
+    """The cos/sin table of a RoPE schedule ([n_pos, dims] float32: cos of plane
+    i at [:, i], sin at [:, dims // 2 + i]), computed on the host by the
+    library (angles in double, rounded once); moved to ``device`` if given."""
+    import torch
+    table = torch.empty((int(n_pos), int(dims)), dtype=torch.float32)
+    f = None
+    if inv_freq is not None:
+        f = torch.as_tensor(inv_freq, dtype=torch.float32).contiguous().cpu()
+        if f.numel() != dims // 2:
+            raise ValueError("inv_freq must hold dims // 2 values")
+    _check(load_library().rn_rope_table(int(dims), float(base), float(scale),
+                                        None if f is None else ctypes.c_void_p(f.data_ptr()),
+                                        int(n_pos), ctypes.c_void_p(table.data_ptr())
+                                        if table.numel() else None))
+    return table if device is None else table.to(device)
+
+
+def rn_dual_head_rms_norm_rope(q, k, wq, wk, eps, table, offset, dims, heads_q=None,
+                               heads_k=None, traditional=False, out_q=None, out_k=None,
+                               stream=None):
+    """(RoPE(RMSNorm(q, wq)), RoPE(RMSNorm(k, wk))) from one kernel launch.
+    q [tokens, heads_q, D] and k [tokens, heads_k, Dk] (or 2-D head rows with
+    the head counts given); ``table`` is a CUDA float32 rope_table."""
+    import torch
+    _require_cuda(q, k, wq, wk, table, out_q, out_k)
+    if heads_q is None:
+        heads_q = q.shape[-2] if q.dim() >= 3 else 1
+    if heads_k is None:
+        heads_k = k.shape[-2] if k.dim() >= 3 else 1
+    if table.dtype != torch.float32 or not table.is_contiguous() or table.dim() != 2:
+        raise ValueError("table must be a contiguous [n_pos, dims] float32 tensor")
+    if table.shape[1] != dims:
+        raise ValueError(f"table has {table.shape[1]} columns, dims is {dims}")
+    out_q = torch.empty_like(q) if out_q is None else out_q
+    out_k = torch.empty_like(k) if out_k is None else out_k
+    qv, kv, yqv, ykv = _view(q), _view(k), _view(out_q), _view(out_k)
+    if wq is None or wk is None:
+        raise ValueError("dual head norm needs both wq and wk")
+    rope = rn_rope(table.data_ptr() if table.numel() else None, table.shape[0], int(offset),
+                   int(dims), int(bool(traditional)), int(heads_q), int(heads_k))
+    lib = load_library()
+    with torch.cuda.device(q.device):
+        _check(lib.rn_dual_head_rms_norm_rope(
+            ctypes.byref(qv), ctypes.byref(kv), _vector(wq, qv.dim, q), _vector(wk, kv.dim, k),
+            float(eps), ctypes.byref(rope), ctypes.byref(yqv), ctypes.byref(ykv),
+            _stream(q, stream)))
+    return out_q, out_k
+
+
 rms_norm = rn_rms_norm
 layer_norm = rn_layer_norm
+dual_head_rms_norm_rope = rn_dual_head_rms_norm_rope
 dual_head_rms_norm = rn_dual_head_rms_norm
 add_rms_norm = rn_add_rms_norm
 gated_rms_norm = rn_gated_rms_norm

@@ -300,6 +300,7 @@ struct Launch {
   // staged kernels only
   int stages, stage_bytes, tile_rows[2], contiguous[2], cache_offset;
   int64_t tiles[2];
+  int stage_word;   // kOpRmsRope: staging rows after the slots and the cache
 };
 
 constexpr int kNarrowTileBytes = 16 * 1024;  // rows per stage ~ 16 KB (lane-group rows)
@@ -441,7 +442,17 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
       (g_path_override == 0 && (merged.family == 0 || merged.lanes >= 256));
   const int prefetch =
       want_prefetch && cache + pf_bytes <= device_info(dev).smem_per_block - 1024 ? 1 : 0;
-  const int smem = cache + (prefetch ? pf_bytes : 0);
+  int smem = cache + (prefetch ? pf_bytes : 0);
+  out->stage_word = smem / 16;
+  if (op == rn::kOpRmsRope) {
+    // one binary32 staging row per lane group of the block
+    int64_t stage = 0;
+    for (int i = 0; i < nseg; ++i) {
+      const int64_t b = (int64_t)(rn::kWarpBlock / plans[i].lanes) * xs[i]->dim * 4;
+      if (b > stage) stage = b;
+    }
+    smem += (int)stage;
+  }
   st = blocks_per_sm(dev, fn, threads, smem, &bps);
   if (st) return st;
   int64_t needed = 1;
@@ -521,6 +532,7 @@ int launch(const Launch& l, const rn::Params& params, void* stream) {
   } else {
     rn::Params pr = params;
     pr.prefetch = l.prefetch;
+    pr.stage_word = l.stage_word;
     void* args[] = {&pr};
     e = cudaLaunchKernel(l.fn, dim3((unsigned)l.info.grid_blocks),
                          dim3((unsigned)l.info.block_threads), args, (size_t)l.smem,
@@ -677,6 +689,73 @@ int run_second(int op, const rn_view* x, const rn_view* x2, const void* w, float
   return launch(l, params, stream);
 }
 
+// Dual q/k head RMSNorm followed by RoPE, one launch over both row spaces.
+int run_dual_rope(const rn_view* q, const rn_view* k, const void* wq, const void* wk, float eps,
+                  const rn_rope* rope, const rn_view* yq, const rn_view* yk, void* stream) {
+  int st;
+  if (!rope) return fail(RN_ERR_NULL, "rope is NULL");
+  if ((st = check_view(q, "q"))) return st;
+  if ((st = check_view(k, "k"))) return st;
+  if ((st = check_view(yq, "yq"))) return st;
+  if ((st = check_view(yk, "yk"))) return st;
+  if (q->dtype != k->dtype) return fail(RN_ERR_DTYPE, "q and k differ in dtype");
+  if ((st = check_pair(q, yq, "q", "yq"))) return st;
+  if ((st = check_pair(k, yk, "k", "yk"))) return st;
+  if (!wq || !wk) return fail(RN_ERR_NULL, "dual head norm: wq and wk are required");
+  if ((st = check_eps(eps))) return st;
+  if ((st = check_vector(wq, q->dtype, "wq"))) return st;
+  if ((st = check_vector(wk, q->dtype, "wk"))) return st;
+  if (q->dim > RN_MAX_HEAD_DIM || k->dim > RN_MAX_HEAD_DIM)
+    return fail(RN_ERR_UNSUPPORTED, "dual head norm: head dims %lld, %lld above %d",
+                (long long)q->dim, (long long)k->dim, RN_MAX_HEAD_DIM);
+  if (rope->heads_q < 1 || rope->heads_k < 1)
+    return fail(RN_ERR_SHAPE, "rope: head counts must be >= 1");
+  if (q->rows % rope->heads_q || k->rows % rope->heads_k)
+    return fail(RN_ERR_SHAPE, "rope: rows are not whole tokens of heads");
+  const int64_t tokens = q->rows / rope->heads_q;
+  if (k->rows / rope->heads_k != tokens)
+    return fail(RN_ERR_SHAPE, "rope: q has %lld tokens, k has %lld", (long long)tokens,
+                (long long)(k->rows / rope->heads_k));
+  if (rope->dims < 0 || rope->dims % 2 || rope->dims > q->dim || rope->dims > k->dim)
+    return fail(RN_ERR_SHAPE, "rope: dims %d must be even and <= both head dims",
+                (int)rope->dims);
+  if (rope->offset < 0 || rope->n_pos < 0 || (tokens > 0 && rope->offset + tokens > rope->n_pos))
+    return fail(RN_ERR_SHAPE, "rope: positions [%lld, %lld) outside the table's %lld",
+                (long long)rope->offset, (long long)(rope->offset + tokens),
+                (long long)rope->n_pos);
+  if (rope->dims > 0 && tokens > 0 && !rope->table) return fail(RN_ERR_NULL, "rope: table is NULL");
+  if (reinterpret_cast<uintptr_t>(rope->table) % 4)
+    return fail(RN_ERR_ALIGN, "rope: table not aligned to 4 bytes");
+  // the table (binary32, n_pos x dims) is checked as a vector of the outputs' type
+  const void* vecs[3] = {wq, wk, rope->table};
+  const int64_t dims[3] = {q->dim, k->dim, rope->n_pos * rope->dims * 4 / elem_size(q->dtype)};
+  const rn_view* not_yq[2] = {k, yk};
+  const rn_view* not_yk[1] = {q};
+  if ((st = check_output(yq, q, not_yq, 2, vecs, dims, 3, "yq"))) return st;
+  if ((st = check_output(yk, k, not_yk, 1, vecs, dims, 3, "yk"))) return st;
+  if (q->rows == 0 && k->rows == 0) return RN_OK;
+  const SegPlan plans[2] = {plan_segment(q, yq, wq, nullptr), plan_segment(k, yk, wk, nullptr)};
+  const rn_view* xs[2] = {q, k};
+  const void* ws[2] = {wq, wk};
+  const void* bs[2] = {nullptr, nullptr};
+  Launch l{};
+  if ((st = plan_launch(q->dtype, rn::kOpRmsRope, plans, xs, ws, bs, 2, &l))) return st;
+  rn::Params params{};
+  params.seg[0] = make_segment(q, yq, wq, nullptr, plans[0]);
+  params.seg[1] = make_segment(k, yk, wk, nullptr, plans[1]);
+  const int heads[2] = {(int)rope->heads_q, (int)rope->heads_k};
+  for (int i = 0; i < 2; ++i) {
+    params.seg[i].rope_table = rope->table;
+    params.seg[i].rope_offset = rope->offset;
+    params.seg[i].rope_heads = heads[i];
+    params.seg[i].rope_dims = rope->dims;
+    params.seg[i].rope_trad = rope->traditional ? 1 : 0;
+  }
+  params.nseg = 2;
+  params.eps = eps;
+  return launch(l, params, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -699,6 +778,33 @@ RN_API int rn_add_rms_norm(const rn_view* x, const rn_view* residual, const void
 RN_API int rn_gated_rms_norm(const rn_view* x, const rn_view* z, const void* weight, float eps,
                              const rn_view* y, void* stream) {
   return run_second(rn::kOpGatedRms, x, z, weight, eps, y, nullptr, stream, nullptr);
+}
+
+RN_API int rn_dual_head_rms_norm_rope(const rn_view* q, const rn_view* k, const void* wq,
+                                      const void* wk, float eps, const rn_rope* rope,
+                                      const rn_view* yq, const rn_view* yk, void* stream) {
+  return run_dual_rope(q, k, wq, wk, eps, rope, yq, yk, stream);
+}
+
+RN_API int rn_rope_table(int32_t dims, float base, float scale, const float* inv_freq,
+                         int64_t n_pos, float* table) {
+  if (dims < 0 || dims % 2) return fail(RN_ERR_SHAPE, "rope table: dims %d must be even", dims);
+  if (n_pos < 0) return fail(RN_ERR_SHAPE, "rope table: n_pos < 0");
+  if (n_pos > 0 && dims > 0 && !table) return fail(RN_ERR_NULL, "rope table: table is NULL");
+  if (!inv_freq && !(base > 0.0f && std::isfinite(base)))
+    return fail(RN_ERR_EPS, "rope table: base must be finite and > 0");
+  if (!std::isfinite(scale)) return fail(RN_ERR_EPS, "rope table: scale must be finite");
+  const int half = dims / 2;
+  for (int i = 0; i < half; ++i) {
+    const double f = inv_freq ? (double)inv_freq[i]
+                              : std::pow((double)base, -2.0 * (double)i / (double)dims);
+    for (int64_t p = 0; p < n_pos; ++p) {
+      const double theta = (double)p * (double)scale * f;
+      table[p * dims + i] = (float)std::cos(theta);
+      table[p * dims + half + i] = (float)std::sin(theta);
+    }
+  }
+  return RN_OK;
 }
 
 RN_API int rn_dual_head_rms_norm(const rn_view* q, const rn_view* k, const void* wq,

@@ -22,6 +22,12 @@
 //               y_j  = (h_j * rstd) * w_j          use the stored values)
 //               y_j  = ((x_j * rstd) * w_j) * silu(z_j),
 //               silu(t) = t / (1 + exp(-t))       (binary32, __expf called)
+//   Dual q/k head RMSNorm + RoPE ("Emily.Fast", rope/3, rope_with_freqs/4):
+//               o_j  = (x_j * rstd) * w_j          (binary32, not rounded)
+//               plane (a, b), angle theta at the row's position:
+//               y_a  = o_a * cos - o_b * sin,  y_b = o_b * cos + o_a * sin
+//               (each as fma(o_own, cos, -/+ (o_partner * sin)); columns
+//               from rope_dims on: y = o)
 //
 // Row layout. A row is moved as 16-byte chunks on the 16-byte address grid:
 // the columns between the first and the last 16-byte boundary inside the row
@@ -55,7 +61,7 @@
 
 namespace rn {
 
-enum : int { kOpRms = 0, kOpLn = 1, kOpAddRms = 2, kOpGatedRms = 3 };
+enum : int { kOpRms = 0, kOpLn = 1, kOpAddRms = 2, kOpGatedRms = 3, kOpRmsRope = 4 };
 
 // A second input row space read beside x: the residual (kOpAddRms) or the
 // gate (kOpGatedRms).
@@ -99,6 +105,15 @@ struct Segment {
   void* h;
   long long x2_stride;
   long long h_stride;
+  // RoPE after the norm (kOpRmsRope): row r is token r / rope_heads at
+  // position rope_offset + token; rope_table[pos][i] = cos theta_i and
+  // rope_table[pos][rope_dims / 2 + i] = sin theta_i (binary32)
+  const float* rope_table;
+  long long rope_offset;
+  int rope_heads;
+  int rope_dims;
+  int rope_trad;   // 1: planes (2i, 2i + 1); 0: planes (i, i + rope_dims / 2)
+  int rope_pad_;
 };
 
 // ---------------------------------------------------------------------------
@@ -592,6 +607,93 @@ __device__ __forceinline__ void normalize_store(const Segment& s, const Row<T>& 
     if constexpr (OP == kOpGatedRms) o = __fmul_rn(o, silu(gate.edge()));
     Elem<T>::put(g.y_row + edge_column(g, s.dim, k0), o);
   }
+}
+
+// RoPE after the RMSNorm (kOpRmsRope, lane-group rows). The row's normalized,
+// weighted values go to the lane group's staging row in shared memory
+// (`stage`, dim floats); after a sync of the group's lanes (`mask`) each
+// thread reads its own columns and their plane partners back from there,
+// rotates, stores, and syncs again before the staging row is rewritten.
+template <typename T, bool EXACT, int SLOTS, int NSLOT, typename Src>
+__device__ __forceinline__ void normalize_rope_store(const Segment& s, const Row<T>& g,
+                                                     F2 (&v)[NSLOT][Elem<T>::P], float xe,
+                                                     const Src& src, int k0, int step,
+                                                     float rstd, bool has_edge, long long r,
+                                                     float* stage, unsigned mask) {
+  constexpr int V = Elem<T>::V;
+  constexpr int P = Elem<T>::P;
+  const F2 R2 = splat(rstd);
+#pragma unroll
+  for (int p = 0; p < NSLOT; ++p) {
+    const int f = k0 + step * p;
+    if (!slot_present<SLOTS, NSLOT>(p, f, g.nfull)) continue;
+    F2 wf[P], bf[P];
+    src.get(p, f, wf, bf);
+    float* dst = stage + g.head + f * V;
+#pragma unroll
+    for (int j = 0; j < P; ++j) {
+      v[p][j] = mul2(mul2(v[p][j], R2), wf[j]);
+      if constexpr (EXACT) {
+        *reinterpret_cast<float2*>(dst + 2 * j) = v[p][j];
+      } else {
+        dst[2 * j] = v[p][j].x;
+        dst[2 * j + 1] = v[p][j].y;
+      }
+    }
+  }
+  if (!EXACT && has_edge) {
+    float we, be;
+    src.edge(we, be);
+    stage[edge_column(g, s.dim, k0)] = __fmul_rn(__fmul_rn(xe, rstd), we);
+  }
+  __syncwarp(mask);
+  const int dims = s.rope_dims;
+  const int half = dims >> 1;
+  const long long pos = s.rope_offset + r / s.rope_heads;
+  const float* tab = s.rope_table + pos * dims;
+  // column c rotated with its plane partner, both read back from the
+  // staging row (so no value stays in registers across the sync)
+  auto rotate = [&](int c) -> float {
+    const float o = stage[c];
+    if (c >= dims) return o;
+    int i, partner;
+    bool first;
+    if (s.rope_trad) {
+      i = c >> 1;
+      partner = c ^ 1;
+      first = (c & 1) == 0;
+    } else {
+      first = c < half;
+      i = first ? c : c - half;
+      partner = first ? c + half : c - half;
+    }
+    const float t = __fmul_rn(stage[partner], __ldg(tab + half + i));
+    return __fmaf_rn(o, __ldg(tab + i), first ? -t : t);
+  };
+#pragma unroll 1
+  for (int p = 0; p < NSLOT; ++p) {
+    const int f = k0 + step * p;
+    if (!slot_present<SLOTS, NSLOT>(p, f, g.nfull)) continue;
+    const int c0 = g.head + f * V;
+    F2 o[P];
+#pragma unroll
+    for (int j = 0; j < P; ++j) o[j] = make2(rotate(c0 + 2 * j), rotate(c0 + 2 * j + 1));
+    T* yc = g.y_row + c0;
+    if (EXACT || s.vector_y) {
+      store_stream(yc, Elem<T>::pack(o));
+    } else {
+#pragma unroll
+      for (int j = 0; j < P; ++j) {
+        Elem<T>::put(yc + 2 * j, o[j].x);
+        Elem<T>::put(yc + 2 * j + 1, o[j].y);
+      }
+    }
+  }
+  if (!EXACT && has_edge) {
+    const int c = edge_column(g, s.dim, k0);
+    Elem<T>::put(g.y_row + c, rotate(c));
+  }
+  __syncwarp(mask);
 }
 
 // rstd (and mean) of one row from the thread's slots and edge element, with

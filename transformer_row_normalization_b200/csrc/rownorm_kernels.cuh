@@ -36,6 +36,7 @@ struct Params {
   int nseg;
   float eps;
   int prefetch;  // 1: next-row prefetch through shared memory; 0: direct loads
+  int stage_word;  // kOpRmsRope: first 16-byte word of the lane groups' staging rows
 };
 
 __device__ __forceinline__ Segment pick_segment(const Segment (&seg)[2], int i) {
@@ -164,7 +165,8 @@ template <typename T, int OP, bool EXACT, int SLOTS, int NSLOT, int NST, typenam
 __device__ __forceinline__ void segment_rows(const Segment& s, const Prefetch<T, NSLOT>& pf,
                                              const Prefetch<T, NSLOT>& pf2, long long r0,
                                              long long stride, int k0, int step, float eps,
-                                             Reduce reduce, Src& src) {
+                                             Reduce reduce, Src& src, float* stage,
+                                             unsigned mask) {
   static_assert(NST >= 2, "at least one row ahead");
   constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
@@ -251,6 +253,9 @@ __device__ __forceinline__ void segment_rows(const Segment& s, const Prefetch<T,
       const GateSrc<T, NSLOT> gate{&pf2, x2_row_of<T>(s, r) + g.head, st, x2e};
       normalize_store<T, OP, EXACT, SLOTS, NSLOT>(s, g, v, xe, src, k0, step, rstd, mean,
                                                   has_edge, gate);
+    } else if constexpr (OP == kOpRmsRope) {
+      normalize_rope_store<T, EXACT, SLOTS, NSLOT>(s, g, v, xe, src, k0, step, rstd, has_edge,
+                                                   r, stage, mask);
     } else {
       normalize_store<T, OP, EXACT, SLOTS, NSLOT>(s, g, v, xe, src, k0, step, rstd, mean,
                                                   has_edge);
@@ -268,7 +273,8 @@ template <typename T, int OP, bool EXACT, int SLOTS, int NSLOT, int NST, typenam
 __device__ __forceinline__ void run_segment(const Segment& s, const Prefetch<T, NSLOT>& pf,
                                             const Prefetch<T, NSLOT>& pf2, long long r0,
                                             long long stride, int k0, int step, float eps,
-                                            Reduce reduce, int cache_word) {
+                                            Reduce reduce, int cache_word, float* stage,
+                                            unsigned mask) {
   constexpr bool BIAS = OP == kOpLn;
   static_assert(EXACT || SLOTS != kSlotsFull, "only EXACT rows divide evenly");
   const T* w = static_cast<const T*>(s.w);
@@ -277,17 +283,17 @@ __device__ __forceinline__ void run_segment(const Segment& s, const Prefetch<T, 
     if (w && (!BIAS || b)) {
       AffineDirect<T, BIAS, true> src{w, b};
       segment_rows<T, OP, true, SLOTS, NSLOT, NST>(s, pf, pf2, r0, stride, k0, step, eps, reduce,
-                                                   src);
+                                                   src, stage, mask);
     } else {
       AffineDirect<T, BIAS, false> src{w, b};
       segment_rows<T, OP, true, SLOTS, NSLOT, NST>(s, pf, pf2, r0, stride, k0, step, eps, reduce,
-                                                   src);
+                                                   src, stage, mask);
     }
   } else {
     AffineCache<T, NSLOT, BIAS> src;
     src.init(cache_word);
     segment_rows<T, OP, false, SLOTS, NSLOT, NST>(s, pf, pf2, r0, stride, k0, step, eps, reduce,
-                                                  src);
+                                                  src, stage, mask);
   }
 }
 
@@ -310,8 +316,13 @@ rows_warp_kernel(const Params p) {
     const int gi = lane / G;
     const unsigned mask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << (gi * G));
     auto reduce = [&](float t) { return group_sum(t, G, mask); };
+    float* stage = nullptr;
+    if constexpr (OP == kOpRmsRope)
+      stage = reinterpret_cast<float*>(dyn_smem + p.stage_word) +
+              ((threadIdx.x >> 5) * per_warp + gi) * s.dim;
     run_segment<T, OP, EXACT, SLOTS, VPL, kWarpPrefetchStages>(
-        s, pf, pf2, warp * per_warp + gi, nwarps * per_warp, gl, G, p.eps, reduce, cache_word);
+        s, pf, pf2, warp * per_warp + gi, nwarps * per_warp, gl, G, p.eps, reduce, cache_word,
+        stage, mask);
   }
 }
 
@@ -319,6 +330,7 @@ template <typename T, int OP, bool EXACT, int SLOTS, int NT, int VPT>
 __global__ void __launch_bounds__(NT, kMinThreadsPerSm / NT)
 rows_cta_kernel(const Params p) {
   static_assert(NT >= 2 * (Elem<T>::V - 1), "every edge element needs its own thread");
+  static_assert(OP != kOpRmsRope, "RoPE rows are head rows: lane groups only");
   // Two alternating reduction buffers: a buffer is rewritten only after every
   // thread has passed the barrier of the reduction in between.
   __shared__ float red[2][NT / 32];
@@ -336,7 +348,8 @@ rows_cta_kernel(const Params p) {
   for (int si = 0; si < p.nseg; ++si) {
     const Segment s = pick_segment(p.seg, si);
     run_segment<T, OP, EXACT, SLOTS, VPT, kCtaPrefetchStages>(
-        s, pf, pf2, blockIdx.x, gridDim.x, threadIdx.x, NT, p.eps, reduce, cache_word);
+        s, pf, pf2, blockIdx.x, gridDim.x, threadIdx.x, NT, p.eps, reduce, cache_word, nullptr,
+        0u);
   }
 }
 

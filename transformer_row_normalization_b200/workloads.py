@@ -30,6 +30,10 @@ comment), at the shapes of the rows they fuse with:
                               prefill token count: x, z N(0,1), w N(1, 0.1).
   add_rms_f32_4x128x1024,     the same two ops at the small f32 shape of the
   gated_rms_f32_4x128x1024    Part 1 Correctness cell (x, r/z U(-1,1)).
+  dual_rope_bf16_prefill      the dual q/k head norm followed by RoPE
+                              ("Emily.Fast", rope/3): the prefill heads above,
+                              positions 0..8191, base 10000, all 128 columns
+                              rotated, split-half planes.
 """
 from dataclasses import dataclass, field
 from typing import Dict, Optional, Tuple
@@ -43,7 +47,7 @@ CONSTANT_ROW_PERIOD = 64
 @dataclass(frozen=True)
 class Workload:
     name: str
-    op: str                      # "rms", "ln", "dual", "add_rms" or "gated_rms"
+    op: str                      # "rms", "ln", "dual", "dual_rope", "add_rms", "gated_rms"
     dtype: torch.dtype
     shape: Tuple[int, ...]       # x (or q) shape; last axis is the row
     eps: float
@@ -82,10 +86,13 @@ class Workload:
     def algorithmic_bytes(self) -> int:
         """Read x + write y + read each per-column vector once."""
         s = self.element_size
-        if self.op == "dual":
+        if self.op in ("dual", "dual_rope"):
             kd = self.k_shape[-1]
-            return (2 * self.rows * self.dim * s + self.dim * s
-                    + 2 * self.k_rows * kd * s + kd * s)
+            b = (2 * self.rows * self.dim * s + self.dim * s
+                 + 2 * self.k_rows * kd * s + kd * s)
+            if self.op == "dual_rope":  # the cos/sin rows of the positions used
+                b += self.shape[0] * self.meta["rope_dims"] * 4
+            return b
         if self.op == "add_rms":   # read x, r; write y, h
             return 4 * self.rows * self.dim * s + self.dim * s
         if self.op == "gated_rms":  # read x, z; write y
@@ -116,6 +123,8 @@ _register(Workload("add_rms_bf16_16x4096x4096", "add_rms", torch.bfloat16, (16, 
                    1e-5, 60))
 _register(Workload("gated_rms_bf16_8192x32x128", "gated_rms", torch.bfloat16, (8192, 32, 128),
                    1e-6, 61))
+_register(Workload("dual_rope_bf16_prefill", "dual_rope", torch.bfloat16, (8192, 32, 128), 1e-6,
+                   64, k_shape=(8192, 8, 128), meta={"rope_dims": 128, "rope_base": 10000.0}))
 _register(Workload("add_rms_f32_4x128x1024", "add_rms", torch.float32, (4, 128, 1024), 1e-6, 62))
 _register(Workload("gated_rms_f32_4x128x1024", "gated_rms", torch.float32, (4, 128, 1024),
                    1e-6, 63))
@@ -125,7 +134,8 @@ LARGE_SUITE = ("dual_bf16_prefill", "rms_bf16_16x4096x4096") + tuple(
     f"ln_bf16_65536x{d}" for d in LN_WIDTHS)
 SMALL_SUITE = ("rms_f32_4x128x1024", "ln_f32_1x1024x768", "dual_bf16_decode")
 # The fused extensions, measured beside (not inside) the benchmark step.
-FUSED_SUITE = ("add_rms_bf16_16x4096x4096", "gated_rms_bf16_8192x32x128")
+FUSED_SUITE = ("add_rms_bf16_16x4096x4096", "gated_rms_bf16_8192x32x128",
+               "dual_rope_bf16_prefill")
 
 
 def _gen(device, seed):
@@ -155,7 +165,7 @@ def make_inputs(w: Workload, device="cpu") -> Dict[str, torch.Tensor]:
         out["x"] = _uniform(w.shape, -1.0, 1.0, g, device)
         out["w"] = _uniform((w.dim,), 0.5, 1.5, g, device)
         out["b"] = _uniform((w.dim,), -0.1, 0.1, g, device)
-    elif w.op == "dual":
+    elif w.op in ("dual", "dual_rope"):
         out["q"] = _normal(w.shape, 0.0, 1.0, g, device)
         out["k"] = _normal(w.k_shape, 0.0, 1.0, g, device)
         out["wq"] = _normal((w.dim,), 1.0, 0.1, g, device)
