@@ -315,8 +315,8 @@ def cpu_baseline(step, chunk_rows=2048):
 
 
 def time_fused(device, rank, dist, peak, reps=30, oracle_rows=2048):
-    """The fused extensions (residual-add RMSNorm, gated RMSNorm), measured
-    beside the step: the median CUDA-event time of single launches on the
+    """The fused extensions (residual-add RMSNorm, gated RMSNorm, dual head
+    RMSNorm + RoPE), measured beside the step: the median CUDA-event time of single launches on the
     launching stream, each after a 256 MB read that evicts L2 (max over
     ranks), and on rank 0 the fp64 oracle's rows/s on the first
     `oracle_rows` rows on all host cores."""
@@ -326,48 +326,70 @@ def time_fused(device, rank, dist, peak, reps=30, oracle_rows=2048):
     out = []
     for name in wl.FUSED_SUITE:
         w = wl.WORKLOADS[name]
-        rw = wl.Workload(w.name, w.op, w.dtype, w.shape, w.eps, rank_seed(w.seed, rank))
+        rw = wl.Workload(w.name, w.op, w.dtype, w.shape, w.eps, rank_seed(w.seed, rank),
+                         k_shape=w.k_shape, meta=w.meta)
         a = wl.make_inputs(rw, device=device)
-        second = a["r"] if w.op == "add_rms" else a["z"]
-        y, h = torch.empty_like(a["x"]), torch.empty_like(a["x"])
+        if w.op == "dual_rope":
+            table = rn.rope_table(w.meta["rope_dims"], w.shape[0], base=w.meta["rope_base"],
+                                  device=device)
+            yq, yk = torch.empty_like(a["q"]), torch.empty_like(a["k"])
 
-        def launch():
-            if w.op == "add_rms":
-                rn.add_rms_norm(a["x"], second, a["w"], w.eps, out=y, out_h=h)
-            else:
-                rn.gated_rms_norm(a["x"], second, a["w"], w.eps, out=y)
+            def launch():
+                rn.dual_head_rms_norm_rope(a["q"], a["k"], a["wq"], a["wk"], w.eps, table, 0,
+                                           w.meta["rope_dims"], out_q=yq, out_k=yk)
+        else:
+            second = a["r"] if w.op == "add_rms" else a["z"]
+            y, h = torch.empty_like(a["x"]), torch.empty_like(a["x"])
+
+            def launch():
+                if w.op == "add_rms":
+                    rn.add_rms_norm(a["x"], second, a["w"], w.eps, out=y, out_h=h)
+                else:
+                    rn.gated_rms_norm(a["x"], second, a["w"], w.eps, out=y)
 
         for _ in range(3):
             launch()
-        times = []
-        for _ in range(reps):
+        # all reps queued before any is read back: the host stays ahead of the
+        # GPU (each eviction read takes ~40 us), so no launch waits on the host
+        # inside its event pair
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(reps)]
+        for s, e in ev:
             evict.sum()
-            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             s.record()
             launch()
             e.record()
-            e.synchronize()
-            times.append(s.elapsed_time(e))
+        torch.cuda.synchronize(device)
+        times = [s.elapsed_time(e) for s, e in ev]
         t = max_over_ranks(sorted(times)[len(times) // 2], dist, device)
         g = w.algorithmic_bytes() / (t * 1e-3) / 1e9
         item = {"workload": name, "us": round(t * 1e3, 2),
-                "rows_per_s": round(w.rows / (t * 1e-3)), "gbs": round(g, 1),
+                "rows_per_s": round(w.total_rows / (t * 1e-3)), "gbs": round(g, 1),
                 "frac": round(g / peak, 4), "algorithmic_bytes": w.algorithmic_bytes()}
         if rank == 0:
             import oracle
-            x = a["x"].reshape(-1, w.dim)[:oracle_rows].cpu()
-            x2 = second.reshape(-1, w.dim)[:oracle_rows].cpu()
-            wt = a["w"].cpu()
-            fn = oracle.add_rms_norm if w.op == "add_rms" else oracle.gated_rms_norm
-            fn(x[:64], x2[:64], wt, w.eps, nthreads=cores)  # warm-up
+            if w.op == "dual_rope":
+                # whole tokens: oracle_rows // 40 tokens of 32 query + 8 key heads
+                nt = max(1, oracle_rows // 40)
+                args = (a["q"].reshape(-1, w.dim)[:nt * 32].cpu(),
+                        a["k"].reshape(-1, w.dim)[:nt * 8].cpu(), a["wq"].cpu(), a["wk"].cpu(),
+                        w.eps, 32, 8, 0, w.meta["rope_dims"])
+                fn, nrows = oracle.dual_head_rms_norm_rope, nt * 40
+            else:
+                x = a["x"].reshape(-1, w.dim)[:oracle_rows].cpu()
+                x2 = second.reshape(-1, w.dim)[:oracle_rows].cpu()
+                args = (x, x2, a["w"].cpu(), w.eps)
+                fn = oracle.add_rms_norm if w.op == "add_rms" else oracle.gated_rms_norm
+                nrows = x.shape[0]
+            fn(*args, nthreads=cores)  # warm-up
             t0 = time.perf_counter()
-            fn(x, x2, wt, w.eps, nthreads=cores)
+            fn(*args, nthreads=cores)
             busy = time.perf_counter() - t0
-            item["oracle_rows_per_s"] = round(x.shape[0] / busy, 1)
+            item["oracle_rows_per_s"] = round(nrows / busy, 1)
         out.append(item)
     return {"workloads": out, "cores": cores,
-            "timing": f"median of {reps} single launches, each after a 256 MB read "
-                      "that evicts L2; oracle on the first "
+            "timing": f"median of {reps} single launches (queued back to back), each after "
+                      "a 256 MB read that evicts L2; oracle on the first "
                       f"{oracle_rows} rows, fp64, {cores} threads"}
 
 

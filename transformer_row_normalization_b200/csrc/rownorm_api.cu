@@ -738,8 +738,22 @@ int run_dual_rope(const rn_view* q, const rn_view* k, const void* wq, const void
   const rn_view* xs[2] = {q, k};
   const void* ws[2] = {wq, wk};
   const void* bs[2] = {nullptr, nullptr};
+  // in-thread planes when every plane's partner is the same thread's: on
+  // 16-byte aligned rows whose rotated width is a multiple of 2 V, either
+  // interleaved planes, or full split-half rotary whose chunks divide evenly
+  // over an even slot count (slot p's partner is slot p + slots / 2)
+  const int V = 16 / elem_size(q->dtype);
+  const int slots = plans[0].chunks > plans[1].chunks ? plans[0].chunks : plans[1].chunks;
+  bool local = rope->dims > 0 && rope->dims % (2 * V) == 0;
+  for (int i = 0; i < 2; ++i) {
+    local = local && plans[i].exact;
+    if (!rope->traditional)
+      local = local && slots % 2 == 0 && rope->dims / 2 == plans[i].lanes * (slots / 2) * V;
+  }
   Launch l{};
-  if ((st = plan_launch(q->dtype, rn::kOpRmsRope, plans, xs, ws, bs, 2, &l))) return st;
+  if ((st = plan_launch(q->dtype, local ? rn::kOpRmsRopeLocal : rn::kOpRmsRope, plans, xs, ws,
+                        bs, 2, &l)))
+    return st;
   rn::Params params{};
   params.seg[0] = make_segment(q, yq, wq, nullptr, plans[0]);
   params.seg[1] = make_segment(k, yk, wk, nullptr, plans[1]);

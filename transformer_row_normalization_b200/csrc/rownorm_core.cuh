@@ -61,7 +61,17 @@
 
 namespace rn {
 
-enum : int { kOpRms = 0, kOpLn = 1, kOpAddRms = 2, kOpGatedRms = 3, kOpRmsRope = 4 };
+enum : int {
+  kOpRms = 0,
+  kOpLn = 1,
+  kOpAddRms = 2,
+  kOpGatedRms = 3,
+  kOpRmsRope = 4,       // RMSNorm + RoPE, plane partners through shared memory
+  kOpRmsRopeLocal = 5,  // RMSNorm + RoPE, every plane's partner in the same thread
+};
+__host__ __device__ constexpr bool op_is_rope(int op) {
+  return op == kOpRmsRope || op == kOpRmsRopeLocal;
+}
 
 // A second input row space read beside x: the residual (kOpAddRms) or the
 // gate (kOpGatedRms).
@@ -609,12 +619,59 @@ __device__ __forceinline__ void normalize_store(const Segment& s, const Row<T>& 
   }
 }
 
-// RoPE after the RMSNorm (kOpRmsRope, lane-group rows). The row's normalized,
-// weighted values go to the lane group's staging row in shared memory
-// (`stage`, dim floats); after a sync of the group's lanes (`mask`) each
-// thread reads its own columns and their plane partners back from there,
+// RoPE after the RMSNorm (kOpRmsRope, lane-group rows). Each thread forms
+// the normalized, weighted values o of its columns (binary32). A column's
+// plane partner is usually another thread's, so the values go to the lane
+// group's staging row in shared memory (`stage`, dim floats) and, after a
+// sync of the group's lanes (`mask`), each thread reads its partners back,
 // rotates, stores, and syncs again before the staging row is rewritten.
-template <typename T, bool EXACT, int SLOTS, int NSLOT, typename Src>
+// Aligned rows (EXACT, dims a multiple of 2 V) take whole chunks at a time:
+// a chunk lies in one half of the rotated columns, so its partners and its
+// cos / sin are contiguous 16-byte vectors; interleaved planes need no
+// staging at all (both values of a plane are one pair of the thread's), nor
+// does full split-half rotary whose chunks divide evenly over the threads
+// (a chunk's partner chunk is then the same thread's). Every path computes
+// the same operations, so the bits do not depend on the path.
+template <int N>
+__device__ __forceinline__ void load_floats(const float* p, float (&d)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; i += 4) {
+    const float4 t = *reinterpret_cast<const float4*>(p + i);
+    d[i] = t.x;
+    d[i + 1] = t.y;
+    d[i + 2] = t.z;
+    d[i + 3] = t.w;
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void ldg_floats(const float* p, float (&d)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; i += 4) {
+    const float4 t = __ldg(reinterpret_cast<const float4*>(p + i));
+    d[i] = t.x;
+    d[i + 1] = t.y;
+    d[i + 2] = t.z;
+    d[i + 3] = t.w;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void store_chunk(const Segment& s, T* yc, const F2 (&o)[Elem<T>::P],
+                                            bool vector) {
+  constexpr int P = Elem<T>::P;
+  if (vector) {
+    store_stream(yc, Elem<T>::pack(o));
+  } else {
+#pragma unroll
+    for (int j = 0; j < P; ++j) {
+      Elem<T>::put(yc + 2 * j, o[j].x);
+      Elem<T>::put(yc + 2 * j + 1, o[j].y);
+    }
+  }
+}
+
+template <typename T, bool LOCAL, bool EXACT, int SLOTS, int NSLOT, typename Src>
 __device__ __forceinline__ void normalize_rope_store(const Segment& s, const Row<T>& g,
                                                      F2 (&v)[NSLOT][Elem<T>::P], float xe,
                                                      const Src& src, int k0, int step,
@@ -622,7 +679,88 @@ __device__ __forceinline__ void normalize_rope_store(const Segment& s, const Row
                                                      float* stage, unsigned mask) {
   constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
+  const int dims = s.rope_dims;
+  const int half = dims >> 1;
+  const bool trad = s.rope_trad != 0;
+  // whole-chunk rotation: every chunk lies in one half (or past dims), and
+  // every vector access below is 16-byte aligned
+  const bool vec = EXACT && dims % (2 * V) == 0;
+  static_assert(!LOCAL || EXACT, "in-thread planes need 16-byte aligned rows");
+  const bool vstore = EXACT || s.vector_y;
   const F2 R2 = splat(rstd);
+  // token = r / heads (32-bit division: head rows never reach 2^31)
+  const long long token = r < 0x7fffffffLL ? (long long)((unsigned)r / (unsigned)s.rope_heads)
+                                           : r / s.rope_heads;
+  const float* tab = s.rope_table + (s.rope_offset + token) * dims;
+  if constexpr (LOCAL && NSLOT % 2 == 0) {
+    if (!trad) {
+      // full split-half rotary whose chunks divide evenly: slot p < NSLOT/2
+      // holds chunk f of the first half, slot p + NSLOT/2 its partner chunk
+      // f + half / V (same planes, same cos / sin); all slots are present
+      // (dims / V = step * NSLOT full chunks), nothing is staged
+#pragma unroll
+      for (int p = 0; p < NSLOT; ++p) {
+        F2 wf[P], bf[P];
+        src.get(p, k0 + step * p, wf, bf);
+#pragma unroll
+        for (int j = 0; j < P; ++j) v[p][j] = mul2(mul2(v[p][j], R2), wf[j]);
+      }
+#pragma unroll
+      for (int p = 0; p < NSLOT / 2; ++p) {
+        const int c0 = (k0 + step * p) * V;
+        float cs[V], sn[V];
+        ldg_floats<V>(tab + c0, cs);
+        ldg_floats<V>(tab + half + c0, sn);
+        F2 ya[P], yb[P];
+#pragma unroll
+        for (int j = 0; j < P; ++j) {
+          const F2 a = v[p][j], b = v[p + NSLOT / 2][j];
+          ya[j] = make2(__fmaf_rn(a.x, cs[2 * j], -__fmul_rn(b.x, sn[2 * j])),
+                        __fmaf_rn(a.y, cs[2 * j + 1], -__fmul_rn(b.y, sn[2 * j + 1])));
+          yb[j] = make2(__fmaf_rn(b.x, cs[2 * j], __fmul_rn(a.x, sn[2 * j])),
+                        __fmaf_rn(b.y, cs[2 * j + 1], __fmul_rn(a.y, sn[2 * j + 1])));
+        }
+        store_chunk<T>(s, g.y_row + c0, ya, vstore);
+        store_chunk<T>(s, g.y_row + c0 + half, yb, vstore);
+      }
+      return;
+    }
+  }
+  if constexpr (LOCAL) {
+    // planes (c0 + 2j, c0 + 2j + 1) are pairs of this thread's own chunk:
+    // rotate as the chunk is normalized, nothing staged
+#pragma unroll
+    for (int p = 0; p < NSLOT; ++p) {
+      const int f = k0 + step * p;
+      if (!slot_present<SLOTS, NSLOT>(p, f, g.nfull)) continue;
+      F2 wf[P], bf[P], o[P];
+      src.get(p, f, wf, bf);
+      const int c0 = f * V;
+#pragma unroll
+      for (int j = 0; j < P; ++j) o[j] = mul2(mul2(v[p][j], R2), wf[j]);
+      if (c0 < dims) {
+        float cs[P], sn[P];
+        if constexpr (P % 4 == 0) {
+          ldg_floats<P>(tab + (c0 >> 1), cs);
+          ldg_floats<P>(tab + half + (c0 >> 1), sn);
+        } else {
+#pragma unroll
+          for (int j = 0; j < P; ++j) {
+            cs[j] = __ldg(tab + (c0 >> 1) + j);
+            sn[j] = __ldg(tab + half + (c0 >> 1) + j);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < P; ++j) {
+          const float a = o[j].x, b = o[j].y;
+          o[j] = make2(__fmaf_rn(a, cs[j], -__fmul_rn(b, sn[j])),
+                       __fmaf_rn(b, cs[j], __fmul_rn(a, sn[j])));
+        }
+      }
+      store_chunk<T>(s, g.y_row + c0, o, vstore);
+    }
+    return;
+  }
 #pragma unroll
   for (int p = 0; p < NSLOT; ++p) {
     const int f = k0 + step * p;
@@ -632,12 +770,12 @@ __device__ __forceinline__ void normalize_rope_store(const Segment& s, const Row
     float* dst = stage + g.head + f * V;
 #pragma unroll
     for (int j = 0; j < P; ++j) {
-      v[p][j] = mul2(mul2(v[p][j], R2), wf[j]);
+      const F2 o = mul2(mul2(v[p][j], R2), wf[j]);
       if constexpr (EXACT) {
-        *reinterpret_cast<float2*>(dst + 2 * j) = v[p][j];
+        *reinterpret_cast<float2*>(dst + 2 * j) = o;
       } else {
-        dst[2 * j] = v[p][j].x;
-        dst[2 * j + 1] = v[p][j].y;
+        dst[2 * j] = o.x;
+        dst[2 * j + 1] = o.y;
       }
     }
   }
@@ -647,18 +785,13 @@ __device__ __forceinline__ void normalize_rope_store(const Segment& s, const Row
     stage[edge_column(g, s.dim, k0)] = __fmul_rn(__fmul_rn(xe, rstd), we);
   }
   __syncwarp(mask);
-  const int dims = s.rope_dims;
-  const int half = dims >> 1;
-  const long long pos = s.rope_offset + r / s.rope_heads;
-  const float* tab = s.rope_table + pos * dims;
-  // column c rotated with its plane partner, both read back from the
-  // staging row (so no value stays in registers across the sync)
+  // column c rotated with its plane partner, both read from the staging row
   auto rotate = [&](int c) -> float {
     const float o = stage[c];
     if (c >= dims) return o;
     int i, partner;
     bool first;
-    if (s.rope_trad) {
+    if (trad) {
       i = c >> 1;
       partner = c ^ 1;
       first = (c & 1) == 0;
@@ -670,24 +803,36 @@ __device__ __forceinline__ void normalize_rope_store(const Segment& s, const Row
     const float t = __fmul_rn(stage[partner], __ldg(tab + half + i));
     return __fmaf_rn(o, __ldg(tab + i), first ? -t : t);
   };
+  // one chunk at a time: its own, partner and cos / sin vectors are 32
+  // floats in flight, kept out of the next chunk's registers
 #pragma unroll 1
   for (int p = 0; p < NSLOT; ++p) {
     const int f = k0 + step * p;
     if (!slot_present<SLOTS, NSLOT>(p, f, g.nfull)) continue;
     const int c0 = g.head + f * V;
     F2 o[P];
+    if (vec && c0 < dims) {
+      // split-half, whole chunk: its partners are the chunk half a
+      // rotated width away
+      const bool first = c0 < half;
+      const int i0 = first ? c0 : c0 - half;
+      float own[V], pt[V], cs[V], sn[V];
+      load_floats<V>(stage + c0, own);
+      load_floats<V>(stage + (first ? c0 + half : c0 - half), pt);
+      ldg_floats<V>(tab + i0, cs);
+      ldg_floats<V>(tab + half + i0, sn);
 #pragma unroll
-    for (int j = 0; j < P; ++j) o[j] = make2(rotate(c0 + 2 * j), rotate(c0 + 2 * j + 1));
-    T* yc = g.y_row + c0;
-    if (EXACT || s.vector_y) {
-      store_stream(yc, Elem<T>::pack(o));
+      for (int j = 0; j < V; j += 2) {
+        const float t0 = __fmul_rn(pt[j], sn[j]);
+        const float t1 = __fmul_rn(pt[j + 1], sn[j + 1]);
+        o[j / 2] = make2(__fmaf_rn(own[j], cs[j], first ? -t0 : t0),
+                         __fmaf_rn(own[j + 1], cs[j + 1], first ? -t1 : t1));
+      }
     } else {
 #pragma unroll
-      for (int j = 0; j < P; ++j) {
-        Elem<T>::put(yc + 2 * j, o[j].x);
-        Elem<T>::put(yc + 2 * j + 1, o[j].y);
-      }
+      for (int j = 0; j < P; ++j) o[j] = make2(rotate(c0 + 2 * j), rotate(c0 + 2 * j + 1));
     }
+    store_chunk<T>(s, g.y_row + c0, o, vstore);
   }
   if (!EXACT && has_edge) {
     const int c = edge_column(g, s.dim, k0);

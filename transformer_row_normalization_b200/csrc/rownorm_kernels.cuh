@@ -253,9 +253,9 @@ __device__ __forceinline__ void segment_rows(const Segment& s, const Prefetch<T,
       const GateSrc<T, NSLOT> gate{&pf2, x2_row_of<T>(s, r) + g.head, st, x2e};
       normalize_store<T, OP, EXACT, SLOTS, NSLOT>(s, g, v, xe, src, k0, step, rstd, mean,
                                                   has_edge, gate);
-    } else if constexpr (OP == kOpRmsRope) {
-      normalize_rope_store<T, EXACT, SLOTS, NSLOT>(s, g, v, xe, src, k0, step, rstd, has_edge,
-                                                   r, stage, mask);
+    } else if constexpr (op_is_rope(OP)) {
+      normalize_rope_store<T, OP == kOpRmsRopeLocal, EXACT, SLOTS, NSLOT>(
+          s, g, v, xe, src, k0, step, rstd, has_edge, r, stage, mask);
     } else {
       normalize_store<T, OP, EXACT, SLOTS, NSLOT>(s, g, v, xe, src, k0, step, rstd, mean,
                                                   has_edge);
@@ -317,7 +317,7 @@ rows_warp_kernel(const Params p) {
     const unsigned mask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << (gi * G));
     auto reduce = [&](float t) { return group_sum(t, G, mask); };
     float* stage = nullptr;
-    if constexpr (OP == kOpRmsRope)
+    if constexpr (OP == kOpRmsRope)  // the in-thread variant stages nothing
       stage = reinterpret_cast<float*>(dyn_smem + p.stage_word) +
               ((threadIdx.x >> 5) * per_warp + gi) * s.dim;
     run_segment<T, OP, EXACT, SLOTS, VPL, kWarpPrefetchStages>(
@@ -330,7 +330,7 @@ template <typename T, int OP, bool EXACT, int SLOTS, int NT, int VPT>
 __global__ void __launch_bounds__(NT, kMinThreadsPerSm / NT)
 rows_cta_kernel(const Params p) {
   static_assert(NT >= 2 * (Elem<T>::V - 1), "every edge element needs its own thread");
-  static_assert(OP != kOpRmsRope, "RoPE rows are head rows: lane groups only");
+  static_assert(!op_is_rope(OP), "RoPE rows are head rows: lane groups only");
   // Two alternating reduction buffers: a buffer is rewritten only after every
   // thread has passed the barrier of the reduction in between.
   __shared__ float red[2][NT / 32];
