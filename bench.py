@@ -547,35 +547,62 @@ def run_reference(args):
 
 def run_profile_case(args):
     """One workload, launched --steps times after --warmup launches, for
-    profiler captures: OP:DTYPE:ROWS:DIM, e.g. ln:bf16:8192:16384. Prints the
-    median CUDA-event time per launch (each launch after a 256 MB read that
-    evicts L2) on stderr; this is not the benchmark line."""
+    profiler captures: OP:DTYPE:ROWS:DIM with OP one of rms, ln, add_rms,
+    gated_rms, dual, dual_rope (for the dual ops ROWS counts tokens of 32
+    query and 8 key heads of DIM columns; RoPE rotates all DIM columns,
+    split-half, base 10000, positions 0..ROWS-1). Prints the median
+    CUDA-event time per launch (each launch after a 256 MB read that evicts
+    L2) on stderr; this is not the benchmark line."""
     import transformer_row_normalization_b200 as rn
     op, dt, rows, dim = args.profile_case.split(":")
     dtype = torch.bfloat16 if dt == "bf16" else torch.float32
     rows, dim = int(rows), int(dim)
     device = torch.device("cuda", 0)
-    x = wl.random_rows(rows, dim, dtype, seed=1, device=device, mean=0.5, std=2.0)
-    w = wl.random_vector(dim, dtype, seed=2, device=device)
-    b = wl.random_vector(dim, dtype, seed=3, device=device, mean=0.0, std=0.1)
-    y = torch.empty_like(x)
     rn.set_path_override(args.path)
+    if op in ("dual", "dual_rope"):
+        q = wl.random_rows(rows * 32, dim, dtype, seed=1, device=device)
+        k = wl.random_rows(rows * 8, dim, dtype, seed=2, device=device)
+        wq = wl.random_vector(dim, dtype, seed=3, device=device)
+        wk = wl.random_vector(dim, dtype, seed=4, device=device)
+        yq, yk = torch.empty_like(q), torch.empty_like(k)
+        table = rn.rope_table(dim, rows, device=device) if op == "dual_rope" else None
+        plan = rn.plan(rn.RN_OP_DUAL, q, weight=wq, bias=wk, k=k)
+
+        def launch():
+            if op == "dual":
+                rn.dual_head_rms_norm(q, k, wq, wk, 1e-6, out_q=yq, out_k=yk)
+            else:
+                rn.dual_head_rms_norm_rope(q, k, wq, wk, 1e-6, table, 0, dim, heads_q=32,
+                                           heads_k=8, out_q=yq, out_k=yk)
+    else:
+        x = wl.random_rows(rows, dim, dtype, seed=1, device=device, mean=0.5, std=2.0)
+        w = wl.random_vector(dim, dtype, seed=2, device=device)
+        b = wl.random_vector(dim, dtype, seed=3, device=device, mean=0.0, std=0.1)
+        x2 = wl.random_rows(rows, dim, dtype, seed=4, device=device)
+        y, h = torch.empty_like(x), torch.empty_like(x)
+        plan = rn.plan(rn.RN_OP_LN if op == "ln" else rn.RN_OP_RMS, x, weight=w,
+                       bias=b if op == "ln" else None)
+
+        def launch():
+            if op == "rms":
+                rn.rms_norm(x, w, 1e-5, out=y)
+            elif op == "ln":
+                rn.layer_norm(x, w, b, 1e-5, out=y)
+            elif op == "add_rms":
+                rn.add_rms_norm(x, x2, w, 1e-5, out=y, out_h=h)
+            else:
+                rn.gated_rms_norm(x, x2, w, 1e-5, out=y)
     evict = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=device)
     times = []
     for i in range(args.warmup + args.steps):
         evict.sum()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record()
-        if op == "rms":
-            rn.rms_norm(x, w, 1e-5, out=y)
-        else:
-            rn.layer_norm(x, w, b, 1e-5, out=y)
+        launch()
         e.record()
         torch.cuda.synchronize()
         if i >= args.warmup:
             times.append(s.elapsed_time(e) * 1e3)
-    plan = rn.plan(rn.RN_OP_LN if op == "ln" else rn.RN_OP_RMS, x, weight=w,
-                   bias=b if op == "ln" else None)
     log(f"{args.profile_case} path={args.path} median {sorted(times)[len(times) // 2]:.1f} us "
         f"plan={plan} timeouts={rn.device_error_count()}")
 
