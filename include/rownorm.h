@@ -65,7 +65,7 @@ extern "C" {
 #define RN_API
 #endif
 
-#define RN_ABI_VERSION 2
+#define RN_ABI_VERSION 3
 
 /* Largest supported dim. Rows are held on chip (registers) between reading
  * and writing, so x is read from HBM exactly once; wider rows are rejected
@@ -93,12 +93,28 @@ typedef enum rn_status {
                             /* query or launch); see rn_last_error()          */
 } rn_status;
 
+/*
+ * A [rows, dim] view whose last axis is contiguous. Rows either sit
+ * row_stride elements apart (inner_rows = 0), or form blocks of inner_rows
+ * rows: row r starts at (r / inner_rows) * outer_stride + (r % inner_rows)
+ * * row_stride elements from data. The second form describes head rows
+ * sliced out of a packed buffer, e.g. the query heads [tokens, Hq, D] of a
+ * [tokens, (Hq + 2 Hk) * D] QKV projection ("kernel_micro_ab.rs", section 2:
+ * the packed QKV op writes the head buffers): inner_rows = Hq, row_stride =
+ * D, outer_stride = (Hq + 2 Hk) * D. The norm stays on the last axis
+ * ("Emily.Bumblebee.FastKernels", What's not rewritten); only the row layout
+ * widens.
+ */
 typedef struct rn_view {
-    void *data;         /* device pointer to element [0, 0]                 */
-    int64_t rows;       /* number of rows, >= 0                              */
-    int64_t dim;        /* elements per row (the normalized axis), >= 1      */
-    int64_t row_stride; /* elements between the starts of consecutive rows  */
-    int32_t dtype;      /* rn_dtype                                          */
+    void *data;           /* device pointer to element [0, 0]                 */
+    int64_t rows;         /* number of rows, >= 0                              */
+    int64_t dim;          /* elements per row (the normalized axis), >= 1      */
+    int64_t row_stride;   /* elements between the starts of consecutive rows  */
+                          /* (of one block when inner_rows > 0)               */
+    int32_t dtype;        /* rn_dtype                                          */
+    int64_t inner_rows;   /* 0: one row stride; > 0: rows per block            */
+    int64_t outer_stride; /* inner_rows > 0: elements between block starts;   */
+                          /* >= (inner_rows - 1) * row_stride + dim            */
 } rn_view;
 
 /*

@@ -53,7 +53,7 @@ def test_only_declared_symbols_are_exported(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.rn_abi_version() == 2
+    assert lib.rn_abi_version() == 3
     assert lib.rn_status_string(0) == b"ok"
     for st in range(1, 9):
         assert lib.rn_status_string(st) not in (b"ok", b"unknown status")
@@ -309,3 +309,42 @@ def test_rope_validation(lib):
     z = dict(rows=0, dim=64)
     assert rope_call(lib, V(**z), V(data=FAKE + MB, **z), V(data=FAKE + 2 * MB, **z),
                      V(data=FAKE + 3 * MB, **z), R()) == 0
+
+
+# ---------------------------------------------------------------------------
+# head rows in blocks (e.g. a slice of a packed QKV buffer)
+
+
+@pytest.mark.parametrize("shape,strides,want", [
+    ((2, 3, 8), (40, 8, 1), (6, 8, 8, 3, 40)),
+    ((5, 32, 128), (48 * 128, 128, 1), (160, 128, 128, 32, 48 * 128)),   # q of a QKV
+    ((2, 4, 3, 16), (400, 100, 16, 1), (24, 16, 16, 3, 100)),            # blocks fold
+    ((4, 128, 1024), (128 * 1024, 1024, 1), (512, 1024, 1024, 0, 0)),  # one stride
+])
+def test_view_layout_blocks(shape, strides, want):
+    assert rn.view_layout(shape, strides) == want
+
+
+@pytest.mark.parametrize("shape,strides", [
+    ((2, 3, 8), (20, 8, 1)),         # blocks overlap (20 < 2 * 8 + 8)
+    ((2, 3, 8), (40, 4, 1)),         # rows overlap
+    ((2, 2, 3, 8), (50, 100, 8, 1)),  # block axes do not fold
+])
+def test_view_layout_rejects(shape, strides):
+    with pytest.raises(ValueError):
+        rn.view_layout(shape, strides)
+
+
+def test_block_views_are_validated(lib):
+    def B(data=FAKE, rows=12, dim=64, stride=64, inner=4, outer=512, dtype=1):
+        return rn_view(data, rows, dim, stride, dtype, inner, outer)
+    y = V(data=FAKE + MB, rows=12, dim=64)
+    assert rms(lib, B(outer=200), y) == 2          # blocks overlap
+    assert rms(lib, B(inner=-1), y) == 2
+    assert rms(lib, B(stride=32), y) == 2          # rows overlap inside a block
+    # overlap is judged on each view's whole span (first to last row), so an
+    # output anywhere inside the input's span, even between its blocks, is
+    # refused unless it is the same view
+    assert rms(lib, B(), B(data=FAKE + 512 * 2 + 2 * 64 * 2)) == 6
+    assert rms(lib, B(), V(data=FAKE + 4 * 64 * 2, dim=64, rows=12)) == 6
+    assert rms(lib, B(rows=0), B(rows=0)) == 0

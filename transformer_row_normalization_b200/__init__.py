@@ -3,25 +3,32 @@
 Thin Python binding over the C ABI of ``librownorm.so`` (declared in
 ``include/rownorm.h``). This module only marshals arguments: it turns torch
 CUDA tensors into ``rn_view`` descriptors (data pointer, rows, dim, row
-stride, dtype), passes the current CUDA stream, and raises on a nonzero
-status. Every step of the computation runs in the library's CUDA kernels;
+stride, dtype, and for head rows sliced out of a packed buffer the block
+layout), passes the current CUDA stream, and raises on a nonzero status. Every step of the computation runs in the library's CUDA kernels;
 there is no CPU or framework fallback, and calling with CPU tensors or
 without the built library raises.
 
     rn_rms_norm(x, weight, eps, out=None)               RMSNorm
     rn_layer_norm(x, weight, bias, eps, out=None)       LayerNorm
     rn_dual_head_rms_norm(q, k, wq, wk, eps, ...)       q/k head RMSNorm, one launch
+    rn_dual_head_rms_norm_rope(q, k, wq, wk, eps, table, offset, dims, ...)
+                                                        ... followed by RoPE
+    rn_add_rms_norm(x, residual, weight, eps, ...)      residual add + RMSNorm
+    rn_gated_rms_norm(x, z, weight, eps, ...)           RMSNorm * silu(gate)
+    rope_table(dims, n_pos, base, scale, inv_freq)      RoPE cos/sin table
 
-``rms_norm``, ``layer_norm`` and ``dual_head_rms_norm`` are the same calls.
+The names without the ``rn_`` prefix are the same calls.
 """
 import ctypes
 import os
 
 __all__ = [
     "RowNormError", "rn_rms_norm", "rn_layer_norm", "rn_dual_head_rms_norm",
-    "rms_norm", "layer_norm", "dual_head_rms_norm", "plan", "set_grid_override",
+    "rn_dual_head_rms_norm_rope", "rn_add_rms_norm", "rn_gated_rms_norm", "rope_table",
+    "rms_norm", "layer_norm", "dual_head_rms_norm", "dual_head_rms_norm_rope",
+    "add_rms_norm", "gated_rms_norm", "plan", "set_grid_override",
     "set_path_override", "device_error_count",
-    "library_path", "load_library", "view_params",
+    "library_path", "load_library", "view_params", "view_layout",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -43,7 +50,8 @@ class RowNormError(RuntimeError):
 class rn_view(ctypes.Structure):
     _fields_ = [("data", ctypes.c_void_p), ("rows", ctypes.c_int64),
                 ("dim", ctypes.c_int64), ("row_stride", ctypes.c_int64),
-                ("dtype", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("inner_rows", ctypes.c_int64),
+                ("outer_stride", ctypes.c_int64)]
 
 
 class rn_rope(ctypes.Structure):
@@ -97,7 +105,8 @@ def load_library():
         lib.rn_last_error.restype = ctypes.c_char_p
         for fn in (lib.rn_rms_norm, lib.rn_layer_norm, lib.rn_dual_head_rms_norm,
                    lib.rn_add_rms_norm, lib.rn_gated_rms_norm, lib.rn_plan,
-                   lib.rn_dual_head_rms_norm_rope, lib.rn_rope_table, lib.rn_set_grid_override, lib.rn_abi_version,
+                   lib.rn_dual_head_rms_norm_rope, lib.rn_rope_table,
+                   lib.rn_set_grid_override, lib.rn_abi_version,
                    lib.rn_set_path_override, lib.rn_device_error_count):
             fn.restype = ctypes.c_int
         _lib = lib
@@ -139,6 +148,49 @@ def view_params(shape, strides):
     return rows, dim, row_stride
 
 
+def _fold(axes):
+    """Stride of one axis equivalent to the (size, stride) axes, or None."""
+    if not axes:
+        return None
+    stride = axes[-1][1]
+    expect = stride
+    for n, st in reversed(axes):
+        if st != expect:
+            return None
+        expect = st * n
+    return stride
+
+
+def view_layout(shape, strides):
+    """(rows, dim, row_stride, inner_rows, outer_stride) of a [..., dim] layout
+    whose last axis is contiguous: one row stride when the leading axes fold
+    into one row axis (inner_rows = 0), else blocks of the last leading axis
+    (inner_rows rows row_stride apart, blocks outer_stride apart) when the
+    other leading axes fold into one block axis -- e.g. the heads of a packed
+    QKV buffer. Raises ValueError otherwise. Pure shape arithmetic."""
+    try:
+        rows, dim, row_stride = view_params(shape, strides)
+        return rows, dim, row_stride, 0, 0
+    except ValueError as single:
+        shape, strides = tuple(shape), tuple(strides)
+        if len(shape) < 3 or (shape[-1] > 1 and strides[-1] != 1):
+            raise single
+        dim = shape[-1]
+        lead = [(n, st) for n, st in zip(shape[:-1], strides[:-1]) if n != 1]
+        if len(lead) < 2:
+            raise single
+        inner, row_stride = lead[-1]
+        outer = _fold(lead[:-1])
+        if outer is None:
+            raise ValueError("leading axes do not fold into rows or blocks of rows")
+        if row_stride < dim or outer < (inner - 1) * row_stride + dim:
+            raise ValueError("rows overlap")
+        rows = 1
+        for n in shape[:-1]:
+            rows *= n
+        return rows, dim, row_stride, inner, outer
+
+
 def _dtype_code(t):
     import torch
     if t.dtype == torch.float32:
@@ -155,8 +207,9 @@ def _require_cuda(*tensors):
 
 
 def _view(t):
-    rows, dim, row_stride = view_params(t.shape, t.stride())
-    return rn_view(t.data_ptr() if t.numel() else None, rows, dim, row_stride, _dtype_code(t))
+    rows, dim, row_stride, inner, outer = view_layout(t.shape, t.stride())
+    return rn_view(t.data_ptr() if t.numel() else None, rows, dim, row_stride, _dtype_code(t),
+                   inner, outer)
 
 
 def _vector(v, dim, like):

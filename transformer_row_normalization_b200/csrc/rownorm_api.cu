@@ -31,6 +31,19 @@ int fail(int status, const char* fmt, ...) {
 
 int elem_size(int dtype) { return dtype == RN_F32 ? 4 : 2; }
 
+// Rows in blocks of inner_rows (row r at (r / inner) * outer + (r % inner) *
+// row_stride) when there is more than one block; else one row stride.
+bool two_level(const rn_view* v) { return v->inner_rows > 0 && v->rows > v->inner_rows; }
+
+// Element offset of the start of row r.
+int64_t row_start(const rn_view* v, int64_t r) {
+  if (!two_level(v)) return r * v->row_stride;
+  return (r / v->inner_rows) * v->outer_stride + (r % v->inner_rows) * v->row_stride;
+}
+
+// Start of the last row (the furthest, since blocks do not overlap).
+int64_t last_row_start(const rn_view* v) { return v->rows > 0 ? row_start(v, v->rows - 1) : 0; }
+
 // rows == 0 views are valid (they enqueue nothing); the checks below still
 // run so that malformed descriptors are reported consistently.
 int check_view(const rn_view* v, const char* name) {
@@ -39,13 +52,27 @@ int check_view(const rn_view* v, const char* name) {
     return fail(RN_ERR_DTYPE, "%s: unknown dtype %d", name, (int)v->dtype);
   if (v->rows < 0) return fail(RN_ERR_SHAPE, "%s: rows %lld < 0", name, (long long)v->rows);
   if (v->dim < 1) return fail(RN_ERR_SHAPE, "%s: dim %lld < 1", name, (long long)v->dim);
-  if (v->rows > 1 && v->row_stride < v->dim)
+  const int64_t inner = two_level(v) ? v->inner_rows : v->rows;  // rows of one stride
+  if (inner > 1 && v->row_stride < v->dim)
     return fail(RN_ERR_SHAPE, "%s: row_stride %lld < dim %lld", name,
                 (long long)v->row_stride, (long long)v->dim);
+  if (v->inner_rows < 0 || v->inner_rows > INT32_MAX)
+    return fail(RN_ERR_SHAPE, "%s: inner_rows %lld outside [0, 2^31)", name,
+                (long long)v->inner_rows);
   const int es = elem_size(v->dtype);
-  if (v->rows > 1) {
-    const int64_t limit = (INT64_MAX / es - v->dim) / (v->rows - 1);
+  if (inner > 1) {
+    const int64_t limit = (INT64_MAX / es - v->dim) / (inner - 1);
     if (v->row_stride > limit) return fail(RN_ERR_SHAPE, "%s: extent overflows", name);
+  }
+  if (two_level(v)) {
+    // blocks must not overlap: the next block starts past this block's rows
+    const int64_t block = (v->inner_rows - 1) * v->row_stride + v->dim;
+    if (v->outer_stride < block)
+      return fail(RN_ERR_SHAPE, "%s: outer_stride %lld < one block (%lld)", name,
+                  (long long)v->outer_stride, (long long)block);
+    const int64_t blocks = (v->rows - 1) / v->inner_rows;
+    if (v->outer_stride > (INT64_MAX / es - block) / blocks)
+      return fail(RN_ERR_SHAPE, "%s: extent overflows", name);
   }
   if (v->rows > 0 && !v->data) return fail(RN_ERR_NULL, "%s: data is NULL", name);
   if (reinterpret_cast<uintptr_t>(v->data) % es)
@@ -70,7 +97,7 @@ struct Span {
 Span span_of(const rn_view* v) {
   const uintptr_t lo = reinterpret_cast<uintptr_t>(v->data);
   if (v->rows == 0) return {lo, lo};
-  const int64_t n = (v->rows - 1) * v->row_stride + v->dim;
+  const int64_t n = last_row_start(v) + v->dim;
   return {lo, lo + static_cast<uintptr_t>(n) * elem_size(v->dtype)};
 }
 
@@ -81,8 +108,34 @@ Span span_of_vector(const void* p, int64_t dim, int dtype) {
 
 bool intersects(Span a, Span b) { return a.lo < b.hi && b.lo < a.hi && a.lo != a.hi && b.lo != b.hi; }
 
+// Whether two views can share an element. Beyond their spans: views laid out
+// in blocks with one common block stride (head rows of one packed buffer,
+// e.g. the q and k heads of a QKV projection) repeat with that period, so
+// their rows are disjoint when, within one period, each block's footprint
+// fits and misses the other's.
+bool views_overlap(const rn_view* a, const rn_view* b) {
+  if (!intersects(span_of(a), span_of(b))) return false;
+  if (!two_level(a) || !two_level(b) || a->outer_stride != b->outer_stride ||
+      a->dtype != b->dtype)
+    return true;
+  const int es = elem_size(a->dtype);
+  const intptr_t bytes = reinterpret_cast<intptr_t>(b->data) -
+                         reinterpret_cast<intptr_t>(a->data);
+  if (bytes % es) return true;
+  const int64_t o = a->outer_stride;
+  const int64_t la = (a->inner_rows - 1) * a->row_stride + a->dim;  // block footprints
+  const int64_t lb = (b->inner_rows - 1) * b->row_stride + b->dim;
+  int64_t beta = (int64_t)(bytes / es) % o;  // b's block start within a's period
+  if (beta < 0) beta += o;
+  return !(la <= o && lb <= o && beta >= la && beta + lb <= o);
+}
+
 bool same_view(const rn_view* a, const rn_view* b) {
-  return a->data == b->data && (a->rows <= 1 || a->row_stride == b->row_stride);
+  if (a->data != b->data || two_level(a) != two_level(b)) return false;
+  if (a->rows <= 1) return true;
+  if (!two_level(a)) return a->row_stride == b->row_stride;
+  return a->row_stride == b->row_stride && a->inner_rows == b->inner_rows &&
+         a->outer_stride == b->outer_stride;
 }
 
 // An output may be its own input exactly, and must not touch anything else.
@@ -90,10 +143,10 @@ int check_output(const rn_view* y, const rn_view* x_own, const rn_view* const* o
                  int n_others, const void* const* vecs, const int64_t* vec_dims,
                  int n_vecs, const char* name) {
   const Span sy = span_of(y);
-  if (intersects(sy, span_of(x_own)) && !same_view(y, x_own))
+  if (views_overlap(y, x_own) && !same_view(y, x_own))
     return fail(RN_ERR_OVERLAP, "%s partially overlaps its input", name);
   for (int i = 0; i < n_others; ++i)
-    if (intersects(sy, span_of(others[i])))
+    if (views_overlap(y, others[i]))
       return fail(RN_ERR_OVERLAP, "%s overlaps another argument", name);
   for (int i = 0; i < n_vecs; ++i)
     if (vecs[i] && intersects(sy, span_of_vector(vecs[i], vec_dims[i], y->dtype)))
@@ -118,6 +171,29 @@ int check_pair(const rn_view* x, const rn_view* y, const char* xn, const char* y
 
 // ---------------------------------------------------------------------------
 // planning
+
+// Every row of v starts at the same 16-byte phase as v's first row.
+bool strides_aligned(const rn_view* v) {
+  const int es = elem_size(v->dtype);
+  const int64_t inner = two_level(v) ? v->inner_rows : v->rows;
+  if (inner > 1 && (v->row_stride * es) % 16) return false;
+  if (two_level(v) && (v->outer_stride * es) % 16) return false;
+  return true;
+}
+
+// Every row of `v` starts at the same 16-byte phase as the matching row of x.
+bool same_phase(const rn_view* x, const rn_view* v) {
+  const int es = elem_size(x->dtype);
+  const uintptr_t xa = reinterpret_cast<uintptr_t>(x->data);
+  const uintptr_t va = reinterpret_cast<uintptr_t>(v->data);
+  if ((va - xa) % 16) return false;
+  if (strides_aligned(x) && strides_aligned(v)) return true;
+  if (two_level(x) != two_level(v)) return false;
+  if (!two_level(x)) return x->rows <= 1 || ((v->row_stride - x->row_stride) * es) % 16 == 0;
+  return x->inner_rows == v->inner_rows &&
+         ((v->row_stride - x->row_stride) * es) % 16 == 0 &&
+         ((v->outer_stride - x->outer_stride) * es) % 16 == 0;
+}
 
 constexpr int kWarpFamilyMaxDim = 1024;
 
@@ -151,8 +227,7 @@ SegPlan plan_segment(const rn_view* x, const rn_view* y, const void* w, const vo
   const int V = 16 / es;
   const int64_t D = x->dim;
   const uintptr_t xa = reinterpret_cast<uintptr_t>(x->data);
-  const bool rows_aligned = (xa % 16 == 0) && (D % V == 0) &&
-                            (x->rows <= 1 || (x->row_stride * es) % 16 == 0);
+  const bool rows_aligned = (xa % 16 == 0) && (D % V == 0) && strides_aligned(x);
   const int64_t nfull = D / V;  // full chunks of a row, at most (any phase)
   SegPlan p{};
   const int per_thread = rn::kTargetChunksPerThread;
@@ -175,17 +250,16 @@ SegPlan plan_segment(const rn_view* x, const rn_view* y, const void* w, const vo
     if (p.chunks < rn::kCtaMinChunks) p.chunks = rn::kCtaMinChunks;
   }
   const uintptr_t ya = reinterpret_cast<uintptr_t>(y->data);
-  p.vector_y = ((ya - xa) % 16 == 0) &&
-               (x->rows <= 1 || (((y->row_stride - x->row_stride) * es) % 16 == 0));
+  p.vector_y = same_phase(x, y);
   p.phase_period = 1;
-  if (x->rows > 1) {
+  if (x->rows > 1 && !two_level(x)) {
     int64_t step = (x->row_stride * es) % 16;  // row-to-row phase advance, bytes
     int period = 1;
     for (int64_t acc = step; acc % 16 != 0; acc += step) ++period;
     p.phase_period = period;
   }
   p.exact = rows_aligned && ya % 16 == 0 &&
-            (y->rows <= 1 || (y->row_stride * es) % 16 == 0) &&
+            strides_aligned(y) &&
             reinterpret_cast<uintptr_t>(w) % 16 == 0 && reinterpret_cast<uintptr_t>(b) % 16 == 0;
   p.nfull_max = nfull;
   p.nfull_min = rows_aligned ? nfull : (nfull > 0 ? nfull - 1 : 0);
@@ -323,6 +397,7 @@ bool plan_staged(int dtype, int op, const SegPlan* plans, const rn_view* const* 
   const int es = elem_size(dtype);
   const bool wide = plans[0].family == 1;
   for (int i = 0; i < nseg; ++i) {
+    if (two_level(xs[i])) return false;  // tiles address rows with one stride
     if (plans[i].family != plans[0].family) return false;
     if (!wide && !plans[i].exact) return false;
   }
@@ -502,6 +577,10 @@ rn::Segment make_segment(const rn_view* x, const rn_view* y, const void* w, cons
   s.rows = x->rows;
   s.x_stride = x->rows > 1 ? x->row_stride : x->dim;
   s.y_stride = y->rows > 1 ? y->row_stride : y->dim;
+  s.x_inner = two_level(x) ? (int)x->inner_rows : 0;
+  s.x_outer = x->outer_stride;
+  s.y_inner = two_level(y) ? (int)y->inner_rows : 0;
+  s.y_outer = y->outer_stride;
   s.dim = (int)x->dim;
   s.lanes = p.lanes;
   s.vector_y = p.vector_y;
@@ -621,15 +700,6 @@ int run_dual(const rn_view* q, const rn_view* k, const void* wq, const void* wk,
   return launch(l, params, stream);
 }
 
-// Every row of `v` starts at the same 16-byte phase as the matching row of x.
-bool same_phase(const rn_view* x, const rn_view* v) {
-  const int es = elem_size(x->dtype);
-  const uintptr_t xa = reinterpret_cast<uintptr_t>(x->data);
-  const uintptr_t va = reinterpret_cast<uintptr_t>(v->data);
-  return ((va - xa) % 16 == 0) &&
-         (x->rows <= 1 || (((v->row_stride - x->row_stride) * es) % 16 == 0));
-}
-
 // Residual add + RMSNorm (op kOpAddRms: x2 = residual, h = stored sum) and
 // gated RMSNorm (kOpGatedRms: x2 = gate, h unused).
 int run_second(int op, const rn_view* x, const rn_view* x2, const void* w, float eps,
@@ -658,9 +728,9 @@ int run_second(int op, const rn_view* x, const rn_view* x2, const void* w, float
   if (add) {
     // h may be x or the residual exactly (an in-place residual stream)
     const Span sh = span_of(h);
-    if (intersects(sh, span_of(x)) && !same_view(h, x))
+    if (views_overlap(h, x) && !same_view(h, x))
       return fail(RN_ERR_OVERLAP, "h partially overlaps x");
-    if (intersects(sh, span_of(x2)) && !same_view(h, x2))
+    if (views_overlap(h, x2) && !same_view(h, x2))
       return fail(RN_ERR_OVERLAP, "h partially overlaps the residual");
     if (w && intersects(sh, span_of_vector(w, x->dim, x->dtype)))
       return fail(RN_ERR_OVERLAP, "h overlaps the weight");
@@ -680,9 +750,13 @@ int run_second(int op, const rn_view* x, const rn_view* x2, const void* w, float
   params.seg[0] = make_segment(x, y, w, nullptr, p);
   params.seg[0].x2 = x2->data;
   params.seg[0].x2_stride = x2->rows > 1 ? x2->row_stride : x2->dim;
+  params.seg[0].x2_inner = two_level(x2) ? (int)x2->inner_rows : 0;
+  params.seg[0].x2_outer = x2->outer_stride;
   if (add) {
     params.seg[0].h = h->data;
     params.seg[0].h_stride = h->rows > 1 ? h->row_stride : h->dim;
+    params.seg[0].h_inner = two_level(h) ? (int)h->inner_rows : 0;
+    params.seg[0].h_outer = h->outer_stride;
   }
   params.nseg = 1;
   params.eps = eps;

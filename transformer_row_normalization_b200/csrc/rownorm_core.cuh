@@ -123,8 +123,28 @@ struct Segment {
   int rope_heads;
   int rope_dims;
   int rope_trad;   // 1: planes (2i, 2i + 1); 0: planes (i, i + rope_dims / 2)
-  int rope_pad_;
+  // rows in blocks (head rows of a packed buffer): for a tensor with inner
+  // count n > 0, row r starts at (r / n) * outer + (r % n) * stride; n = 0:
+  // at r * stride
+  int x_inner;
+  int y_inner;
+  int x2_inner;
+  int h_inner;
+  int blocks_pad_;
+  long long x_outer;
+  long long y_outer;
+  long long x2_outer;
+  long long h_outer;
 };
+
+// Element offset of row r of a tensor with row stride `stride` and block
+// layout (inner, outer) as in Segment (32-bit division while r fits).
+__device__ __forceinline__ long long row_off(long long r, long long stride, int inner,
+                                             long long outer) {
+  if (inner <= 0) return r * stride;
+  const long long t = r < 0x7fffffffLL ? (long long)((unsigned)r / (unsigned)inner) : r / inner;
+  return t * outer + (r - t * inner) * stride;
+}
 
 // ---------------------------------------------------------------------------
 // packed binary32 pairs
@@ -308,8 +328,8 @@ template <typename T, bool EXACT>
 __device__ __forceinline__ Row<T> row_geometry(const Segment& s, long long r) {
   constexpr int V = Elem<T>::V;
   Row<T> g;
-  g.x_row = static_cast<const T*>(s.x) + r * s.x_stride;
-  g.y_row = static_cast<T*>(s.y) + r * s.y_stride;
+  g.x_row = static_cast<const T*>(s.x) + row_off(r, s.x_stride, s.x_inner, s.x_outer);
+  g.y_row = static_cast<T*>(s.y) + row_off(r, s.y_stride, s.y_inner, s.y_outer);
   if constexpr (EXACT) {
     g.phase = 0;
     g.head = 0;

@@ -129,7 +129,7 @@ __host__ __device__ constexpr int prefetch_smem_words(int threads) {
 
 template <typename T>
 __device__ __forceinline__ const T* x2_row_of(const Segment& s, long long r) {
-  return static_cast<const T*>(s.x2) + r * s.x2_stride;
+  return static_cast<const T*>(s.x2) + row_off(r, s.x2_stride, s.x2_inner, s.x2_outer);
 }
 
 // The edge element of thread k0 in a row of a second row space that shares
@@ -218,7 +218,7 @@ __device__ __forceinline__ void segment_rows(const Segment& s, const Prefetch<T,
     if constexpr (OP == kOpAddRms) {
       // h = x + r rounded to T: stored, and what the row statistics see
       const T* full2 = x2_row_of<T>(s, r) + g.head;
-      T* hrow = static_cast<T*>(s.h) + r * s.h_stride;
+      T* hrow = static_cast<T*>(s.h) + row_off(r, s.h_stride, s.h_inner, s.h_outer);
 #pragma unroll
       for (int p = 0; p < NSLOT; ++p) {
         const int f = k0 + step * p;
