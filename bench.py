@@ -315,8 +315,9 @@ def cpu_baseline(step, chunk_rows=2048):
 
 
 def time_fused(device, rank, dist, peak, reps=30, oracle_rows=2048):
-    """The fused extensions (residual-add RMSNorm, gated RMSNorm, dual head
-    RMSNorm + RoPE), measured beside the step: the median CUDA-event time of single launches on the
+    """The extensions (residual-add RMSNorm, gated RMSNorm, dual head RMSNorm +
+    RoPE, rows streamed past the register kernels' width), measured beside the
+    step: the median CUDA-event time of single launches on the
     launching stream, each after a 256 MB read that evicts L2 (max over
     ranks), and on rank 0 the fp64 oracle's rows/s on the first
     `oracle_rows` rows on all host cores."""
@@ -329,7 +330,15 @@ def time_fused(device, rank, dist, peak, reps=30, oracle_rows=2048):
         rw = wl.Workload(w.name, w.op, w.dtype, w.shape, w.eps, rank_seed(w.seed, rank),
                          k_shape=w.k_shape, meta=w.meta)
         a = wl.make_inputs(rw, device=device)
-        if w.op == "dual_rope":
+        if w.op in ("rms", "ln"):
+            y = torch.empty_like(a["x"])
+
+            def launch():
+                if w.op == "ln":
+                    rn.layer_norm(a["x"], a["w"], a["b"], w.eps, out=y)
+                else:
+                    rn.rms_norm(a["x"], a["w"], w.eps, out=y)
+        elif w.op == "dual_rope":
             table = rn.rope_table(w.meta["rope_dims"], w.shape[0], base=w.meta["rope_base"],
                                   device=device)
             yq, yk = torch.empty_like(a["q"]), torch.empty_like(a["k"])
@@ -368,7 +377,14 @@ def time_fused(device, rank, dist, peak, reps=30, oracle_rows=2048):
                 "frac": round(g / peak, 4), "algorithmic_bytes": w.algorithmic_bytes()}
         if rank == 0:
             import oracle
-            if w.op == "dual_rope":
+            if w.op in ("rms", "ln"):
+                nr = max(1, oracle_rows // 256)  # 65536-wide rows: a few MB of oracle work
+                xs = a["x"].reshape(-1, w.dim)[:nr].cpu()
+                args = ((xs, a["w"].cpu(), a["b"].cpu(), w.eps) if w.op == "ln"
+                        else (xs, a["w"].cpu(), w.eps))
+                fn = oracle.layer_norm if w.op == "ln" else oracle.rms_norm
+                nrows = nr
+            elif w.op == "dual_rope":
                 # whole tokens: oracle_rows // 40 tokens of 32 query + 8 key heads
                 nt = max(1, oracle_rows // 40)
                 args = (a["q"].reshape(-1, w.dim)[:nt * 32].cpu(),

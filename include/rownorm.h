@@ -70,8 +70,13 @@ extern "C" {
 /* Largest supported dim. Rows are held on chip (registers) between reading
  * and writing, so x is read from HBM exactly once; wider rows are rejected
  * with RN_ERR_UNSUPPORTED. */
+/* Widest rows the register kernels hold (every op). rn_rms_norm and
+ * rn_layer_norm take wider rows, up to RN_MAX_DIM_STREAM, through streaming
+ * kernels that read each row once per pass (two passes for RMSNorm, three for
+ * LayerNorm; the later ones from L2 while the rows in flight fit there). */
 #define RN_MAX_DIM_BF16 32768
 #define RN_MAX_DIM_F32 16384
+#define RN_MAX_DIM_STREAM 4194304
 /* rn_dual_head_rms_norm: both head dims at most this (one launch keeps the
  * query and key rows in one warp-level kernel). */
 #define RN_MAX_HEAD_DIM 1024
@@ -87,8 +92,9 @@ typedef enum rn_status {
     RN_ERR_EPS = 4,         /* eps is negative, NaN or infinite               */
     RN_ERR_ALIGN = 5,       /* a pointer not aligned to its element size      */
     RN_ERR_OVERLAP = 6,     /* an output partially overlaps an input/output  */
-    RN_ERR_UNSUPPORTED = 7, /* dim beyond RN_MAX_DIM_*, or a dual head dim    */
-                            /* beyond RN_MAX_HEAD_DIM                         */
+    RN_ERR_UNSUPPORTED = 7, /* dim beyond RN_MAX_DIM_STREAM (RMSNorm,         */
+                            /* LayerNorm) or RN_MAX_DIM_BF16/F32 (fused ops), */
+                            /* or a dual head dim beyond RN_MAX_HEAD_DIM      */
     RN_ERR_CUDA = 8         /* the CUDA runtime reported an error (device    */
                             /* query or launch); see rn_last_error()          */
 } rn_status;

@@ -124,10 +124,18 @@ def test_rejects_overlap_but_allows_in_place(lib):
 
 
 def test_rejects_unsupported_widths(lib):
-    y = V(data=FAKE + (1 << 30), dim=32769)
-    assert rms(lib, V(dim=32769), y) == 7
-    y = V(data=FAKE + (1 << 30), dim=16385, dtype=0)
-    assert rms(lib, V(dim=16385, dtype=0), y) == 7
+    # RMSNorm / LayerNorm stream rows up to RN_MAX_DIM_STREAM (4M) columns
+    big = (1 << 22) + 1
+    y = V(data=FAKE + (1 << 40), rows=2, dim=big, stride=big)
+    assert rms(lib, V(rows=2, dim=big, stride=big), y) == 7
+    assert ln(lib, V(rows=2, dim=big, stride=big), y) == 7
+    # the fused ops hold rows in registers: 32768 bf16 / 16384 f32 at most
+    x, r = V(rows=2, dim=32769, stride=32769), V(data=FAKE + (1 << 30), rows=2, dim=32769,
+                                                 stride=32769)
+    y, h = V(data=FAKE + (2 << 30), rows=2, dim=32769, stride=32769), \
+        V(data=FAKE + (3 << 30), rows=2, dim=32769, stride=32769)
+    assert add_rms(lib, x, r, y, h) == 7
+    assert b"fused ops" in lib.rn_last_error()
 
 
 def test_rows_zero_is_a_no_op(lib):

@@ -232,6 +232,9 @@ def test_errors_surface_as_exceptions():
         rn.rms_norm(x, None, -1.0)
     with pytest.raises(rn.RowNormError, match="RN_ERR_OVERLAP"):
         rn.rms_norm(x[:, :4], None, 1e-6, out=x[:, 2:6])
+    big = torch.zeros(1, 32769, device="cuda", dtype=torch.bfloat16)
     with pytest.raises(rn.RowNormError, match="RN_ERR_UNSUPPORTED"):
-        big = torch.zeros(1, 32769, device="cuda", dtype=torch.bfloat16)
-        rn.rms_norm(big, None, 1e-6)
+        rn.add_rms_norm(big, big.clone(), None, 1e-6)  # fused ops: registers only
+    with pytest.raises(rn.RowNormError, match="RN_ERR_UNSUPPORTED"):
+        huge = torch.zeros(1, (1 << 22) + 1, device="cuda", dtype=torch.bfloat16)
+        rn.rms_norm(huge, None, 1e-6)  # beyond the streaming limit

@@ -20,8 +20,9 @@ LIB = os.path.join(PKG, "librownorm.so")
 
 SOURCES = ["rownorm_api.cu", "rownorm_warp_f32.cu", "rownorm_warp_bf16.cu",
            "rownorm_cta_f32.cu", "rownorm_cta_bf16.cu", "rownorm_staged_f32.cu",
-           "rownorm_staged_bf16.cu"]
-HEADERS = ["rownorm_core.cuh", "rownorm_kernels.cuh", "rownorm_staged.cuh", "rownorm_launch.h"]
+           "rownorm_staged_bf16.cu", "rownorm_stream.cu"]
+HEADERS = ["rownorm_core.cuh", "rownorm_kernels.cuh", "rownorm_staged.cuh", "rownorm_launch.h",
+           "rownorm_stream.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",

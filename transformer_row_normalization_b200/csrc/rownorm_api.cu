@@ -77,10 +77,9 @@ int check_view(const rn_view* v, const char* name) {
   if (v->rows > 0 && !v->data) return fail(RN_ERR_NULL, "%s: data is NULL", name);
   if (reinterpret_cast<uintptr_t>(v->data) % es)
     return fail(RN_ERR_ALIGN, "%s: data not aligned to its %d-byte element", name, es);
-  const int64_t max_dim = v->dtype == RN_F32 ? RN_MAX_DIM_F32 : RN_MAX_DIM_BF16;
-  if (v->dim > max_dim)
+  if (v->dim > RN_MAX_DIM_STREAM)
     return fail(RN_ERR_UNSUPPORTED, "%s: dim %lld above the supported maximum %lld", name,
-                (long long)v->dim, (long long)max_dim);
+                (long long)v->dim, (long long)RN_MAX_DIM_STREAM);
   return RN_OK;
 }
 
@@ -205,8 +204,11 @@ int pow2_ceil(int64_t v) {
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Widest rows the register kernels hold; wider RMSNorm / LayerNorm rows stream.
+int64_t register_max_dim(int dtype) { return dtype == RN_F32 ? RN_MAX_DIM_F32 : RN_MAX_DIM_BF16; }
+
 struct SegPlan {
-  int family;        // 0 warp, 1 block
+  int family;        // 0 warp, 1 block, 2 streaming block (rows wider than registers hold)
   int lanes;         // family 0: lanes per row; family 1: threads per block
   int chunks;        // capacity of 16-byte chunks per thread
   int vector_y;      // y rows share x's 16-byte phase
@@ -231,7 +233,11 @@ SegPlan plan_segment(const rn_view* x, const rn_view* y, const void* w, const vo
   const int64_t nfull = D / V;  // full chunks of a row, at most (any phase)
   SegPlan p{};
   const int per_thread = rn::kTargetChunksPerThread;
-  if (D <= kWarpFamilyMaxDim) {
+  if (D > register_max_dim(x->dtype)) {
+    p.family = 2;
+    p.lanes = rn::kStreamBlockThreads;
+    p.chunks = (int)ceil_div(nfull, p.lanes);
+  } else if (D <= kWarpFamilyMaxDim) {
     p.family = 0;
     int g = pow2_ceil(ceil_div(ceil_div(D, V), per_thread));
     if (!rows_aligned && g < pow2_ceil(2 * (V - 1))) g = pow2_ceil(2 * (V - 1));
@@ -281,6 +287,7 @@ int slot_class(const SegPlan& p, int chunks) {
 
 const void* kernel_for(int dtype, int op, const SegPlan& p, int slots) {
   const bool ex = p.exact != 0;
+  if (p.family == 2) return rn::stream_kernel(dtype == RN_F32, op, ex);
   if (p.family == 0)
     return dtype == RN_F32 ? rn::warp_kernel_f32(op, ex, slots, p.chunks)
                            : rn::warp_kernel_bf16(op, ex, slots, p.chunks);
@@ -396,6 +403,7 @@ bool plan_staged(int dtype, int op, const SegPlan* plans, const rn_view* const* 
   if (g_path_override != 2 || rn::op_has_second(op)) return false;
   const int es = elem_size(dtype);
   const bool wide = plans[0].family == 1;
+  if (plans[0].family == 2) return false;  // rows wider than the register kernels hold
   for (int i = 0; i < nseg; ++i) {
     if (two_level(xs[i])) return false;  // tiles address rows with one stride
     if (plans[i].family != plans[0].family) return false;
@@ -502,7 +510,11 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
   if (st) return st;
   if (plan_staged(dtype, op, plans, xs, ws, bs, nseg, dev, sms, out)) return RN_OK;
   const int threads = merged.family == 0 ? rn::kWarpBlock : merged.lanes;
-  const int cache = merged.exact ? 0 : rn::affine_cache_smem_bytes(op, threads, merged.chunks);
+  // the streaming kernels keep no weight cache and prefetch nothing
+  const bool stream = merged.family == 2;
+  const int cache = (merged.exact || stream)
+                        ? 0
+                        : rn::affine_cache_smem_bytes(op, threads, merged.chunks);
   const int pf_bytes = rn::prefetch_slots_smem_bytes(
                            threads, merged.chunks,
                            merged.family == 0 ? rn::kWarpPrefetchStages : rn::kCtaPrefetchStages) *
@@ -516,7 +528,9 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
       g_path_override == 3 ||
       (g_path_override == 0 && (merged.family == 0 || merged.lanes >= 256));
   const int prefetch =
-      want_prefetch && cache + pf_bytes <= device_info(dev).smem_per_block - 1024 ? 1 : 0;
+      !stream && want_prefetch && cache + pf_bytes <= device_info(dev).smem_per_block - 1024
+          ? 1
+          : 0;
   int smem = cache + (prefetch ? pf_bytes : 0);
   out->stage_word = smem / 16;
   if (op == rn::kOpRmsRope) {
@@ -716,6 +730,10 @@ int run_second(int op, const rn_view* x, const rn_view* x2, const void* w, float
   if (add && (st = check_pair(x, h, "x", "h"))) return st;
   if ((st = check_eps(eps))) return st;
   if ((st = check_vector(w, x->dtype, "weight"))) return st;
+  if (x->dim > register_max_dim(x->dtype))
+    return fail(RN_ERR_UNSUPPORTED, "%s: dim %lld above %lld (fused ops hold rows in registers)",
+                add ? "add_rms_norm" : "gated_rms_norm", (long long)x->dim,
+                (long long)register_max_dim(x->dtype));
   if (!same_phase(x, x2))
     return fail(RN_ERR_ALIGN, "%s rows must share x's 16-byte alignment", x2n);
   if (add && !same_phase(x, h))

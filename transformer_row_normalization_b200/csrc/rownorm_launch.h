@@ -49,6 +49,11 @@ const void* cta_kernel_f32(int op, bool exact, int slots, int threads, int chunk
 const void* cta_kernel_bf16(int op, bool exact, int slots, int threads, int chunks);
 // Bulk-copy staged kernels: wide (one block per row) or narrow (lane groups,
 // rows 16-byte aligned); nullptr if not compiled.
+// Streaming kernels (rows wider than the register kernels hold): RMSNorm
+// and LayerNorm, any layout.
+const void* stream_kernel(int dtype_f32, int op, bool exact);
+constexpr int kStreamBlockThreads = 1024;
+
 const void* staged_kernel_f32(int op, bool wide, bool exact, int threads, int chunks);
 const void* staged_kernel_bf16(int op, bool wide, bool exact, int threads, int chunks);
 // Timed-out stage waits recorded by the staged kernels of each element type

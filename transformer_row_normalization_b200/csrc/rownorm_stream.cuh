@@ -1,0 +1,214 @@
+// Streaming row normalization for rows too wide to hold in registers
+// (sm_100a).
+//
+// One block of kStreamThreads threads per row, rows strided statically over
+// a persistent grid. The row is read once per pass: RMSNorm makes two
+// passes (sum of squares, then normalize and store), LayerNorm three (sum
+// of d = x - K with K = x_0, then sum of (d - mean)^2, then normalize and
+// store): the same shifted two-pass statistics as the register kernels, so
+// a constant row still gives exactly the bias. Passes after the first find
+// the row in L2 while the rows in flight (one per SM) fit there.
+//
+// Ownership and summation order (fixed; they depend only on D, the element
+// type and the row's 16-byte phase): thread t owns the full chunks t,
+// t + kStreamThreads, ... and edge element t (rownorm_core.cuh's row split);
+// each pass sums the thread's chunks into even / odd binary32 pair
+// partials in chunk order, adds the edge element's term, and combines the
+// threads with block_sum. The arithmetic of each element is that of the
+// register kernels.
+#pragma once
+
+#include "rownorm_core.cuh"
+#include "rownorm_kernels.cuh"
+
+namespace rn {
+
+constexpr int kStreamThreads = 1024;
+// chunks a thread loads before it uses the first of them (loads in flight)
+constexpr int kStreamUnroll = 4;
+
+// Cached 16-byte load (the row is read again by the next pass).
+__device__ __forceinline__ uint4 load_keep(const void* p) {
+  return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+// Weight (and bias) of chunk f's columns for any layout: one aligned 16-byte
+// load per vector when the vector's columns are aligned with the row's
+// chunks, else element by element.
+template <typename T, bool BIAS>
+__device__ __forceinline__ void stream_affine(const Segment& s, const Row<T>& g, int f,
+                                              bool aligned, F2 (&wf)[Elem<T>::P],
+                                              F2 (&bf)[Elem<T>::P]) {
+  constexpr int V = Elem<T>::V;
+  constexpr int P = Elem<T>::P;
+  const T* w = static_cast<const T*>(s.w);
+  const T* b = static_cast<const T*>(s.b);
+  const int c0 = g.head + f * V;
+  if (aligned) {
+    if (w) {
+      Elem<T>::unpack(load_cached(w + c0), wf);
+    } else {
+#pragma unroll
+      for (int j = 0; j < P; ++j) wf[j] = splat(1.f);
+    }
+    if constexpr (BIAS) {
+      if (b) {
+        Elem<T>::unpack(load_cached(b + c0), bf);
+      } else {
+#pragma unroll
+        for (int j = 0; j < P; ++j) bf[j] = zero2();
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < P; ++j) {
+      wf[j] = w ? make2(Elem<T>::get(w + c0 + 2 * j), Elem<T>::get(w + c0 + 2 * j + 1))
+                : splat(1.f);
+      if constexpr (BIAS)
+        bf[j] = b ? make2(Elem<T>::get(b + c0 + 2 * j), Elem<T>::get(b + c0 + 2 * j + 1))
+                  : zero2();
+    }
+  }
+}
+
+// One pass over the thread's chunks of row g: `chunk(v)` folds each chunk's
+// pairs into the accumulator (chunk order), kStreamUnroll loads in flight.
+template <typename T, typename Fold>
+__device__ __forceinline__ void stream_pass(const Row<T>& g, int tid, Fold fold) {
+  constexpr int V = Elem<T>::V;
+  constexpr int P = Elem<T>::P;
+  int f = tid;
+#pragma unroll 1
+  constexpr int kStep = kStreamUnroll * kStreamThreads;
+  for (; f + (kStreamUnroll - 1) * kStreamThreads < g.nfull; f += kStep) {
+    uint4 u[kStreamUnroll];
+#pragma unroll
+    for (int q = 0; q < kStreamUnroll; ++q)
+      u[q] = load_keep(g.x_full + (long long)(f + q * kStreamThreads) * V);
+#pragma unroll
+    for (int q = 0; q < kStreamUnroll; ++q) {
+      F2 v[P];
+      Elem<T>::unpack(u[q], v);
+      fold(v);
+    }
+  }
+#pragma unroll 1
+  for (; f < g.nfull; f += kStreamThreads) {
+    F2 v[P];
+    Elem<T>::unpack(load_keep(g.x_full + (long long)f * V), v);
+    fold(v);
+  }
+}
+
+template <typename T, int OP, bool EXACT>
+__global__ void __launch_bounds__(kStreamThreads, 1) rows_stream_kernel(const Params p) {
+  static_assert(OP == kOpRms || OP == kOpLn, "streaming covers RMSNorm and LayerNorm");
+  constexpr int V = Elem<T>::V;
+  constexpr int P = Elem<T>::P;
+  constexpr bool BIAS = OP == kOpLn;
+  __shared__ float red[2][kStreamThreads / 32];
+  int slot = 0;
+  auto reduce = [&](float t) {
+    const float r = block_sum<kStreamThreads>(t, red[slot]);
+    slot ^= 1;
+    return r;
+  };
+  const Segment& s = p.seg[0];
+  const int tid = threadIdx.x;
+  const int D = s.dim;
+  const float inv_d = __frcp_rn((float)D);
+#pragma unroll 1
+  for (long long r = blockIdx.x; r < s.rows; r += gridDim.x) {
+    const Row<T> g = row_geometry<T, EXACT>(s, r);
+    const bool has_edge = !EXACT && tid < g.nedge;
+    float xe = load_edge<T, EXACT>(g, D, tid);
+    float rstd, mean = 0.f;
+    if constexpr (OP == kOpRms) {
+      F2 acc = zero2();
+      stream_pass<T>(g, tid, [&](F2 (&v)[P]) {
+#pragma unroll
+        for (int j = 0; j < P; ++j) acc = fma2(v[j], v[j], acc);
+      });
+      float part = hsum2(acc);
+      if (has_edge) part = __fmaf_rn(xe, xe, part);
+      rstd = rsqrtf(__fadd_rn(__fmul_rn(reduce(part), inv_d), p.eps));
+    } else {
+      const float K = Elem<T>::get(g.x_row);
+      const F2 K2 = splat(K);
+      F2 acc = zero2();
+      stream_pass<T>(g, tid, [&](F2 (&v)[P]) {
+#pragma unroll
+        for (int j = 0; j < P; ++j) acc = add2(acc, sub2(v[j], K2));
+      });
+      float part = hsum2(acc);
+      if (has_edge) {
+        xe = __fsub_rn(xe, K);
+        part = __fadd_rn(part, xe);
+      }
+      mean = __fmul_rn(reduce(part), inv_d);
+      const F2 M2 = splat(mean);
+      acc = zero2();
+      stream_pass<T>(g, tid, [&](F2 (&v)[P]) {
+#pragma unroll
+        for (int j = 0; j < P; ++j) {
+          const F2 t = sub2(sub2(v[j], K2), M2);
+          acc = fma2(t, t, acc);
+        }
+      });
+      part = hsum2(acc);
+      if (has_edge) {
+        const float t = __fsub_rn(xe, mean);
+        part = __fmaf_rn(t, t, part);
+      }
+      rstd = rsqrtf(__fadd_rn(__fmul_rn(reduce(part), inv_d), p.eps));
+    }
+    // last pass: normalize, weight (and bias), store
+    const F2 R2 = splat(rstd);
+    const F2 M2 = splat(mean);
+    const F2 K2 = splat(OP == kOpLn ? Elem<T>::get(g.x_row) : 0.f);  // LayerNorm shift
+    // the vectors' columns of a chunk start 16-byte aligned (EXACT: always)
+    auto vec_aligned = [&](const void* v) {
+      return !v || (reinterpret_cast<uintptr_t>(static_cast<const T*>(v) + g.head) % 16) == 0;
+    };
+    const bool aligned = EXACT || (vec_aligned(s.w) && (!BIAS || vec_aligned(s.b)));
+#pragma unroll 1
+    for (int f = tid; f < g.nfull; f += kStreamThreads) {
+      F2 v[P], wf[P], bf[P], o[P];
+      Elem<T>::unpack(load_stream(g.x_full + (long long)f * V), v);
+      stream_affine<T, BIAS>(s, g, f, aligned, wf, bf);
+#pragma unroll
+      for (int j = 0; j < P; ++j) {
+        if constexpr (OP == kOpLn)
+          o[j] = fma2(mul2(sub2(sub2(v[j], K2), M2), R2), wf[j], bf[j]);
+        else
+          o[j] = mul2(mul2(v[j], R2), wf[j]);
+      }
+      T* yc = g.y_row + g.head + (long long)f * V;
+      if (EXACT || s.vector_y) {
+        store_stream(yc, Elem<T>::pack(o));
+      } else {
+#pragma unroll
+        for (int j = 0; j < P; ++j) {
+          Elem<T>::put(yc + 2 * j, o[j].x);
+          Elem<T>::put(yc + 2 * j + 1, o[j].y);
+        }
+      }
+    }
+    if (has_edge) {
+      const int c = edge_column(g, D, tid);
+      const T* w = static_cast<const T*>(s.w);
+      const T* b = static_cast<const T*>(s.b);
+      const float we = w ? Elem<T>::get(w + c) : 1.f;
+      float o;
+      if constexpr (OP == kOpLn) {
+        const float be = b ? Elem<T>::get(b + c) : 0.f;
+        o = __fmaf_rn(__fmul_rn(__fsub_rn(xe, mean), rstd), we, be);
+      } else {
+        o = __fmul_rn(__fmul_rn(xe, rstd), we);
+      }
+      Elem<T>::put(g.y_row + c, o);
+    }
+  }
+}
+
+}  // namespace rn

@@ -34,6 +34,10 @@ comment), at the shapes of the rows they fuse with:
                               ("Emily.Fast", rope/3): the prefill heads above,
                               positions 0..8191, base 10000, all 128 columns
                               rotated, split-half planes.
+  ln_bf16_8192x65536,         rows wider than the register kernels hold
+  rms_bf16_8192x65536         (streamed): the LayerNorm width sweep's recipe
+                              (N(0.5, 2), every 64th row constant) and the
+                              RMSNorm recipe (N(0,1)), 1 GB each way.
 """
 from dataclasses import dataclass, field
 from typing import Dict, Optional, Tuple
@@ -134,8 +138,10 @@ LARGE_SUITE = ("dual_bf16_prefill", "rms_bf16_16x4096x4096") + tuple(
     f"ln_bf16_65536x{d}" for d in LN_WIDTHS)
 SMALL_SUITE = ("rms_f32_4x128x1024", "ln_f32_1x1024x768", "dual_bf16_decode")
 # The fused extensions, measured beside (not inside) the benchmark step.
+_register(Workload("ln_bf16_8192x65536", "ln", torch.bfloat16, (8192, 65536), 1e-5, 65))
+_register(Workload("rms_bf16_8192x65536", "rms", torch.bfloat16, (8192, 65536), 1e-5, 66))
 FUSED_SUITE = ("add_rms_bf16_16x4096x4096", "gated_rms_bf16_8192x32x128",
-               "dual_rope_bf16_prefill")
+               "dual_rope_bf16_prefill", "ln_bf16_8192x65536", "rms_bf16_8192x65536")
 
 
 def _gen(device, seed):
@@ -175,7 +181,7 @@ def make_inputs(w: Workload, device="cpu") -> Dict[str, torch.Tensor]:
         out["w"] = _normal((w.dim,), 1.0, 0.1, g, device)
         outliers = torch.rand(w.shape, generator=g, device=device) < 0.01
         out["x"] = torch.where(outliers, x * 50.0, x)
-    elif w.name.startswith("ln_bf16_65536x"):
+    elif w.name.startswith("ln_bf16_65536x") or w.name == "ln_bf16_8192x65536":
         x = _normal(w.shape, 0.5, 2.0, g, device)
         out["w"] = _normal((w.dim,), 1.0, 0.1, g, device)
         out["b"] = _normal((w.dim,), 0.0, 0.1, g, device)
@@ -183,6 +189,9 @@ def make_inputs(w: Workload, device="cpu") -> Dict[str, torch.Tensor]:
         values = _normal((const_rows.numel(), 1), 0.5, 2.0, g, device)
         x[const_rows] = values.expand(-1, w.dim)
         out["x"] = x
+    elif w.name == "rms_bf16_8192x65536":
+        out["x"] = _normal(w.shape, 0.0, 1.0, g, device)
+        out["w"] = _normal((w.dim,), 1.0, 0.1, g, device)
     elif w.op in ("add_rms", "gated_rms") and w.dtype == torch.float32:
         second = "r" if w.op == "add_rms" else "z"
         out["x"] = _uniform(w.shape, -1.0, 1.0, g, device)
