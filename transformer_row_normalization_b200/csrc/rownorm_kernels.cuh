@@ -44,10 +44,23 @@ __device__ __forceinline__ Segment pick_segment(const Segment (&seg)[2], int i) 
 }
 
 constexpr int kWarpBlock = 256;
-// Register budgets: at least this many threads resident per SM (lane-group
-// family 768, i.e. up to 85 registers; block family 1024, 64 registers).
-constexpr int kMinThreadsPerSmWarp = 768;
+// Block-family register budget: at least 1024 threads resident per SM (64
+// registers).
 constexpr int kMinThreadsPerSm = 1024;
+
+// Lane-group register budget, as blocks of kWarpBlock threads resident per
+// SM: 3 (up to 80 registers, 24 warps) or 2 (up to 128, 16 warps). Measured
+// on B200 over bf16 and binary32 rows of 64 to 1024 columns, LayerNorm ran
+// 7-22 % faster with more warps except where its values spill at 80
+// registers (bf16 rows of 4 chunks per lane with a partial last chunk;
+// binary32 rows of 6 or more chunks per lane: 2-8 % faster with 128, 1.6x at
+// D = 1001), and every RMSNorm ran as fast or faster with 128.
+template <typename T, int OP, int SLOTS, int VPL>
+__host__ __device__ constexpr int warp_blocks_per_sm() {
+  if (OP != kOpLn) return 2;
+  if (Elem<T>::V == 8) return VPL == 4 && SLOTS != kSlotsFull ? 2 : 3;
+  return VPL >= 6 ? 2 : 3;
+}
 
 // Per-thread prefetch slots: [stages][NSLOT][blockDim.x] 16-byte words
 // from 16-byte word `base` of the dynamic shared memory (a second bank
@@ -114,10 +127,11 @@ struct Prefetch {
   }
 };
 
-// Prefetch stages (rows in flight per thread group: the one being normalized
-// and NST - 1 ahead). Measured on B200, a third stage gained nothing for lane
-// groups (LayerNorm 768, 1000, 1024; RMSNorm 512) and cost up to 8 % for
-// blocks, so both families keep one row ahead.
+// Prefetch stages per thread: rows in flight while one is normalized from
+// registers. Measured on B200 (back-to-back bf16 LayerNorm, D = 768 to
+// 16384), two rows ahead beat one by 2-4 % for blocks, while a third stage
+// cost blocks 10-14 % (its slots squeeze the L1 share that holds the weight
+// and bias) and moved lane groups by no more than noise.
 constexpr int kWarpPrefetchStages = 2;
 constexpr int kCtaPrefetchStages = 2;
 
@@ -157,9 +171,13 @@ struct GateSrc {
 
 // The rows r0, r0 + stride, ... of one segment, owned by one thread group (a
 // lane group, or a block) in which this thread is k0 of `step`. Each row's
-// chunks (and those of the second input) are prefetched NST - 1 rows ahead,
-// stage i % NST holding row i; the shift K and the thread's edge elements of
-// the rows ahead wait in register queues. `src` supplies weight and bias.
+// chunks (and those of the second input) are prefetched NST rows ahead into
+// the thread's own slots, stage i % NST holding row i. A row's stage is
+// refilled with the row NST ahead as soon as the thread has read the stage
+// into registers, so NST rows are in flight while the row is normalized (for
+// the gated op, whose gate is read from its stage while the row is stored,
+// once the row is stored). The shift K and the thread's edge elements of the
+// rows ahead wait in register queues. `src` supplies weight and bias.
 template <typename T, int OP, bool EXACT, int SLOTS, int NSLOT, int NST, typename Src,
           typename Reduce>
 __device__ __forceinline__ void segment_rows(const Segment& s, const Prefetch<T, NSLOT>& pf,
@@ -167,13 +185,14 @@ __device__ __forceinline__ void segment_rows(const Segment& s, const Prefetch<T,
                                              long long stride, int k0, int step, float eps,
                                              Reduce reduce, Src& src, float* stage,
                                              unsigned mask) {
-  static_assert(NST >= 2, "at least one row ahead");
+  static_assert(NST >= 1, "at least one row ahead");
   constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
   constexpr bool SECOND = op_has_second(OP);
+  constexpr bool LATE_REFILL = OP == kOpGatedRms;
   const int D = s.dim;
-  float Kq[NST - 1], Eq[NST - 1], E2q[NST - 1];
-  // queue the loads of row ra into stage `stage`
+  float Kq[NST], Eq[NST], E2q[NST];
+  // queue the loads of row ra into stage `stage`, its scalars at queue entry j
   auto ahead = [&](long long ra, int stage, int j) {
     const Row<T> ga = row_geometry<T, EXACT>(s, ra);
     pf.template issue<SLOTS>(ga.x_full, ga.nfull, k0, step, stage);
@@ -185,8 +204,15 @@ __device__ __forceinline__ void segment_rows(const Segment& s, const Prefetch<T,
       E2q[j] = load_edge_at<T, EXACT>(row2, ga, D, k0);
     }
   };
+  // stage `st` is free again: start row r + NST there (an empty group past
+  // the end keeps one group per row)
+  auto refill = [&](long long r, int st) {
+    const long long ra = r + NST * stride;
+    if (ra < s.rows) ahead(ra, st, NST - 1);
+    cp_async_commit();
+  };
 #pragma unroll
-  for (int j = 0; j < NST - 1; ++j) {
+  for (int j = 0; j < NST; ++j) {
     const long long rj = r0 + j * stride;
     Kq[j] = 0.f;
     Eq[j] = 0.f;
@@ -201,17 +227,12 @@ __device__ __forceinline__ void segment_rows(const Segment& s, const Prefetch<T,
     float xe = Eq[0];
     const float x2e = E2q[0];
 #pragma unroll
-    for (int j = 0; j + 1 < NST - 1; ++j) {
+    for (int j = 0; j + 1 < NST; ++j) {
       Kq[j] = Kq[j + 1];
       Eq[j] = Eq[j + 1];
       E2q[j] = E2q[j + 1];
     }
-    // the stage the previous row was taken from receives row r + (NST-1) stride
-    const int sa = st == 0 ? NST - 1 : st - 1;
-    const long long ra = r + (NST - 1) * stride;
-    if (ra < s.rows) ahead(ra, sa, NST - 2);
-    cp_async_commit();
-    cp_async_wait<NST - 1>();
+    cp_async_wait<NST - 1>();  // row r has landed
     const Row<T> g = row_geometry<T, EXACT>(s, r);
     const bool has_edge = !EXACT && k0 < g.nedge;
     F2 v[NSLOT][P];
@@ -236,12 +257,14 @@ __device__ __forceinline__ void segment_rows(const Segment& s, const Prefetch<T,
           for (int j = 0; j < P; ++j) v[p][j] = zero2();
         }
       }
+      if constexpr (!LATE_REFILL) refill(r, st);
       if (has_edge) {
         xe = Elem<T>::stored(__fadd_rn(xe, x2e));
         Elem<T>::put(hrow + edge_column(g, D, k0), xe);
       }
     } else {
       pf.template take<SLOTS>(g.x_full, g.nfull, k0, step, st, v);
+      if constexpr (!LATE_REFILL) refill(r, st);
     }
     float rstd, mean;
     row_stats<T, OP, EXACT, SLOTS, NSLOT>(v, xe, g, D, k0, step, K, eps, has_edge, reduce, rstd,
@@ -260,6 +283,7 @@ __device__ __forceinline__ void segment_rows(const Segment& s, const Prefetch<T,
       normalize_store<T, OP, EXACT, SLOTS, NSLOT>(s, g, v, xe, src, k0, step, rstd, mean,
                                                   has_edge);
     }
+    if constexpr (LATE_REFILL) refill(r, st);
     st = st == NST - 1 ? 0 : st + 1;
   }
   cp_async_wait<0>();
@@ -282,23 +306,23 @@ __device__ __forceinline__ void run_segment(const Segment& s, const Prefetch<T, 
   if constexpr (EXACT) {
     if (w && (!BIAS || b)) {
       AffineDirect<T, BIAS, true> src{w, b};
-      segment_rows<T, OP, true, SLOTS, NSLOT, NST>(s, pf, pf2, r0, stride, k0, step, eps, reduce,
-                                                   src, stage, mask);
+      segment_rows<T, OP, true, SLOTS, NSLOT, NST>(
+          s, pf, pf2, r0, stride, k0, step, eps, reduce, src, stage, mask);
     } else {
       AffineDirect<T, BIAS, false> src{w, b};
-      segment_rows<T, OP, true, SLOTS, NSLOT, NST>(s, pf, pf2, r0, stride, k0, step, eps, reduce,
-                                                   src, stage, mask);
+      segment_rows<T, OP, true, SLOTS, NSLOT, NST>(
+          s, pf, pf2, r0, stride, k0, step, eps, reduce, src, stage, mask);
     }
   } else {
     AffineCache<T, NSLOT, BIAS> src;
     src.init(cache_word);
-    segment_rows<T, OP, false, SLOTS, NSLOT, NST>(s, pf, pf2, r0, stride, k0, step, eps, reduce,
-                                                  src, stage, mask);
+    segment_rows<T, OP, false, SLOTS, NSLOT, NST>(
+        s, pf, pf2, r0, stride, k0, step, eps, reduce, src, stage, mask);
   }
 }
 
 template <typename T, int OP, bool EXACT, int SLOTS, int VPL>
-__global__ void __launch_bounds__(kWarpBlock, kMinThreadsPerSmWarp / kWarpBlock)
+__global__ void __launch_bounds__(kWarpBlock, (warp_blocks_per_sm<T, OP, SLOTS, VPL>()))
 rows_warp_kernel(const Params p) {
   constexpr int BANK = prefetch_smem_words<VPL, kWarpPrefetchStages>(kWarpBlock);
   const Prefetch<T, VPL> pf{p.prefetch, 0};
