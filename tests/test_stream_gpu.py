@@ -65,6 +65,21 @@ def test_wide_layouts(dtype):
           what="ln gapped out, null vectors")
 
 
+@pytest.mark.parametrize("op,dtype,dim,threads", [
+    ("ln", torch.bfloat16, 65536, 512), ("ln", torch.bfloat16, 98304, 512),
+    ("ln", torch.bfloat16, 98305, 1024), ("ln", torch.bfloat16, 262144, 1024),
+    ("ln", torch.float32, 49152, 512), ("ln", torch.float32, 49153, 1024),
+    ("rms", torch.bfloat16, 65536, 1024), ("rms", torch.float32, 32768, 1024)])
+def test_stream_block_size(op, dtype, dim, threads):
+    """LayerNorm rows of at most 192 KB stream two rows per SM (512 threads
+    each); wider rows and RMSNorm one row per SM (1024 threads)."""
+    x = torch.empty(2, dim, dtype=dtype, device="cuda")
+    w = torch.empty(dim, dtype=dtype, device="cuda")
+    kind = rn.RN_OP_LN if op == "ln" else rn.RN_OP_RMS
+    p = rn.plan(kind, x, weight=w, bias=w if op == "ln" else None)
+    assert p["family"] == 2 and p["threads_per_row"] == threads and p["block_threads"] == threads
+
+
 def test_wide_in_place_and_grids():
     dim = 70000
     x = wl.random_rows(300, dim, torch.bfloat16, seed=9).cuda()

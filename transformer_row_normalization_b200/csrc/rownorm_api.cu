@@ -287,7 +287,7 @@ int slot_class(const SegPlan& p, int chunks) {
 
 const void* kernel_for(int dtype, int op, const SegPlan& p, int slots) {
   const bool ex = p.exact != 0;
-  if (p.family == 2) return rn::stream_kernel(dtype == RN_F32, op, ex);
+  if (p.family == 2) return rn::stream_kernel(dtype == RN_F32, op, ex, p.lanes);
   if (p.family == 0)
     return dtype == RN_F32 ? rn::warp_kernel_f32(op, ex, slots, p.chunks)
                            : rn::warp_kernel_bf16(op, ex, slots, p.chunks);
@@ -650,12 +650,31 @@ int validate_single(const rn_view* x, const void* w, const void* b, float eps,
   return check_output(y, x, nullptr, 0, vecs, dims, 2, "y");
 }
 
+// Streaming rows: LayerNorm reads each row three times, the last two from
+// L2, so while two rows per SM fit there comfortably (rows of at most
+// kStreamPairMaxRowBytes: 296 rows in flight, 57 MB of the 126 MB L2) it
+// runs two blocks of 512 threads per SM, one row's passes overlapping the
+// other's. Measured on B200: bf16 D = 65536 497 -> 412 us, binary32
+// D = 32768 457 -> 404 us, bf16 D = 40001 1161 -> 993 us; at bf16
+// D = 262144 (512 KB rows, which two per SM overflow L2) 642 -> 662 us.
+// RMSNorm (two passes) ran slower with two blocks (381 -> 403 us at bf16
+// D = 65536) and keeps one block of 1024.
+SegPlan stream_plan(int op, const rn_view* x, SegPlan p) {
+  const int64_t row_bytes = x->dim * elem_size(x->dtype);
+  if (op == rn::kOpLn && row_bytes <= rn::kStreamPairMaxRowBytes) {
+    p.lanes = rn::kStreamPairThreads;
+    p.chunks = (int)ceil_div(x->dim / (16 / elem_size(x->dtype)), p.lanes);
+  }
+  return p;
+}
+
 int run_single(int op, const rn_view* x, const void* w, const void* b, float eps,
                const rn_view* y, void* stream, rn_launch_info* plan_only) {
   int st = validate_single(x, w, b, eps, y);
   if (st) return st;
   if (x->rows == 0 && !plan_only) return RN_OK;
-  const SegPlan p = plan_segment(x, y, w, b);
+  SegPlan p = plan_segment(x, y, w, b);
+  if (p.family == 2) p = stream_plan(op, x, p);
   Launch l{};
   const rn_view* xs[1] = {x};
   const void* ws[1] = {w};

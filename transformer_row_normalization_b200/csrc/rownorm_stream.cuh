@@ -1,17 +1,17 @@
 // Streaming row normalization for rows too wide to hold in registers
 // (sm_100a).
 //
-// One block of kStreamThreads threads per row, rows strided statically over
-// a persistent grid. The row is read once per pass: RMSNorm makes two
+// One block of NT threads per row (1024, or 512 for two rows per SM), rows
+// strided statically over a persistent grid. The row is read once per pass: RMSNorm makes two
 // passes (sum of squares, then normalize and store), LayerNorm three (sum
 // of d = x - K with K = x_0, then sum of (d - mean)^2, then normalize and
 // store): the same shifted two-pass statistics as the register kernels, so
 // a constant row still gives exactly the bias. Passes after the first find
-// the row in L2 while the rows in flight (one per SM) fit there.
+// the row in L2 while the rows in flight (one or two per SM) fit there.
 //
 // Ownership and summation order (fixed; they depend only on D, the element
 // type and the row's 16-byte phase): thread t owns the full chunks t,
-// t + kStreamThreads, ... and edge element t (rownorm_core.cuh's row split);
+// t + NT, ... and edge element t (rownorm_core.cuh's row split);
 // each pass sums the thread's chunks into even / odd binary32 pair
 // partials in chunk order, adds the edge element's term, and combines the
 // threads with block_sum. The arithmetic of each element is that of the
@@ -23,7 +23,6 @@
 
 namespace rn {
 
-constexpr int kStreamThreads = 1024;
 // chunks a thread loads before it uses the first of them (loads in flight)
 constexpr int kStreamUnroll = 4;
 
@@ -73,18 +72,18 @@ __device__ __forceinline__ void stream_affine(const Segment& s, const Row<T>& g,
 
 // One pass over the thread's chunks of row g: `chunk(v)` folds each chunk's
 // pairs into the accumulator (chunk order), kStreamUnroll loads in flight.
-template <typename T, typename Fold>
+template <typename T, int NT, typename Fold>
 __device__ __forceinline__ void stream_pass(const Row<T>& g, int tid, Fold fold) {
   constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
   int f = tid;
 #pragma unroll 1
-  constexpr int kStep = kStreamUnroll * kStreamThreads;
-  for (; f + (kStreamUnroll - 1) * kStreamThreads < g.nfull; f += kStep) {
+  constexpr int kStep = kStreamUnroll * NT;
+  for (; f + (kStreamUnroll - 1) * NT < g.nfull; f += kStep) {
     uint4 u[kStreamUnroll];
 #pragma unroll
     for (int q = 0; q < kStreamUnroll; ++q)
-      u[q] = load_keep(g.x_full + (long long)(f + q * kStreamThreads) * V);
+      u[q] = load_keep(g.x_full + (long long)(f + q * NT) * V);
 #pragma unroll
     for (int q = 0; q < kStreamUnroll; ++q) {
       F2 v[P];
@@ -93,23 +92,23 @@ __device__ __forceinline__ void stream_pass(const Row<T>& g, int tid, Fold fold)
     }
   }
 #pragma unroll 1
-  for (; f < g.nfull; f += kStreamThreads) {
+  for (; f < g.nfull; f += NT) {
     F2 v[P];
     Elem<T>::unpack(load_keep(g.x_full + (long long)f * V), v);
     fold(v);
   }
 }
 
-template <typename T, int OP, bool EXACT>
-__global__ void __launch_bounds__(kStreamThreads, 1) rows_stream_kernel(const Params p) {
+template <typename T, int OP, bool EXACT, int NT>
+__global__ void __launch_bounds__(NT, 1024 / NT) rows_stream_kernel(const Params p) {
   static_assert(OP == kOpRms || OP == kOpLn, "streaming covers RMSNorm and LayerNorm");
   constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
   constexpr bool BIAS = OP == kOpLn;
-  __shared__ float red[2][kStreamThreads / 32];
+  __shared__ float red[2][NT / 32];
   int slot = 0;
   auto reduce = [&](float t) {
-    const float r = block_sum<kStreamThreads>(t, red[slot]);
+    const float r = block_sum<NT>(t, red[slot]);
     slot ^= 1;
     return r;
   };
@@ -125,7 +124,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) rows_stream_kernel(const Pa
     float rstd, mean = 0.f;
     if constexpr (OP == kOpRms) {
       F2 acc = zero2();
-      stream_pass<T>(g, tid, [&](F2 (&v)[P]) {
+      stream_pass<T, NT>(g, tid, [&](F2 (&v)[P]) {
 #pragma unroll
         for (int j = 0; j < P; ++j) acc = fma2(v[j], v[j], acc);
       });
@@ -136,7 +135,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) rows_stream_kernel(const Pa
       const float K = Elem<T>::get(g.x_row);
       const F2 K2 = splat(K);
       F2 acc = zero2();
-      stream_pass<T>(g, tid, [&](F2 (&v)[P]) {
+      stream_pass<T, NT>(g, tid, [&](F2 (&v)[P]) {
 #pragma unroll
         for (int j = 0; j < P; ++j) acc = add2(acc, sub2(v[j], K2));
       });
@@ -148,7 +147,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) rows_stream_kernel(const Pa
       mean = __fmul_rn(reduce(part), inv_d);
       const F2 M2 = splat(mean);
       acc = zero2();
-      stream_pass<T>(g, tid, [&](F2 (&v)[P]) {
+      stream_pass<T, NT>(g, tid, [&](F2 (&v)[P]) {
 #pragma unroll
         for (int j = 0; j < P; ++j) {
           const F2 t = sub2(sub2(v[j], K2), M2);
@@ -172,7 +171,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) rows_stream_kernel(const Pa
     };
     const bool aligned = EXACT || (vec_aligned(s.w) && (!BIAS || vec_aligned(s.b)));
 #pragma unroll 1
-    for (int f = tid; f < g.nfull; f += kStreamThreads) {
+    for (int f = tid; f < g.nfull; f += NT) {
       F2 v[P], wf[P], bf[P], o[P];
       Elem<T>::unpack(load_stream(g.x_full + (long long)f * V), v);
       stream_affine<T, BIAS>(s, g, f, aligned, wf, bf);
