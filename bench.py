@@ -186,14 +186,15 @@ class ClockSampler:
 
 
 class Step:
-    """The large bf16 workloads on one device, with outputs preallocated."""
+    """Workloads (by default the large bf16 suite) on one device, with outputs
+    preallocated."""
 
-    def __init__(self, device, rank):
+    def __init__(self, device, rank, names=wl.LARGE_SUITE):
         import transformer_row_normalization_b200 as rn
         self.rn = rn
         self.device = device
         self.items = []
-        for name in wl.LARGE_SUITE:
+        for name in names:
             w = wl.WORKLOADS[name]
             rw = wl.Workload(w.name, w.op, w.dtype, w.shape, w.eps, rank_seed(w.seed, rank),
                              k_shape=w.k_shape)
@@ -409,6 +410,71 @@ def time_fused(device, rank, dist, peak, reps=30, oracle_rows=2048):
                       f"{oracle_rows} rows, fp64, {cores} threads"}
 
 
+def time_configs(step, small, device, dist, peak, reps=30, burst=100):
+    """Every config alone, cold and warm: min and median of `reps` CUDA-event
+    timings on the launching stream after 3 warm-up launches. Cold: each rep
+    follows a 256 MB read (over twice the 126 MB L2), which evicts the
+    config's data and leaves L2 clean; a flush by writing would leave ~126 MB
+    of dirty lines for the timed launch to write back. Warm: no flush; each
+    rep times one launch of a large config right after another, or one replay
+    of a CUDA graph of `burst` launches of a small one (per-launch time =
+    total / burst; eager Python launches of a few-microsecond kernel would
+    time the host). Large configs carry a roofline fraction (cold median); the
+    small ones fit in L2 and are launch-bound, so they carry none. Max over
+    ranks."""
+    flush = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    out = []
+    for st, large in ((step, True), (small, False)):
+        for i, (w, _, _) in enumerate(st.items):
+            for _ in range(3):
+                st.launch(i)
+            n = 1 if large else burst
+            graph = None
+            if not large:
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph):
+                    for _ in range(n):
+                        st.launch(i)
+                graph.replay()
+            cold = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                    for _ in range(reps)]
+            for a, b in cold:
+                flush.sum()
+                a.record(stream)
+                st.launch(i)
+                b.record(stream)
+            warm = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                    for _ in range(reps)]
+            for a, b in warm:
+                a.record(stream)
+                if graph is not None:
+                    graph.replay()
+                else:
+                    st.launch(i)
+                b.record(stream)
+            torch.cuda.synchronize(device)
+            del graph
+            tc = sorted(a.elapsed_time(b) * 1e3 for a, b in cold)
+            tw = sorted(a.elapsed_time(b) * 1e3 / n for a, b in warm)
+            tc = [max_over_ranks(t, dist, device) for t in (tc[0], tc[len(tc) // 2])]
+            tw = [max_over_ranks(t, dist, device) for t in (tw[0], tw[len(tw) // 2])]
+            item = {"workload": w.name, "us_cold_min": round(tc[0], 2),
+                    "us_cold_median": round(tc[1], 2), "us_warm_min": round(tw[0], 2),
+                    "us_warm_median": round(tw[1], 2),
+                    "rows_per_s_cold": round(w.total_rows / (tc[1] * 1e-6)),
+                    "rows_per_s_warm": round(w.total_rows / (tw[1] * 1e-6))}
+            if large:
+                g = w.algorithmic_bytes() / (tc[1] * 1e-6) / 1e9
+                item["gbs_cold"] = round(g, 1)
+                item["frac_cold"] = round(g / peak, 4)
+            out.append(item)
+    return {"items": out,
+            "timing": f"min and median of {reps} reps after 3 warm-up launches; cold: each "
+                      "rep after a 256 MB read that evicts L2; warm: no flush, small configs "
+                      f"timed as one replay of a CUDA graph of {burst} launches"}
+
+
 # ---------------------------------------------------------------------------
 
 
@@ -480,6 +546,7 @@ def run_ours(args):
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
     fused = time_fused(device, rank, dist, peak)
+    configs = time_configs(step, Step(device, rank, wl.SMALL_SUITE), device, dist, peak)
     base = cpu_baseline(step) if (rank == 0 and world == 1) else None
     if dist is not None:
         barrier(dist, device)
@@ -495,7 +562,7 @@ def run_ours(args):
                     "peak_source": peak_kind},
             "roofline": roofline, "cpu_baseline": base, "e2e": e2e,
             "gpu_launches": 7 * args.steps, "clocks": clk, "per_config": per_config,
-            "fused": fused,
+            "configs": configs, "fused": fused,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -71,8 +71,9 @@ def test_wide_layouts(dtype):
     ("ln", torch.float32, 49152, 512), ("ln", torch.float32, 49153, 1024),
     ("rms", torch.bfloat16, 65536, 1024), ("rms", torch.float32, 32768, 1024)])
 def test_stream_block_size(op, dtype, dim, threads):
-    """LayerNorm rows of at most 192 KB stream two rows per SM (512 threads
-    each); wider rows and RMSNorm one row per SM (1024 threads)."""
+    """LayerNorm rows of at most 192 KB stream in blocks of 512 threads
+    (several rows per SM); wider rows and RMSNorm in blocks of 1024 (one row
+    per SM)."""
     x = torch.empty(2, dim, dtype=dtype, device="cuda")
     w = torch.empty(dim, dtype=dtype, device="cuda")
     kind = rn.RN_OP_LN if op == "ln" else rn.RN_OP_RMS

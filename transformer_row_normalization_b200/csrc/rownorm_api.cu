@@ -651,12 +651,12 @@ int validate_single(const rn_view* x, const void* w, const void* b, float eps,
 }
 
 // Streaming rows: LayerNorm reads each row three times, the last two from
-// L2, so while two rows per SM fit there comfortably (rows of at most
-// kStreamPairMaxRowBytes: 296 rows in flight, 57 MB of the 126 MB L2) it
-// runs two blocks of 512 threads per SM, one row's passes overlapping the
-// other's. Measured on B200: bf16 D = 65536 497 -> 412 us, binary32
+// L2, so while several rows per SM fit there (rows of at most
+// kStreamPairMaxRowBytes; at 38 registers 3 blocks of 512 threads run per
+// SM, 444 rows in flight, 85 MB of the 126 MB L2 at the limit) it runs
+// blocks of 512 threads, one row's passes overlapping the others'. Measured on B200: bf16 D = 65536 497 -> 412 us, binary32
 // D = 32768 457 -> 404 us, bf16 D = 40001 1161 -> 993 us; at bf16
-// D = 262144 (512 KB rows, which two per SM overflow L2) 642 -> 662 us.
+// D = 262144 (512 KB rows, which several per SM overflow L2) 642 -> 662 us.
 // RMSNorm (two passes) ran slower with two blocks (381 -> 403 us at bf16
 // D = 65536) and keeps one block of 1024.
 SegPlan stream_plan(int op, const rn_view* x, SegPlan p) {

@@ -52,8 +52,8 @@ const void* cta_kernel_bf16(int op, bool exact, int slots, int threads, int chun
 // Streaming kernels (rows wider than the register kernels hold): RMSNorm
 // and LayerNorm, any layout.
 const void* stream_kernel(int dtype_f32, int op, bool exact, int threads);
-// Threads per row of the streaming kernels: one block of 1024 per SM, or
-// (LayerNorm rows up to kStreamPairMaxRowBytes) two blocks of 512 per SM.
+// Threads per row of the streaming kernels: 1024 (one block per SM), or 512
+// for LayerNorm rows up to kStreamPairMaxRowBytes (several blocks per SM).
 constexpr int kStreamBlockThreads = 1024;
 constexpr int kStreamPairThreads = 512;
 constexpr long long kStreamPairMaxRowBytes = 192 * 1024;

@@ -1,13 +1,14 @@
 // Streaming row normalization for rows too wide to hold in registers
 // (sm_100a).
 //
-// One block of NT threads per row (1024, or 512 for two rows per SM), rows
-// strided statically over a persistent grid. The row is read once per pass: RMSNorm makes two
-// passes (sum of squares, then normalize and store), LayerNorm three (sum
-// of d = x - K with K = x_0, then sum of (d - mean)^2, then normalize and
-// store): the same shifted two-pass statistics as the register kernels, so
-// a constant row still gives exactly the bias. Passes after the first find
-// the row in L2 while the rows in flight (one or two per SM) fit there.
+// One block of NT threads per row (1024, or 512 for several rows per SM),
+// rows strided statically over a persistent grid. The row is read once per
+// pass: RMSNorm makes two passes (sum of squares, then normalize and store),
+// LayerNorm three (sum of d = x - K with K = x_0, then sum of (d - mean)^2,
+// then normalize and store): the same shifted two-pass statistics as the
+// register kernels, so a constant row still gives exactly the bias. Passes
+// after the first find the row in L2 while the rows in flight (one or a few
+// per SM) fit there.
 //
 // Ownership and summation order (fixed; they depend only on D, the element
 // type and the row's 16-byte phase): thread t owns the full chunks t,
