@@ -40,6 +40,7 @@ from transformer_row_normalization_b200 import workloads as wl  # noqa: E402
 METRIC = "normalized rows/sec and achieved HBM GB/s as % of B200 peak, 1 GPU"
 FALLBACK_HBM_GBS = 6650.0
 CSRC = os.path.join(ROOT, "transformer_row_normalization_b200", "csrc")
+INCLUDE = os.path.join(ROOT, "include")
 
 
 def log(*a):
@@ -102,11 +103,14 @@ def measured_peak():
 
 
 def source_digest():
+    """Digest of the sources the kernels are built from: the CUDA sources
+    and the C-ABI header."""
     h = hashlib.sha256()
-    for name in sorted(os.listdir(CSRC)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(CSRC, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for d in (CSRC, INCLUDE):
+        for name in sorted(os.listdir(d)):
+            if name.endswith((".cu", ".cuh", ".h")):
+                with open(os.path.join(d, name), "rb") as f:
+                    h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 

@@ -67,10 +67,9 @@ extern "C" {
 
 #define RN_ABI_VERSION 3
 
-/* Largest supported dim. Rows are held on chip (registers) between reading
- * and writing, so x is read from HBM exactly once; wider rows are rejected
- * with RN_ERR_UNSUPPORTED. */
-/* Widest rows the register kernels hold (every op). rn_rms_norm and
+/* Widest rows the register kernels hold (every op): a row stays on chip
+ * between reading and writing, so x is read from HBM exactly once. The fused
+ * ops reject wider rows with RN_ERR_UNSUPPORTED. rn_rms_norm and
  * rn_layer_norm take wider rows, up to RN_MAX_DIM_STREAM, through streaming
  * kernels that read each row once per pass (two passes for RMSNorm, three for
  * LayerNorm; the later ones from L2 while the rows in flight fit there). */
@@ -272,11 +271,14 @@ RN_API int rn_abi_version(void);
 
 typedef struct rn_launch_info {
     int32_t family;         /* 0: a group of lanes of one warp per row;    */
-                            /* 1: one thread block (CTA) per row           */
+                            /* 1: one thread block (CTA) per row;          */
+                            /* 2: one block per row, streaming (rows wider */
+                            /* than the register kernels hold)             */
     int32_t threads_per_row;/* lanes sharing one row                        */
     int32_t chunks_per_thread; /* 16-byte chunks of a row each thread holds */
-    int32_t smem_bytes;     /* dynamic shared memory per block (weight and  */
-                            /* bias columns of each thread's chunks)        */
+    int32_t smem_bytes;     /* dynamic shared memory per block: realigned   */
+                            /* weight/bias of each thread's chunks (rows   */
+                            /* off the 16-byte grid) and prefetch slots    */
     int32_t block_threads;  /* threads per block                            */
     int32_t grid_blocks;    /* blocks launched (persistent: <= SMs x blocks */
                             /* resident per SM)                             */
