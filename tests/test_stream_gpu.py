@@ -65,6 +65,37 @@ def test_wide_layouts(dtype):
           what="ln gapped out, null vectors")
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_wide_shifted_vectors(dtype):
+    """Rows off the 16-byte grid at every phase. With weight and bias at one
+    common offset from the grid, their chunk columns come from two aligned
+    words shifted into place. Those must give exactly the bits of
+    element-by-element loads, taken when weight and bias sit at different
+    offsets, and parity with the oracle."""
+    dim = 40001 if dtype == torch.bfloat16 else 20001
+    rows = 17  # every 16-byte phase of an odd width, twice
+    x = wl.random_rows(rows, dim, dtype, seed=21, mean=0.5, std=2.0).cuda()
+    wv = wl.random_vector(dim, dtype, seed=22).cuda()
+    bv = wl.random_vector(dim, dtype, seed=23, mean=0.0, std=0.1).cuda()
+    for off in (0, 1, 3):
+        # common offset `off`: shifted loads (or, at 0, aligned ones)
+        wbuf = torch.zeros(dim + 8, dtype=dtype, device="cuda")
+        bbuf = torch.zeros(dim + 8, dtype=dtype, device="cuda")
+        wbuf[off:off + dim] = wv
+        bbuf[off:off + dim] = bv
+        shifted = (rn.layer_norm(x, wbuf[off:off + dim], bbuf[off:off + dim], 1e-5),
+                   rn.rms_norm(x, wbuf[off:off + dim], 1e-6))
+        # bias one element further: weight and bias at different offsets
+        b2 = torch.zeros(dim + 8, dtype=dtype, device="cuda")
+        b2[off + 1:off + 1 + dim] = bv
+        elementwise = rn.layer_norm(x, wbuf[off:off + dim], b2[off + 1:off + 1 + dim], 1e-5)
+        torch.cuda.synchronize()
+        assert torch.equal(shifted[0], elementwise), off
+        check(shifted[0], oracle.layer_norm(host(x), host(wv), host(bv), 1e-5), dtype, bias=bv,
+              what=f"ln offset {off}")
+        check(shifted[1], oracle.rms_norm(host(x), host(wv), 1e-6), dtype, what=f"rms offset {off}")
+
+
 @pytest.mark.parametrize("op,dtype,dim,threads", [
     ("ln", torch.bfloat16, 65536, 512), ("ln", torch.bfloat16, 98304, 512),
     ("ln", torch.bfloat16, 98305, 1024), ("ln", torch.bfloat16, 262144, 1024),

@@ -32,42 +32,64 @@ __device__ __forceinline__ uint4 load_keep(const void* p) {
   return __ldg(reinterpret_cast<const uint4*>(p));
 }
 
-// Weight (and bias) of chunk f's columns for any layout: one aligned 16-byte
-// load per vector when the vector's columns are aligned with the row's
-// chunks, else element by element.
-template <typename T, bool BIAS>
-__device__ __forceinline__ void stream_affine(const Segment& s, const Row<T>& g, int f,
-                                              bool aligned, F2 (&wf)[Elem<T>::P],
-                                              F2 (&bf)[Elem<T>::P]) {
+// Where a vector's columns stand relative to the 16-byte grid at the row's
+// chunks: kVecAligned (each chunk's columns are one aligned 16-byte word),
+// an offset O in 1..V-1 elements past a boundary, or kVecElementwise
+// (weight and bias at different offsets: element-by-element loads).
+constexpr int kVecAligned = 0;
+constexpr int kVecElementwise = -1;
+
+// The V elements at p = pa + O (pa 16-byte aligned, 0 < O < V): the two
+// aligned words at pa shifted down by O elements. Funnel shifts over the
+// little-endian 32-bit lanes of the pair; both words must lie inside the
+// vector (the caller checks).
+template <typename T, int O>
+__device__ __forceinline__ uint4 load_shifted(const T* pa) {
+  constexpr int V = Elem<T>::V;
+  constexpr int kBytes = O * (int)sizeof(T);
+  static_assert(O > 0 && O < V, "offset within one 16-byte word");
+  const uint4 lo = load_cached(pa);
+  const uint4 hi = load_cached(pa + V);
+  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+  uint32_t r[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    if constexpr (kBytes % 4 == 0)
+      r[j] = w[kBytes / 4 + j];
+    else
+      r[j] = __funnelshift_r(w[kBytes / 4 + j], w[kBytes / 4 + j + 1], 8 * (kBytes % 4));
+  }
+  return make_uint4(r[0], r[1], r[2], r[3]);
+}
+
+// Chunk f's columns of vector v (NULL: `none` everywhere) under offset
+// class O.
+template <typename T, int O>
+__device__ __forceinline__ void stream_vector(const T* v, const Row<T>& g, int D, int f,
+                                              float none, F2 (&vf)[Elem<T>::P]) {
   constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
-  const T* w = static_cast<const T*>(s.w);
-  const T* b = static_cast<const T*>(s.b);
+  if (!v) {
+#pragma unroll
+    for (int j = 0; j < P; ++j) vf[j] = splat(none);
+    return;
+  }
   const int c0 = g.head + f * V;
-  if (aligned) {
-    if (w) {
-      Elem<T>::unpack(load_cached(w + c0), wf);
-    } else {
-#pragma unroll
-      for (int j = 0; j < P; ++j) wf[j] = splat(1.f);
-    }
-    if constexpr (BIAS) {
-      if (b) {
-        Elem<T>::unpack(load_cached(b + c0), bf);
-      } else {
-#pragma unroll
-        for (int j = 0; j < P; ++j) bf[j] = zero2();
+  if constexpr (O == kVecAligned) {
+    Elem<T>::unpack(load_cached(v + c0), vf);
+    return;
+  } else {
+    if constexpr (O != kVecElementwise) {
+      // both aligned words inside the vector: all chunks but at most the
+      // first and the last
+      if (c0 - O >= 0 && c0 - O + 2 * V <= D) {
+        Elem<T>::unpack(load_shifted<T, O>(v + (c0 - O)), vf);
+        return;
       }
     }
-  } else {
 #pragma unroll
-    for (int j = 0; j < P; ++j) {
-      wf[j] = w ? make2(Elem<T>::get(w + c0 + 2 * j), Elem<T>::get(w + c0 + 2 * j + 1))
-                : splat(1.f);
-      if constexpr (BIAS)
-        bf[j] = b ? make2(Elem<T>::get(b + c0 + 2 * j), Elem<T>::get(b + c0 + 2 * j + 1))
-                  : zero2();
-    }
+    for (int j = 0; j < P; ++j)
+      vf[j] = make2(Elem<T>::get(v + c0 + 2 * j), Elem<T>::get(v + c0 + 2 * j + 1));
   }
 }
 
@@ -78,7 +100,6 @@ __device__ __forceinline__ void stream_pass(const Row<T>& g, int tid, Fold fold)
   constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
   int f = tid;
-#pragma unroll 1
   constexpr int kStep = kStreamUnroll * NT;
   for (; f + (kStreamUnroll - 1) * NT < g.nfull; f += kStep) {
     uint4 u[kStreamUnroll];
@@ -100,10 +121,61 @@ __device__ __forceinline__ void stream_pass(const Row<T>& g, int tid, Fold fold)
   }
 }
 
+// The last pass over row g: normalize, weight (and bias) under vector
+// offset class O, store the thread's full chunks.
+template <typename T, int OP, bool EXACT, int NT, int O>
+__device__ __forceinline__ void stream_store(const Segment& s, const Row<T>& g, int tid, F2 R2,
+                                             F2 M2, F2 K2) {
+  constexpr int V = Elem<T>::V;
+  constexpr int P = Elem<T>::P;
+  const T* w = static_cast<const T*>(s.w);
+  const T* b = static_cast<const T*>(s.b);
+#pragma unroll 1
+  for (int f = tid; f < g.nfull; f += NT) {
+    F2 v[P], wf[P], bf[P], o[P];
+    Elem<T>::unpack(load_stream(g.x_full + (long long)f * V), v);
+    stream_vector<T, O>(w, g, s.dim, f, 1.f, wf);
+    if constexpr (OP == kOpLn) stream_vector<T, O>(b, g, s.dim, f, 0.f, bf);
+#pragma unroll
+    for (int j = 0; j < P; ++j) {
+      if constexpr (OP == kOpLn)
+        o[j] = fma2(mul2(sub2(sub2(v[j], K2), M2), R2), wf[j], bf[j]);
+      else
+        o[j] = mul2(mul2(v[j], R2), wf[j]);
+    }
+    T* yc = g.y_row + g.head + (long long)f * V;
+    if (EXACT || s.vector_y) {
+      store_stream(yc, Elem<T>::pack(o));
+    } else {
+#pragma unroll
+      for (int j = 0; j < P; ++j) {
+        Elem<T>::put(yc + 2 * j, o[j].x);
+        Elem<T>::put(yc + 2 * j + 1, o[j].y);
+      }
+    }
+  }
+}
+
+// stream_store under the runtime offset class `cls` (rows off the grid).
+template <typename T, int OP, int NT, int O = 1>
+__device__ __forceinline__ void stream_store_offset(int cls, const Segment& s, const Row<T>& g,
+                                                    int tid, F2 R2, F2 M2, F2 K2) {
+  if constexpr (O < Elem<T>::V) {
+    if (cls == O) {
+      stream_store<T, OP, false, NT, O>(s, g, tid, R2, M2, K2);
+    } else {
+      stream_store_offset<T, OP, NT, O + 1>(cls, s, g, tid, R2, M2, K2);
+    }
+  } else if (cls == kVecAligned) {
+    stream_store<T, OP, false, NT, kVecAligned>(s, g, tid, R2, M2, K2);
+  } else {
+    stream_store<T, OP, false, NT, kVecElementwise>(s, g, tid, R2, M2, K2);
+  }
+}
+
 template <typename T, int OP, bool EXACT, int NT>
 __global__ void __launch_bounds__(NT, 1024 / NT) rows_stream_kernel(const Params p) {
   static_assert(OP == kOpRms || OP == kOpLn, "streaming covers RMSNorm and LayerNorm");
-  constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
   constexpr bool BIAS = OP == kOpLn;
   __shared__ float red[2][NT / 32];
@@ -166,33 +238,21 @@ __global__ void __launch_bounds__(NT, 1024 / NT) rows_stream_kernel(const Params
     const F2 R2 = splat(rstd);
     const F2 M2 = splat(mean);
     const F2 K2 = splat(OP == kOpLn ? Elem<T>::get(g.x_row) : 0.f);  // LayerNorm shift
-    // the vectors' columns of a chunk start 16-byte aligned (EXACT: always)
-    auto vec_aligned = [&](const void* v) {
-      return !v || (reinterpret_cast<uintptr_t>(static_cast<const T*>(v) + g.head) % 16) == 0;
-    };
-    const bool aligned = EXACT || (vec_aligned(s.w) && (!BIAS || vec_aligned(s.b)));
-#pragma unroll 1
-    for (int f = tid; f < g.nfull; f += NT) {
-      F2 v[P], wf[P], bf[P], o[P];
-      Elem<T>::unpack(load_stream(g.x_full + (long long)f * V), v);
-      stream_affine<T, BIAS>(s, g, f, aligned, wf, bf);
-#pragma unroll
-      for (int j = 0; j < P; ++j) {
-        if constexpr (OP == kOpLn)
-          o[j] = fma2(mul2(sub2(sub2(v[j], K2), M2), R2), wf[j], bf[j]);
-        else
-          o[j] = mul2(mul2(v[j], R2), wf[j]);
-      }
-      T* yc = g.y_row + g.head + (long long)f * V;
-      if (EXACT || s.vector_y) {
-        store_stream(yc, Elem<T>::pack(o));
-      } else {
-#pragma unroll
-        for (int j = 0; j < P; ++j) {
-          Elem<T>::put(yc + 2 * j, o[j].x);
-          Elem<T>::put(yc + 2 * j + 1, o[j].y);
-        }
-      }
+    if constexpr (EXACT) {
+      stream_store<T, OP, true, NT, kVecAligned>(s, g, tid, R2, M2, K2);
+    } else {
+      // elements from the 16-byte boundary to the columns of the row's
+      // first chunk, per present vector; different offsets go element-wise
+      auto offset = [&](const void* v) {
+        return v ? (int)((reinterpret_cast<uintptr_t>(static_cast<const T*>(v) + g.head) % 16) /
+                         sizeof(T))
+                 : -2;
+      };
+      const int ow = offset(s.w);
+      const int ob = BIAS ? offset(s.b) : -2;
+      const int cls = ow == -2 ? (ob == -2 ? kVecAligned : ob)
+                               : (ob == -2 || ob == ow ? ow : kVecElementwise);
+      stream_store_offset<T, OP, NT>(cls, s, g, tid, R2, M2, K2);
     }
     if (has_edge) {
       const int c = edge_column(g, D, tid);
