@@ -515,9 +515,9 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
   const int cache = (merged.exact || stream)
                         ? 0
                         : rn::affine_cache_smem_bytes(op, threads, merged.chunks);
-  const int pf_bytes = rn::prefetch_slots_smem_bytes(
-                           threads, merged.chunks,
-                           merged.family == 0 ? rn::kWarpPrefetchStages : rn::kCtaPrefetchStages) *
+  const int stages =
+      merged.family == 0 ? rn::kWarpPrefetchStages : rn::cta_prefetch_stages(threads);
+  const int pf_bytes = rn::prefetch_slots_smem_bytes(threads, merged.chunks, stages) *
                        (rn::op_has_second(op) ? 2 : 1);
   // Next-row prefetch where it measured faster on B200: lane-group rows and
   // blocks of 256 or more threads (few blocks per SM, so few rows in

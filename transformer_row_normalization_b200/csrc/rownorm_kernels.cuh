@@ -129,11 +129,17 @@ struct Prefetch {
 
 // Prefetch stages per thread: rows in flight while one is normalized from
 // registers. Measured on B200 (back-to-back bf16 LayerNorm, D = 768 to
-// 16384), two rows ahead beat one by 2-4 % for blocks, while a third stage
-// cost blocks 10-14 % (its slots squeeze the L1 share that holds the weight
-// and bias) and moved lane groups by no more than noise.
+// 16384): lane groups keep two (a third moved them by no more than noise).
+// Blocks of 256 or more threads, which prefetch, keep one: one row in flight
+// in half the shared memory leaves L1 room for the weight and bias
+// (LayerNorm 16384: 777 -> 746 us, 8192: 357 -> 349 us against two stages;
+// a third stage cost 10-14 %). Blocks of 128 threads prefetch nothing; their
+// two queue entries issue the shift and edge loads two rows ahead (LayerNorm
+// 4097: 224 -> 219 us against one).
 constexpr int kWarpPrefetchStages = 2;
-constexpr int kCtaPrefetchStages = 2;
+__host__ __device__ constexpr int cta_prefetch_stages(int threads) {
+  return threads >= 256 ? 1 : 2;
+}
 
 // 16-byte words of prefetch slots of one bank.
 template <int NSLOT, int NST>
@@ -358,7 +364,7 @@ rows_cta_kernel(const Params p) {
   // Two alternating reduction buffers: a buffer is rewritten only after every
   // thread has passed the barrier of the reduction in between.
   __shared__ float red[2][NT / 32];
-  constexpr int BANK = prefetch_smem_words<VPT, kCtaPrefetchStages>(NT);
+  constexpr int BANK = prefetch_smem_words<VPT, cta_prefetch_stages(NT)>(NT);
   const Prefetch<T, VPT> pf{p.prefetch, 0};
   const Prefetch<T, VPT> pf2{p.prefetch, BANK};
   int slot = 0;
@@ -371,7 +377,7 @@ rows_cta_kernel(const Params p) {
 #pragma unroll 1
   for (int si = 0; si < p.nseg; ++si) {
     const Segment s = pick_segment(p.seg, si);
-    run_segment<T, OP, EXACT, SLOTS, VPT, kCtaPrefetchStages>(
+    run_segment<T, OP, EXACT, SLOTS, VPT, cta_prefetch_stages(NT)>(
         s, pf, pf2, blockIdx.x, gridDim.x, threadIdx.x, NT, p.eps, reduce, cache_word, nullptr,
         0u);
   }
