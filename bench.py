@@ -704,7 +704,7 @@ def main(argv=None):
                     help="OP:DTYPE:ROWS:DIM -- launch one workload for a profiler capture")
     ap.add_argument("--path", type=int, default=0,
                     help="kernel choice: 0 automatic, 1 register, 2 staged, "
-                         "3 register with next-row prefetch")
+                         "3 register with prefetch of the rows ahead")
     args = ap.parse_args(argv)
     if args.profile_case:
         return run_profile_case(args)

@@ -319,7 +319,8 @@ RN_API int rn_set_grid_override(int blocks);
 /* Kernel choice: 0 automatic; 1 register-resident kernels loading rows
  * directly; 2 the bulk-copy staged kernels (rows streamed through shared
  * memory) wherever the shape allows; 3 register-resident kernels with a
- * per-thread next-row prefetch through shared memory (cp.async). The per-row
+ * per-thread prefetch of the rows ahead through shared memory (cp.async),
+ * also where the planner would not prefetch. The per-row
  * arithmetic is identical in every kind of kernel, so results do not depend
  * on it. Process-wide; meant for tests and measurements. */
 RN_API int rn_set_path_override(int path);

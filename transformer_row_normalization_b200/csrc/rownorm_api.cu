@@ -375,7 +375,7 @@ int blocks_per_sm(int dev, const void* fn, int threads, int smem, int* out) {
 struct Launch {
   const void* fn;
   int smem;
-  int prefetch;     // register kernels: next-row prefetch through shared memory
+  int prefetch;     // register kernels: rows ahead prefetched through shared memory
   int staged;       // 1: rows_staged_kernel with StagedParams
   rn_launch_info info;
   // staged kernels only
@@ -519,7 +519,7 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
       merged.family == 0 ? rn::kWarpPrefetchStages : rn::cta_prefetch_stages(threads);
   const int pf_bytes = rn::prefetch_slots_smem_bytes(threads, merged.chunks, stages) *
                        (rn::op_has_second(op) ? 2 : 1);
-  // Next-row prefetch where it measured faster on B200: lane-group rows and
+  // Prefetch of the rows ahead where it measured faster on B200: lane groups and
   // blocks of 256 or more threads (few blocks per SM, so few rows in
   // flight); blocks of 128 threads already keep 8+ rows per SM in flight and
   // ran slower with it. Only when the slots fit beside the weight cache

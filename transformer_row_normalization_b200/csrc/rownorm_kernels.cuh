@@ -15,13 +15,13 @@
 // grid is a multiple of the phase period), so the realigned weight/bias
 // cache of non-aligned layouts is filled once.
 //
-// Prefetch. While a thread normalizes row r, its share of its next row is
-// already on its way: each thread copies its own full chunks of row
-// r + stride into its own shared memory slots with cp.async and waits only
-// for its own copies (cp.async.wait_group), so the HBM latency of a row hides
-// behind the previous row's arithmetic without any barrier. The shift K of
-// the next row (LayerNorm) and the thread's edge element of it are loaded
-// into registers at the same time.
+// Prefetch. While a thread normalizes row r, its share of the rows ahead
+// (r + stride, up to NST rows) is already on its way: each thread copies
+// its own full chunks of those rows into its own shared memory slots with
+// cp.async and waits only for its own copies (cp.async.wait_group), so the
+// HBM latency of a row hides behind earlier rows' arithmetic without any
+// barrier. The shift K of each row ahead (LayerNorm) and the thread's edge
+// element of it are loaded into registers when its copies are issued.
 //
 // The bulk-copy staged kernels (rownorm_staged.cuh) run the same per-row
 // code; which kernel the planner picks never changes a bit.
@@ -35,7 +35,7 @@ struct Params {
   Segment seg[2];
   int nseg;
   float eps;
-  int prefetch;  // 1: next-row prefetch through shared memory; 0: direct loads
+  int prefetch;  // 1: rows ahead prefetched through shared memory; 0: direct loads
   int stage_word;  // kOpRmsRope: first 16-byte word of the lane groups' staging rows
 };
 
