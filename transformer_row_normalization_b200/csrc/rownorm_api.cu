@@ -516,7 +516,7 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
                         ? 0
                         : rn::affine_cache_smem_bytes(op, threads, merged.chunks);
   const int stages =
-      merged.family == 0 ? rn::kWarpPrefetchStages : rn::cta_prefetch_stages(threads);
+      merged.family == 0 ? rn::kWarpPrefetchStages : rn::cta_prefetch_stages(threads, op);
   const int pf_bytes = rn::prefetch_slots_smem_bytes(threads, merged.chunks, stages) *
                        (rn::op_has_second(op) ? 2 : 1);
   // Prefetch of the rows ahead where it measured faster on B200: lane groups and

@@ -135,10 +135,12 @@ struct Prefetch {
 // (LayerNorm 16384: 777 -> 746 us, 8192: 357 -> 349 us against two stages;
 // a third stage cost 10-14 %). Blocks of 128 threads prefetch nothing; their
 // two queue entries issue the shift and edge loads two rows ahead (LayerNorm
-// 4097: 224 -> 219 us against one).
+// 4097: 224 -> 219 us against one). The gated op reads its gate from the
+// stage until the row is stored, so it refills late and keeps two stages:
+// one row in flight while it normalizes.
 constexpr int kWarpPrefetchStages = 2;
-__host__ __device__ constexpr int cta_prefetch_stages(int threads) {
-  return threads >= 256 ? 1 : 2;
+__host__ __device__ constexpr int cta_prefetch_stages(int threads, int op) {
+  return threads >= 256 && op != kOpGatedRms ? 1 : 2;
 }
 
 // 16-byte words of prefetch slots of one bank.
@@ -364,7 +366,7 @@ rows_cta_kernel(const Params p) {
   // Two alternating reduction buffers: a buffer is rewritten only after every
   // thread has passed the barrier of the reduction in between.
   __shared__ float red[2][NT / 32];
-  constexpr int BANK = prefetch_smem_words<VPT, cta_prefetch_stages(NT)>(NT);
+  constexpr int BANK = prefetch_smem_words<VPT, cta_prefetch_stages(NT, OP)>(NT);
   const Prefetch<T, VPT> pf{p.prefetch, 0};
   const Prefetch<T, VPT> pf2{p.prefetch, BANK};
   int slot = 0;
@@ -377,7 +379,7 @@ rows_cta_kernel(const Params p) {
 #pragma unroll 1
   for (int si = 0; si < p.nseg; ++si) {
     const Segment s = pick_segment(p.seg, si);
-    run_segment<T, OP, EXACT, SLOTS, VPT, cta_prefetch_stages(NT)>(
+    run_segment<T, OP, EXACT, SLOTS, VPT, cta_prefetch_stages(NT, OP)>(
         s, pf, pf2, blockIdx.x, gridDim.x, threadIdx.x, NT, p.eps, reduce, cache_word, nullptr,
         0u);
   }
