@@ -285,38 +285,50 @@ def time_e2e(step, k, stream):
     return start.elapsed_time(end), h2d, d2h
 
 
-def cpu_baseline(step, chunk_rows=2048):
+def cpu_baseline(step, chunk_rows=2048, single_share=16):
     """The fp64 oracle on the host cores over every row of one step (copied
     from the device in chunks of `chunk_rows` rows; only the oracle calls are
-    timed)."""
+    timed), and on one thread over the first 1/`single_share` of each
+    workload's rows (the step's row mix, a bounded sample)."""
     import oracle
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     # warm-up (page faults, thread pool) on a few rows
     w0, a0, _ = step.items[1]
     oracle.rms_norm(a0["x"].reshape(-1, w0.dim)[:64].cpu(), a0["w"].cpu(), w0.eps, nthreads=cores)
-    busy = 0.0
-    rows = 0
-    for w, a, _ in step.items:
+
+    def parts_of(w, a):
         if w.op == "dual":
-            parts = [(a["q"].reshape(-1, w.dim), a["wq"]), (a["k"].reshape(-1, w.k_shape[-1]), a["wk"])]
-            bias = None
+            return ([(a["q"].reshape(-1, w.dim), a["wq"]),
+                     (a["k"].reshape(-1, w.k_shape[-1]), a["wk"])], None)
+        return [(a["x"].reshape(-1, w.dim), a["w"])], (a["b"].cpu() if "b" in a else None)
+
+    def run(w, xc, wt, bias, n):
+        t0 = time.perf_counter()
+        if w.op == "ln":
+            oracle.layer_norm(xc, wt, bias, w.eps, nthreads=n)
         else:
-            parts = [(a["x"].reshape(-1, w.dim), a["w"])]
-            bias = a["b"].cpu() if "b" in a else None
+            oracle.rms_norm(xc, wt, w.eps, nthreads=n)
+        return time.perf_counter() - t0
+
+    busy = busy1 = 0.0
+    rows = rows1 = 0
+    for w, a, _ in step.items:
+        parts, bias = parts_of(w, a)
         for x, wt in parts:
             wt = wt.cpu()
             for r0 in range(0, x.shape[0], chunk_rows):
                 xc = x[r0:r0 + chunk_rows].cpu()
-                t0 = time.perf_counter()
-                if w.op == "ln":
-                    oracle.layer_norm(xc, wt, bias, w.eps, nthreads=cores)
-                else:
-                    oracle.rms_norm(xc, wt, w.eps, nthreads=cores)
-                busy += time.perf_counter() - t0
+                busy += run(w, xc, wt, bias, cores)
                 rows += xc.shape[0]
+            xc = x[:max(1, x.shape[0] // single_share)].cpu()
+            busy1 += run(w, xc, wt, bias, 1)
+            rows1 += xc.shape[0]
     return {"value": round(rows / busy, 1), "unit": "rows/s", "cores": cores, "kind": "oracle",
             "sample": f"one full step ({rows} rows, every workload), fp64, {cores} threads, "
-                      f"{busy:.1f} s of oracle time"}
+                      f"{busy:.1f} s of oracle time",
+            "single_thread": {"value": round(rows1 / busy1, 1), "unit": "rows/s", "cores": 1,
+                              "sample": f"the first 1/{single_share} of each workload's rows "
+                                        f"({rows1} rows), fp64, 1 thread, {busy1:.1f} s"}}
 
 
 def time_fused(device, rank, dist, peak, reps=30, oracle_rows=2048):

@@ -88,3 +88,21 @@ def test_warmup_minimum_enforced():
     res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--warmup", "1"],
                          capture_output=True, text=True, timeout=120, cwd=ROOT)
     assert res.returncode != 0
+
+
+def test_cpu_baseline_times_all_cores_and_one_thread():
+    """cpu_baseline over a step's items (host tensors here): every row on all
+    cores, and a proportional sample on one thread."""
+    from transformer_row_normalization_b200 import workloads as wl
+
+    class FakeStep:
+        items = [(wl.WORKLOADS[n], wl.make_inputs(wl.WORKLOADS[n]), None)
+                 for n in ("dual_bf16_decode", "rms_f32_4x128x1024", "ln_f32_1x1024x768")]
+
+    b = bench.cpu_baseline(FakeStep(), chunk_rows=256, single_share=4)
+    assert b["kind"] == "oracle" and b["cores"] >= 1 and b["value"] > 0
+    assert "(1576 rows" in b["sample"]  # 32 + 8 query/key head rows, 512, 1024
+    st = b["single_thread"]
+    assert st["cores"] == 1 and st["value"] > 0
+    # a quarter of each part's rows: 32/4 + 8/4 + 512/4 + 1024/4
+    assert "(394 rows)" in st["sample"]
