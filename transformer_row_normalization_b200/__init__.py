@@ -4,9 +4,11 @@ Thin Python binding over the C ABI of ``librownorm.so`` (declared in
 ``include/rownorm.h``). This module only marshals arguments: it turns torch
 CUDA tensors into ``rn_view`` descriptors (data pointer, rows, dim, row
 stride, dtype, and for head rows sliced out of a packed buffer the block
-layout), passes the current CUDA stream, and raises on a nonzero status. Every step of the computation runs in the library's CUDA kernels;
-there is no CPU or framework fallback, and calling with CPU tensors or
-without the built library raises.
+layout), passes the current CUDA stream, and raises on a nonzero status.
+Every step of the computation runs in the library's CUDA kernels; there is
+no CPU or framework fallback, and calling with CPU tensors or without the
+built library raises. Calls are asynchronous on the stream and may be
+captured in CUDA graphs.
 
     rn_rms_norm(x, weight, eps, out=None)               RMSNorm
     rn_layer_norm(x, weight, bias, eps, out=None)       LayerNorm
