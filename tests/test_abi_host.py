@@ -210,6 +210,44 @@ def test_cpu_tensors_are_rejected_loudly():
         rn.rms_norm(x, None, 1e-6)
 
 
+class _OnDevice:
+    """Stands in for a CUDA tensor: the binding's device check reads only
+    is_cuda and device, and raises before any other use."""
+
+    is_cuda = True
+
+    def __init__(self, index):
+        import torch
+        self.device = torch.device("cuda", index)
+
+
+class _Stream:
+    def __init__(self, index):
+        import torch
+        self.device = torch.device("cuda", index)
+
+
+@pytest.mark.parametrize("call", [
+    lambda a, b: rn.rms_norm(a, b, 1e-6),
+    lambda a, b: rn.rms_norm(a, None, 1e-6, out=b),
+    lambda a, b: rn.layer_norm(a, None, b, 1e-5),
+    lambda a, b: rn.dual_head_rms_norm(a, b, a, a, 1e-6),
+    lambda a, b: rn.dual_head_rms_norm(a, a, a, a, 1e-6, out_k=b),
+    lambda a, b: rn.add_rms_norm(a, b, None, 1e-6),
+    lambda a, b: rn.add_rms_norm(a, a, None, 1e-6, out_h=b),
+    lambda a, b: rn.gated_rms_norm(a, b, None, 1e-6),
+    lambda a, b: rn.dual_head_rms_norm_rope(a, a, a, a, 1e-6, b, 0, 8),
+])
+def test_tensors_on_another_device_are_rejected(call):
+    with pytest.raises(TypeError, match="one device"):
+        call(_OnDevice(0), _OnDevice(1))
+
+
+def test_stream_on_another_device_is_rejected():
+    with pytest.raises(TypeError, match="stream"):
+        rn.rms_norm(_OnDevice(0), None, 1e-6, stream=_Stream(1))
+
+
 def add_rms(lib, x, r, y, h, w=None, eps=1e-6):
     return lib.rn_add_rms_norm(ctypes.byref(x), ctypes.byref(r) if r is not None else None, w,
                                eps, ctypes.byref(y), ctypes.byref(h) if h is not None else None,

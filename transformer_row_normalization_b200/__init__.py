@@ -202,10 +202,25 @@ def _dtype_code(t):
     raise TypeError(f"row normalization supports float32 and bfloat16, not {t.dtype}")
 
 
-def _require_cuda(*tensors):
+def _require_cuda(*tensors, stream=None):
+    """Every tensor argument lives on one CUDA device, that of the first (the
+    input the kernel is launched for), and so does a caller's stream. The
+    kernels dereference every pointer on that device, so a tensor on another
+    GPU would be read through a peer mapping or fault; it is rejected here,
+    before anything is launched."""
+    device = None
     for t in tensors:
-        if t is not None and not t.is_cuda:
+        if t is None:
+            continue
+        if not t.is_cuda:
             raise TypeError("tensors must live on a CUDA device: this library has no CPU path")
+        if device is None:
+            device = t.device
+        elif t.device != device:
+            raise TypeError(f"all tensors of a call must be on one device: {t.device} is not "
+                            f"{device}")
+    if stream is not None and device is not None and stream.device != device:
+        raise TypeError(f"stream is on {stream.device}, the tensors on {device}")
 
 
 def _view(t):
@@ -233,7 +248,7 @@ def _stream(t, stream):
 def rn_rms_norm(x, weight, eps=1e-6, out=None, stream=None):
     """RMSNorm over the last axis of the CUDA tensor ``x``; returns ``out``."""
     import torch
-    _require_cuda(x, weight, out)
+    _require_cuda(x, weight, out, stream=stream)
     out = torch.empty_like(x) if out is None else out
     xv, yv = _view(x), _view(out)
     lib = load_library()
@@ -246,7 +261,7 @@ def rn_rms_norm(x, weight, eps=1e-6, out=None, stream=None):
 def rn_layer_norm(x, weight, bias, eps=1e-5, out=None, stream=None):
     """LayerNorm over the last axis of the CUDA tensor ``x``; returns ``out``."""
     import torch
-    _require_cuda(x, weight, bias, out)
+    _require_cuda(x, weight, bias, out, stream=stream)
     out = torch.empty_like(x) if out is None else out
     xv, yv = _view(x), _view(out)
     lib = load_library()
@@ -260,7 +275,7 @@ def rn_layer_norm(x, weight, bias, eps=1e-5, out=None, stream=None):
 def rn_dual_head_rms_norm(q, k, wq, wk, eps=1e-6, out_q=None, out_k=None, stream=None):
     """(RMSNorm(q, wq), RMSNorm(k, wk)) from one kernel launch; queries first."""
     import torch
-    _require_cuda(q, k, wq, wk, out_q, out_k)
+    _require_cuda(q, k, wq, wk, out_q, out_k, stream=stream)
     out_q = torch.empty_like(q) if out_q is None else out_q
     out_k = torch.empty_like(k) if out_k is None else out_k
     qv, kv, yqv, ykv = _view(q), _view(k), _view(out_q), _view(out_k)
@@ -278,7 +293,7 @@ def rn_add_rms_norm(x, residual, weight, eps=1e-6, out=None, out_h=None, stream=
     """(y, h): h = x + residual stored in x's dtype, y = RMSNorm(h) * weight, in
     one pass. ``out_h`` may be ``x`` or ``residual`` (in-place residual stream)."""
     import torch
-    _require_cuda(x, residual, weight, out, out_h)
+    _require_cuda(x, residual, weight, out, out_h, stream=stream)
     out = torch.empty_like(x) if out is None else out
     out_h = torch.empty_like(x) if out_h is None else out_h
     xv, rv, yv, hv = _view(x), _view(residual), _view(out), _view(out_h)
@@ -293,7 +308,7 @@ def rn_add_rms_norm(x, residual, weight, eps=1e-6, out=None, out_h=None, stream=
 def rn_gated_rms_norm(x, z, weight, eps=1e-6, out=None, stream=None):
     """RMSNorm(x) * weight * silu(z) over the last axis, in one pass."""
     import torch
-    _require_cuda(x, z, weight, out)
+    _require_cuda(x, z, weight, out, stream=stream)
     out = torch.empty_like(x) if out is None else out
     xv, zv, yv = _view(x), _view(z), _view(out)
     lib = load_library()
@@ -329,7 +344,7 @@ def rn_dual_head_rms_norm_rope(q, k, wq, wk, eps, table, offset, dims, heads_q=N
     q [tokens, heads_q, D] and k [tokens, heads_k, Dk] (or 2-D head rows with
     the head counts given); ``table`` is a CUDA float32 rope_table."""
     import torch
-    _require_cuda(q, k, wq, wk, table, out_q, out_k)
+    _require_cuda(q, k, wq, wk, table, out_q, out_k, stream=stream)
     if heads_q is None:
         heads_q = q.shape[-2] if q.dim() >= 3 else 1
     if heads_k is None:

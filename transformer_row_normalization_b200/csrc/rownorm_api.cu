@@ -2,6 +2,7 @@
 // The operations and conventions are documented in include/rownorm.h.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdint>
@@ -18,8 +19,10 @@
 namespace {
 
 thread_local char g_last_error[512] = "";
-int g_grid_override = 0;
-int g_path_override = 0;  // 0 automatic, 1 register, 2 staged, 3 register + prefetch
+// Testing controls, process-wide: set by rn_set_grid_override /
+// rn_set_path_override from any thread while other threads plan launches.
+std::atomic<int> g_grid_override{0};
+std::atomic<int> g_path_override{0};  // 0 automatic, 1 register, 2 staged, 3 register + prefetch
 
 int fail(int status, const char* fmt, ...) {
   va_list ap;
@@ -400,7 +403,8 @@ bool plan_staged(int dtype, int op, const SegPlan* plans, const rn_view* const* 
   // HBM bandwidth than this staged pipeline at every shape tried (the staged
   // kernel keeps more bytes in flight but runs fewer warps per SM and pays a
   // block barrier per tile). The staged kernel stays selectable.
-  if (g_path_override != 2 || rn::op_has_second(op)) return false;
+  if (g_path_override.load(std::memory_order_relaxed) != 2 || rn::op_has_second(op))
+    return false;
   const int es = elem_size(dtype);
   const bool wide = plans[0].family == 1;
   if (plans[0].family == 2) return false;  // rows wider than the register kernels hold
@@ -464,7 +468,7 @@ bool plan_staged(int dtype, int op, const SegPlan* plans, const rn_view* const* 
   int64_t grid = (int64_t)sms * bps;
   if (wide && grid >= plans[0].phase_period) grid -= grid % plans[0].phase_period;
   if (needed < grid) grid = needed;
-  if (g_grid_override > 0) grid = g_grid_override;
+  if (const int go = g_grid_override.load(std::memory_order_relaxed)) grid = go;
   rn_launch_info& in = l.info;
   in.family = plans[0].family;
   in.threads_per_row = plans[0].lanes;
@@ -524,9 +528,9 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
   // flight); blocks of 128 threads already keep 8+ rows per SM in flight and
   // ran slower with it. Only when the slots fit beside the weight cache
   // (with a margin for the kernel's static shared memory).
+  const int path = g_path_override.load(std::memory_order_relaxed);
   const bool want_prefetch =
-      g_path_override == 3 ||
-      (g_path_override == 0 && (merged.family == 0 || merged.lanes >= 256));
+      path == 3 || (path == 0 && (merged.family == 0 || merged.lanes >= 256));
   const int prefetch =
       !stream && want_prefetch && cache + pf_bytes <= device_info(dev).smem_per_block - 1024
           ? 1
@@ -562,7 +566,7 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
     grid -= grid % plans[0].phase_period;
   }
   if (needed < grid) grid = needed;
-  if (g_grid_override > 0) grid = g_grid_override;
+  if (const int go = g_grid_override.load(std::memory_order_relaxed)) grid = go;
   out->fn = fn;
   out->smem = smem;
   out->prefetch = prefetch;
@@ -973,13 +977,13 @@ RN_API int rn_plan(int op, const rn_view* x, const rn_view* y, const rn_view* x2
 
 RN_API int rn_set_grid_override(int blocks) {
   if (blocks < 0) return fail(RN_ERR_SHAPE, "grid override must be >= 0");
-  g_grid_override = blocks;
+  g_grid_override.store(blocks, std::memory_order_relaxed);
   return RN_OK;
 }
 
 RN_API int rn_set_path_override(int path) {
   if (path < 0 || path > 3) return fail(RN_ERR_SHAPE, "path override must be 0, 1, 2 or 3");
-  g_path_override = path;
+  g_path_override.store(path, std::memory_order_relaxed);
   return RN_OK;
 }
 

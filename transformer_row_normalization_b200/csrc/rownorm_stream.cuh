@@ -194,6 +194,11 @@ __global__ void __launch_bounds__(NT, 1024 / NT) rows_stream_kernel(const Params
     const Row<T> g = row_geometry<T, EXACT>(s, r);
     const bool has_edge = !EXACT && tid < g.nedge;
     float xe = load_edge<T, EXACT>(g, D, tid);
+    // LayerNorm shift K = x_0, read once before any pass: with y == x the
+    // store pass overwrites column 0, so the row must not be read from
+    // global memory again once the final reduction is done.
+    const float K = OP == kOpLn ? Elem<T>::get(g.x_row) : 0.f;
+    const F2 K2 = splat(K);
     float rstd, mean = 0.f;
     if constexpr (OP == kOpRms) {
       F2 acc = zero2();
@@ -205,8 +210,6 @@ __global__ void __launch_bounds__(NT, 1024 / NT) rows_stream_kernel(const Params
       if (has_edge) part = __fmaf_rn(xe, xe, part);
       rstd = rsqrtf(__fadd_rn(__fmul_rn(reduce(part), inv_d), p.eps));
     } else {
-      const float K = Elem<T>::get(g.x_row);
-      const F2 K2 = splat(K);
       F2 acc = zero2();
       stream_pass<T, NT>(g, tid, [&](F2 (&v)[P]) {
 #pragma unroll
@@ -237,7 +240,6 @@ __global__ void __launch_bounds__(NT, 1024 / NT) rows_stream_kernel(const Params
     // last pass: normalize, weight (and bias), store
     const F2 R2 = splat(rstd);
     const F2 M2 = splat(mean);
-    const F2 K2 = splat(OP == kOpLn ? Elem<T>::get(g.x_row) : 0.f);  // LayerNorm shift
     if constexpr (EXACT) {
       stream_store<T, OP, true, NT, kVecAligned>(s, g, tid, R2, M2, K2);
     } else {
