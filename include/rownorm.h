@@ -291,10 +291,11 @@ typedef struct rn_launch_info {
                             /* aligned and dim fills whole 16-byte chunks;  */
                             /* 2 as 1, and those chunks divide evenly over  */
                             /* the row's threads (no slot is ever empty)    */
-    int32_t staged;         /* 1: rows stream through shared memory by bulk */
-                            /* copies (S stages); 0: loaded into registers  */
-    int32_t stages;         /* staged: stages per block                     */
-    int32_t stage_bytes;    /* staged: bytes per stage                      */
+    int32_t staged;         /* 1: rows come through per-warp rings in      */
+                            /* shared memory filled by bulk copies (S      */
+                            /* stages per warp); 0: per-thread loads       */
+    int32_t stages;         /* staged: stages per warp                      */
+    int32_t stage_bytes;    /* staged: bytes per stage (a tile of rows)     */
 } rn_launch_info;
 
 enum { RN_OP_RMS = 0, RN_OP_LN = 1, RN_OP_DUAL = 2, RN_OP_ADD_RMS = 3, RN_OP_GATED_RMS = 4 };
@@ -313,22 +314,38 @@ RN_API int rn_plan(int op, const rn_view *x, const rn_view *y,
 
 /* Testing control: launch exactly `blocks` blocks (> 0) instead of the
  * automatic persistent grid; 0 restores the automatic choice. Results do not
- * depend on it (rows are statically strided over blocks). Process-wide. */
+ * depend on it (rows are statically strided over blocks). A test hook: it
+ * applies to every thread of the process (an atomic setting). */
 RN_API int rn_set_grid_override(int blocks);
 
 /* Kernel choice: 0 automatic; 1 register-resident kernels loading rows
- * directly; 2 the bulk-copy staged kernels (rows streamed through shared
- * memory) wherever the shape allows; 3 register-resident kernels with a
- * per-thread prefetch of the rows ahead through shared memory (cp.async),
- * also where the planner would not prefetch. The per-row
- * arithmetic is identical in every kind of kernel, so results do not depend
- * on it. Process-wide; meant for tests and measurements. */
+ * directly; 2 the per-warp bulk-copy rings (rows of up to 1024 columns in
+ * 16-byte aligned layouts come through a ring of shared-memory stages per
+ * warp, filled with cp.async.bulk) wherever the shape allows, the register
+ * kernels elsewhere; 3 register-resident kernels with a per-thread prefetch
+ * of the rows ahead through shared memory (cp.async), also where the planner
+ * would not prefetch. The per-row arithmetic is identical in every kind of
+ * kernel, so results do not depend on it. A test hook for tests and
+ * measurements: it applies to every thread of the process (an atomic
+ * setting). */
 RN_API int rn_set_path_override(int path);
 
-/* Number of stage waits in the staged kernels that gave up after their time
- * limit (each makes its block stop early, so a nonzero count means some
- * outputs were not written). Reading synchronizes the current device; reset
- * != 0 clears the counter. Needs a GPU. */
+/* Testing control for the ring kernels' bounded waits: with on = 1 every
+ * ring launch announces 16 bytes more per stage than its copies bring, so no
+ * stage ever completes; each warp (or block) gives up its first wait after
+ * 1 ms, waits at most 2 ms per stage for its copies (which all land), counts
+ * the timeout (rn_device_error_count) and stops, leaving its outputs
+ * unwritten. Nothing faults and the CUDA context stays usable. on = 0
+ * restores the normal limits (2 s per wait). A test hook: it applies to
+ * every thread of the process (an atomic setting). Returns RN_OK, or
+ * RN_ERR_SHAPE for another value. */
+RN_API int rn_set_ring_wait_test(int on);
+
+/* Number of stage waits in the ring kernels that gave up after their time
+ * limit (2 s). Each makes its warp stop early, after waiting for the bulk
+ * copies it still has in flight, so a nonzero count means some outputs were
+ * not written. Reading synchronizes the current device; reset != 0 clears
+ * the counter. Needs a GPU. */
 RN_API int rn_device_error_count(unsigned int *count, int reset);
 
 #ifdef __cplusplus

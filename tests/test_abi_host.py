@@ -178,6 +178,9 @@ def test_testing_controls(lib):
     assert lib.rn_set_grid_override(0) == 0
     assert lib.rn_set_path_override(4) == 2
     assert lib.rn_set_path_override(0) == 0
+    assert lib.rn_set_ring_wait_test(2) == 2
+    assert lib.rn_set_ring_wait_test(-1) == 2
+    assert lib.rn_set_ring_wait_test(0) == 0
     assert lib.rn_device_error_count(None, 0) == 1
 
 

@@ -106,3 +106,30 @@ def test_cpu_baseline_times_all_cores_and_one_thread():
     assert st["cores"] == 1 and st["value"] > 0
     # a quarter of each part's rows: 32/4 + 8/4 + 512/4 + 1024/4
     assert "(394 rows)" in st["sample"]
+
+
+@pytest.mark.parametrize("chunks", [1, 3, 8])
+def test_e2e_chunks_cover_every_row_once(chunks):
+    """The end-to-end pipeline's row chunks (host tensors here) tile each
+    workload exactly: every row in one chunk, outputs beside their inputs,
+    the dual workload cut by whole tokens."""
+    from transformer_row_normalization_b200 import workloads as wl
+    for name in ("dual_bf16_decode", "rms_f32_4x128x1024", "ln_f32_1x1024x768"):
+        w = wl.WORKLOADS[name]
+        a = wl.make_inputs(w)
+        out = ((torch.empty_like(a["q"]), torch.empty_like(a["k"])) if w.op == "dual"
+               else (torch.empty_like(a["x"]),))
+        parts = bench.chunk_views(w, a, out, chunks)
+        assert 1 <= len(parts) <= chunks
+        for ins, outs in parts:
+            assert len(ins) == len(outs)
+            for i, o in zip(ins, outs):
+                assert i.shape == o.shape
+        if w.op == "dual":
+            assert sum(p[0][0].shape[0] for p in parts) == a["q"].shape[0]
+            assert torch.equal(torch.cat([p[0][1] for p in parts]), a["k"])
+        else:
+            got = torch.cat([p[0][0] for p in parts])
+            assert torch.equal(got, a["x"].reshape(-1, w.dim))
+            ptrs = [p[1][0].data_ptr() for p in parts]
+            assert ptrs == sorted(ptrs) and ptrs[0] == out[0].data_ptr()

@@ -76,8 +76,21 @@ PATH_CASES = [
 ]
 
 
+def ring_applies(dtype, dim, offset):
+    """Under rn_set_path_override(2) the rings carry every RMSNorm and
+    LayerNorm row the register kernels hold, except lane-group rows
+    (dim <= 1024) off the 16-byte grid: per-warp rings take lane-group rows
+    whose rows all start on the grid with whole 16-byte chunks, block rings
+    every wider row."""
+    v = 8 if dtype == torch.bfloat16 else 4
+    widest = 32768 if dtype == torch.bfloat16 else 16384
+    if dim > 1024:
+        return dim <= widest
+    return dim % v == 0 and offset == 0
+
+
 @pytest.mark.parametrize("dtype,rows,dim,offset", PATH_CASES)
-def test_register_and_staged_kernels_agree_bitwise(dtype, rows, dim, offset):
+def test_register_and_ring_kernels_agree_bitwise(dtype, rows, dim, offset):
     big = wl.random_rows(rows, dim + offset, dtype, seed=dim, mean=0.5, std=2.0).cuda()
     x = big[:, offset:offset + dim] if offset else big
     w = wl.random_vector(dim, dtype, seed=1).cuda()
@@ -91,13 +104,14 @@ def test_register_and_staged_kernels_agree_bitwise(dtype, rows, dim, offset):
     finally:
         rn.set_path_override(0)
     assert out[1][2] == 0 and out[3][2] == 0
+    assert out[2][2] == int(ring_applies(dtype, dim, offset))
     for path in (2, 3):
         assert torch.equal(out[1][0], out[path][0]), path
         assert torch.equal(out[1][1], out[path][1]), path
     assert rn.device_error_count(reset=True) == 0
 
 
-def test_staged_dual_agrees_with_register_dual():
+def test_ring_dual_agrees_with_register_dual():
     q = wl.random_rows(8192 * 4, 128, torch.bfloat16, seed=9).cuda()
     k = wl.random_rows(8192, 128, torch.bfloat16, seed=10).cuda()
     wq = wl.random_vector(128, torch.bfloat16, seed=11).cuda()
@@ -106,6 +120,7 @@ def test_staged_dual_agrees_with_register_dual():
     try:
         for path in (1, 2):
             rn.set_path_override(path)
+            assert rn.plan(rn.RN_OP_DUAL, q, weight=wq, bias=wk, k=k)["staged"] == path - 1
             res[path] = rn.dual_head_rms_norm(q, k, wq, wk, 1e-6)
     finally:
         rn.set_path_override(0)
@@ -113,17 +128,99 @@ def test_staged_dual_agrees_with_register_dual():
     assert rn.device_error_count(reset=True) == 0
 
 
-def test_staged_plans_for_the_large_workloads():
+@pytest.mark.parametrize("rows", [1, 2, 3, 31, 33, 597, 4096 + 3])
+@pytest.mark.parametrize("dtype,dim", [(torch.bfloat16, 768), (torch.bfloat16, 1000),
+                                       (torch.bfloat16, 128), (torch.float32, 1024),
+                                       (torch.float32, 300)])
+def test_ring_ragged_row_counts(rows, dtype, dim):
+    """Row counts that leave partial tiles, warps without tiles and a ragged
+    last round of lane groups give the register kernels' bits."""
+    x = wl.random_rows(rows, dim, dtype, seed=rows + dim, mean=0.5, std=2.0).cuda()
+    w = wl.random_vector(dim, dtype, seed=3).cuda()
+    b = wl.random_vector(dim, dtype, seed=4, mean=0.0, std=0.1).cuda()
+    res = {}
     try:
-        for dim in (4096, 8192, 16384, 4097):
-            x = torch.empty(65536, dim, dtype=torch.bfloat16, device="cuda")
-            assert rn.plan(rn.RN_OP_LN, x)["staged"] == 0  # default: register kernels
-            rn.set_path_override(2)
-            p = rn.plan(rn.RN_OP_LN, x)
-            rn.set_path_override(0)
-            assert p["staged"] == 1 and p["stages"] >= 2, (dim, p)
+        for path in (1, 2):
+            rn.set_path_override(path)
+            res[path] = (rn.layer_norm(x, w, b, 1e-5), rn.rms_norm(x, None, 1e-6))
     finally:
         rn.set_path_override(0)
+    assert torch.equal(res[1][0], res[2][0]) and torch.equal(res[1][1], res[2][1])
+    assert rn.device_error_count(reset=True) == 0
+
+
+def test_ring_strided_and_block_views():
+    """Rows a stride apart (one copy per row) and head rows of a packed buffer
+    through the rings, against the register kernels."""
+    buf = wl.random_rows(3000, 1024 + 256, torch.bfloat16, seed=77, mean=0.5, std=2.0).cuda()
+    x = buf[:, 256:256 + 768]                       # stride 1280, rows 16-byte aligned
+    heads = buf.view(3000, 10, 128)[:, 2:8, :]      # 6 head rows per token, in blocks
+    w = wl.random_vector(768, torch.bfloat16, seed=5).cuda()
+    wh = wl.random_vector(128, torch.bfloat16, seed=6).cuda()
+    res = {}
+    try:
+        for path in (1, 2):
+            rn.set_path_override(path)
+            assert rn.plan(rn.RN_OP_RMS, x, weight=w)["staged"] == path - 1
+            res[path] = (rn.rms_norm(x, w, 1e-6), rn.rms_norm(heads, wh, 1e-6))
+    finally:
+        rn.set_path_override(0)
+    assert torch.equal(res[1][0], res[2][0]) and torch.equal(res[1][1], res[2][1])
+    assert rn.device_error_count(reset=True) == 0
+
+
+@pytest.mark.parametrize("dim", [768, 4097])
+def test_ring_waits_run_out_and_the_context_survives(dim):
+    """Under the wait test no ring stage completes: every warp (D = 768, warp
+    rings) or block (D = 4097, block rings) gives up its first wait, waits
+    for its copies, counts one timeout and stops without writing. The next
+    normal launch gives the register kernels' bits, with no timeout."""
+    rows = 4096
+    x = wl.random_rows(rows, dim, torch.bfloat16, seed=dim, mean=0.5, std=2.0).cuda()
+    w = wl.random_vector(dim, torch.bfloat16, seed=1).cuda()
+    b = wl.random_vector(dim, torch.bfloat16, seed=2, mean=0.0, std=0.1).cuda()
+    try:
+        rn.set_path_override(1)
+        ref = rn.layer_norm(x, w, b, 1e-5)
+        rn.set_path_override(2)
+        p = rn.plan(rn.RN_OP_LN, x, weight=w, bias=b)
+        assert p["staged"] == 1, p
+        rn.device_error_count(reset=True)
+        rn.set_ring_wait_test(True)
+        y = torch.full_like(x, float("nan"))
+        rn.layer_norm(x, w, b, 1e-5, out=y)
+        torch.cuda.synchronize()
+        rn.set_ring_wait_test(False)
+        if p["family"] == 0:  # a warp ring per warp, tiles of stage_bytes
+            tiles = -(-rows // (p["stage_bytes"] // (2 * dim)))
+            expect = min(p["grid_blocks"] * p["block_threads"] // 32, tiles)
+        else:                 # a block ring per block, one row per stage
+            expect = min(p["grid_blocks"], rows)
+        assert rn.device_error_count(reset=True) == expect
+        assert bool(torch.isnan(y).all())  # no stage completed, nothing written
+        y2 = rn.layer_norm(x, w, b, 1e-5)
+        torch.cuda.synchronize()
+        assert torch.equal(y2, ref)
+        assert rn.device_error_count(reset=True) == 0
+    finally:
+        rn.set_ring_wait_test(False)
+        rn.set_path_override(0)
+
+
+def test_ring_plans_for_the_large_workloads():
+    """By default the rings carry the aligned lane-group rows that fill a warp
+    (the narrow LayerNorm widths); wider rows and head rows keep the register
+    kernels unless the rings are forced."""
+    for dim, ring in ((768, 1), (1000, 1), (4096, 0), (8192, 0), (16384, 0), (4097, 0)):
+        x = torch.empty(65536, dim, dtype=torch.bfloat16, device="cuda")
+        p = rn.plan(rn.RN_OP_LN, x)
+        assert p["staged"] == ring, (dim, p)
+        if ring:
+            assert p["stages"] >= 2 and p["stage_bytes"] >= 2 * dim, p
+    q = torch.empty(8192 * 32, 128, dtype=torch.bfloat16, device="cuda")
+    k = torch.empty(8192 * 8, 128, dtype=torch.bfloat16, device="cuda")
+    w = torch.ones(128, dtype=torch.bfloat16, device="cuda")
+    assert rn.plan(rn.RN_OP_DUAL, q, weight=w, bias=w, k=k)["staged"] == 0
 
 
 @pytest.mark.parametrize("dim,layout", [(128, 2), (768, 2), (1000, 1), (1024, 2), (4096, 2),

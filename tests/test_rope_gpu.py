@@ -1,7 +1,7 @@
 """Parity of the dual q/k head RMSNorm + RoPE ("Emily.Fast", rope/3 and
 rope_with_freqs/4, after the dual head norm of "norm_fusion.rs") with the fp64
 oracle, through the C ABI: plane layouts, partial rotary, offsets, decode,
-frequency tables, misaligned views, full size; and its bits against the
+frequency tables, misaligned views, every token at full size; and its bits against the
 unrotated dual head norm where the rotation is the identity."""
 import numpy as np
 import pytest
@@ -10,6 +10,7 @@ import torch
 import oracle
 import transformer_row_normalization_b200 as rn
 from transformer_row_normalization_b200 import workloads as wl
+from fullsize import each_chunk
 from tolerance import check, guarded_empty
 
 pytestmark = pytest.mark.gpu
@@ -105,23 +106,25 @@ def test_identity_rotation_matches_the_dual_head_norm():
 
 
 def test_full_size_prefill():
+    """Every token of the 8192-token prefill (all its 32 query and 8 key
+    heads) against the oracle, in chunks of whole tokens at their positions."""
     w = wl.WORKLOADS["dual_rope_bf16_prefill"]
     a = wl.make_inputs(w, device="cuda")
     table = rn.rope_table(128, 8192, base=w.meta["rope_base"], device="cuda")
     yq, yk = rn.dual_head_rms_norm_rope(a["q"], a["k"], a["wq"], a["wk"], w.eps, table, 0, 128)
     torch.cuda.synchronize()
     q, k = a["q"].reshape(-1, 128), a["k"].reshape(-1, 128)
-    yq, yk = yq.reshape(-1, 128), yk.reshape(-1, 128)
-    assert bool(torch.isfinite(yq).all()) and bool(torch.isfinite(yk).all())
-    g = np.random.default_rng(64)
-    # whole tokens (all their heads), sampled over the positions
-    toks = sorted({0, 1, 8191, *(int(t) for t in g.choice(8192, 24, replace=False))})
-    for t in toks:
-        rq, rk = oracle.dual_head_rms_norm_rope(host(q[t * 32:(t + 1) * 32]),
-                                                host(k[t * 8:(t + 1) * 8]), host(a["wq"]),
-                                                host(a["wk"]), w.eps, 32, 8, t, 128)
-        check(yq[t * 32:(t + 1) * 32], rq, w.dtype, what=f"token {t} q", rope=(128, False))
-        check(yk[t * 8:(t + 1) * 8], rk, w.dtype, what=f"token {t} k", rope=(128, False))
+    hq, hk, hwq, hwk = host(q), host(k), host(a["wq"]), host(a["wk"])
+    hyq, hyk = host(yq.reshape(-1, 128)), host(yk.reshape(-1, 128))
+
+    def part(t0, t1):
+        rq, rk = oracle.dual_head_rms_norm_rope(hq[t0 * 32:t1 * 32], hk[t0 * 8:t1 * 8], hwq, hwk,
+                                                w.eps, 32, 8, t0, 128)
+        check(hyq[t0 * 32:t1 * 32], rq, w.dtype, what=f"tokens {t0}:{t1} q", rope=(128, False))
+        check(hyk[t0 * 8:t1 * 8], rk, w.dtype, what=f"tokens {t0}:{t1} k", rope=(128, False))
+
+    # a token is 40 head rows of 128 columns
+    assert each_chunk(8192, 40 * 128, part) == 8192
 
 
 def test_bitwise_repeatable_across_grids():

@@ -10,6 +10,7 @@ import torch
 import oracle
 import transformer_row_normalization_b200 as rn
 from transformer_row_normalization_b200 import workloads as wl
+from fullsize import each_chunk
 from tolerance import check, guarded_empty
 
 pytestmark = pytest.mark.gpu
@@ -135,6 +136,7 @@ def test_wide_in_place_and_grids():
 
 @pytest.mark.parametrize("name", [n for n in wl.FUSED_SUITE if wl.WORKLOADS[n].op in ("rms", "ln")])
 def test_full_size_streaming(name):
+    """Every row of the streamed benchmark workloads against the oracle."""
     w_ = wl.WORKLOADS[name]
     a = wl.make_inputs(w_, device="cuda")
     x = a["x"].reshape(-1, w_.dim)
@@ -143,13 +145,17 @@ def test_full_size_streaming(name):
     else:
         y = rn.rms_norm(x, a["w"], w_.eps)
     torch.cuda.synchronize()
-    assert bool(torch.isfinite(y).all())
-    g = np.random.default_rng(w_.seed)
-    idx = sorted({0, w_.rows - 1, *(int(i) for i in g.choice(w_.rows, 14, replace=False))})
-    idx = torch.tensor(idx)
-    xs = host(x)[idx]
-    if w_.op == "ln":
-        check(y[idx.cuda()], oracle.layer_norm(xs, host(a["w"]), host(a["b"]), w_.eps), w_.dtype,
-              bias=a["b"], what=name)
-    else:
-        check(y[idx.cuda()], oracle.rms_norm(xs, host(a["w"]), w_.eps), w_.dtype, what=name)
+    hx, hy, hw = host(x), host(y), host(a["w"])
+    hb = host(a["b"]) if w_.op == "ln" else None
+    del x, y, a
+    torch.cuda.empty_cache()
+
+    def part(r0, r1):
+        if w_.op == "ln":
+            check(hy[r0:r1], oracle.layer_norm(hx[r0:r1], hw, hb, w_.eps), w_.dtype, bias=hb,
+                  what=f"{name} rows {r0}:{r1}")
+        else:
+            check(hy[r0:r1], oracle.rms_norm(hx[r0:r1], hw, w_.eps), w_.dtype,
+                  what=f"{name} rows {r0}:{r1}")
+
+    assert each_chunk(w_.rows, w_.dim, part) == w_.rows

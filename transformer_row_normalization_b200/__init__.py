@@ -29,7 +29,7 @@ __all__ = [
     "rn_dual_head_rms_norm_rope", "rn_add_rms_norm", "rn_gated_rms_norm", "rope_table",
     "rms_norm", "layer_norm", "dual_head_rms_norm", "dual_head_rms_norm_rope",
     "add_rms_norm", "gated_rms_norm", "plan", "set_grid_override",
-    "set_path_override", "device_error_count",
+    "set_path_override", "set_ring_wait_test", "device_error_count",
     "library_path", "load_library", "view_params", "view_layout",
 ]
 
@@ -101,6 +101,7 @@ def load_library():
         lib.rn_set_grid_override.argtypes = [ctypes.c_int]
         lib.rn_set_path_override.argtypes = [ctypes.c_int]
         lib.rn_device_error_count.argtypes = [ctypes.POINTER(ctypes.c_uint), ctypes.c_int]
+        lib.rn_set_ring_wait_test.argtypes = [ctypes.c_int]
         lib.rn_status_string.argtypes = [ctypes.c_int]
         lib.rn_status_string.restype = ctypes.c_char_p
         lib.rn_last_error.argtypes = []
@@ -109,7 +110,8 @@ def load_library():
                    lib.rn_add_rms_norm, lib.rn_gated_rms_norm, lib.rn_plan,
                    lib.rn_dual_head_rms_norm_rope, lib.rn_rope_table,
                    lib.rn_set_grid_override, lib.rn_abi_version,
-                   lib.rn_set_path_override, lib.rn_device_error_count):
+                   lib.rn_set_path_override, lib.rn_device_error_count,
+                   lib.rn_set_ring_wait_test):
             fn.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -412,12 +414,19 @@ def set_grid_override(blocks: int):
 
 
 def set_path_override(path: int):
-    """Testing control: 0 automatic, 1 register kernels, 2 staged kernels."""
+    """Testing control: 0 automatic, 1 register kernels, 2 per-warp bulk-copy
+    rings where they apply, 3 register kernels with per-thread prefetch."""
     _check(load_library().rn_set_path_override(int(path)))
 
 
+def set_ring_wait_test(on: bool):
+    """Testing control: ring stages never complete, so their bounded waits
+    run out (1 ms) and the timeout path runs; False restores the limits."""
+    _check(load_library().rn_set_ring_wait_test(int(bool(on))))
+
+
 def device_error_count(reset: bool = False) -> int:
-    """Stage waits that timed out in the staged kernels (synchronizes)."""
+    """Stage waits that timed out in the ring kernels (synchronizes)."""
     n = ctypes.c_uint(0)
     _check(load_library().rn_device_error_count(ctypes.byref(n), int(reset)))
     return n.value

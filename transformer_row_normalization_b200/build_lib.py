@@ -1,7 +1,8 @@
 """Build librownorm.so (the C-ABI CUDA library) in-tree for sm_100a.
 
-Each translation unit compiles in its own nvcc process (they are independent
-kernel instantiation tables), then everything links into one shared library
+The kernel instantiation tables are generated into the build directory
+(csrc/gen_instantiations.py), each translation unit compiles in its own nvcc
+process (the tables are independent), then everything links into one shared library
 with the CUDA runtime linked statically and only the ``rn_*`` entry points of
 ``include/rownorm.h`` exported.
 """
@@ -18,11 +19,12 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "librownorm.so")
 
-SOURCES = ["rownorm_api.cu", "rownorm_warp_f32.cu", "rownorm_warp_bf16.cu",
-           "rownorm_cta_f32.cu", "rownorm_cta_bf16.cu", "rownorm_staged_f32.cu",
-           "rownorm_staged_bf16.cu", "rownorm_stream.cu"]
-HEADERS = ["rownorm_core.cuh", "rownorm_kernels.cuh", "rownorm_staged.cuh", "rownorm_launch.h",
-           "rownorm_stream.cuh"]
+# hand-written translation units; the kernel instantiation tables are
+# generated into the build directory by csrc/gen_instantiations.py
+SOURCES = ["rownorm_api.cu", "rownorm_stream.cu"]
+HEADERS = ["rownorm_core.cuh", "rownorm_kernels.cuh", "rownorm_ring.cuh", "rownorm_launch.h",
+           "rownorm_stream.cuh", "gen_instantiations.py"]
+GEN = os.path.join(BUILD, "gen")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
@@ -44,8 +46,9 @@ def _newest_input() -> float:
 
 
 def _compile(src: str, extra) -> str:
-    obj = os.path.join(BUILD, os.path.splitext(src)[0] + ".o")
-    cmd = [nvcc()] + CFLAGS + list(extra) + ["-c", os.path.join(CSRC, src), "-o", obj]
+    obj = os.path.join(BUILD, os.path.splitext(os.path.basename(src))[0] + ".o")
+    path = src if os.path.isabs(src) else os.path.join(CSRC, src)
+    cmd = [nvcc()] + CFLAGS + list(extra) + ["-c", path, "-o", obj]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError(f"nvcc failed on {src}:\n{res.stdout}\n{res.stderr}")
@@ -58,10 +61,16 @@ def build(force: bool = False, verbose_ptxas: bool = False, jobs: int = 0) -> st
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _newest_input():
         return LIB
     os.makedirs(BUILD, exist_ok=True)
+    sys.path.insert(0, CSRC)
+    try:
+        import gen_instantiations
+    finally:
+        sys.path.remove(CSRC)
+    units = SOURCES + gen_instantiations.write_tables(GEN)
     extra = ["-Xptxas", "-v"] if verbose_ptxas else []
-    jobs = jobs or min(len(SOURCES), os.cpu_count() or 1)
+    jobs = jobs or min(len(units), os.cpu_count() or 1)
     with cf.ThreadPoolExecutor(jobs) as ex:
-        results = list(ex.map(lambda s: _compile(s, extra), SOURCES))
+        results = list(ex.map(lambda s: _compile(s, extra), units))
     if verbose_ptxas:
         for _, log in results:
             sys.stderr.write(log)

@@ -14,7 +14,7 @@
 #include "rownorm.h"
 #include "rownorm_kernels.cuh"
 #include "rownorm_launch.h"
-#include "rownorm_staged.cuh"
+#include "rownorm_ring.cuh"
 
 namespace {
 
@@ -22,7 +22,8 @@ thread_local char g_last_error[512] = "";
 // Testing controls, process-wide: set by rn_set_grid_override /
 // rn_set_path_override from any thread while other threads plan launches.
 std::atomic<int> g_grid_override{0};
-std::atomic<int> g_path_override{0};  // 0 automatic, 1 register, 2 staged, 3 register + prefetch
+std::atomic<int> g_path_override{0};  // 0 automatic, 1 register, 2 ring, 3 register + prefetch
+std::atomic<int> g_ring_wait_test{0};  // 1: ring stages never complete (bounded-wait test)
 
 int fail(int status, const char* fmt, ...) {
   va_list ap;
@@ -379,107 +380,143 @@ struct Launch {
   const void* fn;
   int smem;
   int prefetch;     // register kernels: rows ahead prefetched through shared memory
-  int staged;       // 1: rows_staged_kernel with StagedParams
+  int ring;         // 1: rows_ring_kernel, 2: rows_cta_ring_kernel (RingParams)
   rn_launch_info info;
-  // staged kernels only
-  int stages, stage_bytes, tile_rows[2], contiguous[2], cache_offset;
-  int64_t tiles[2];
+  // ring kernels only
+  int stages, stage_bytes, tile_rows[2], contiguous[2];
   int stage_word;   // kOpRmsRope: staging rows after the slots and the cache
 };
 
-constexpr int kNarrowTileBytes = 16 * 1024;  // rows per stage ~ 16 KB (lane-group rows)
-constexpr int kMaxStages = 8;
+// Ring tiles: R rows of a lane-group segment per stage, about this many
+// bytes (at least one round of the warp's lane groups); S stages per warp.
+constexpr int kRingTileBytes = 2048;
+constexpr int kRingStages = 4;
 
 int round_up(int64_t v, int64_t m) { return (int)((v + m - 1) / m * m); }
 
-// Plans a bulk-copy staged launch (selected with rn_set_path_override(2))
-// when the shape qualifies: rows wider than the lane-group limit (one block
-// per row, any layout), or lane-group rows in an EXACT layout. Returns false
-// (and leaves the register-kernel plan in charge) otherwise.
-bool plan_staged(int dtype, int op, const SegPlan* plans, const rn_view* const* xs,
-                 const void* const* ws, const void* const* bs, int nseg, int dev, int sms,
-                 Launch* out) {
-  // The register kernels are the default: measured on B200 they sustain more
-  // HBM bandwidth than this staged pipeline at every shape tried (the staged
-  // kernel keeps more bytes in flight but runs fewer warps per SM and pays a
-  // block barrier per tile). The staged kernel stays selectable.
-  if (g_path_override.load(std::memory_order_relaxed) != 2 || rn::op_has_second(op))
-    return false;
-  const int es = elem_size(dtype);
-  const bool wide = plans[0].family == 1;
-  if (plans[0].family == 2) return false;  // rows wider than the register kernels hold
-  for (int i = 0; i < nseg; ++i) {
-    if (two_level(xs[i])) return false;  // tiles address rows with one stride
-    if (plans[i].family != plans[0].family) return false;
-    if (!wide && !plans[i].exact) return false;
-  }
-  int chunks = 0;
-  bool exact = true;
-  for (int i = 0; i < nseg; ++i) {
-    chunks = plans[i].chunks > chunks ? plans[i].chunks : chunks;
-    exact = exact && plans[i].exact;
-  }
-  const int threads = wide ? plans[0].lanes : 256;
-  const void* fn = dtype == RN_F32 ? rn::staged_kernel_f32(op, wide, exact, threads, chunks)
-                                   : rn::staged_kernel_bf16(op, wide, exact, threads, chunks);
+// Whether the planner uses the per-warp bulk-copy rings by default for these
+// segments (they must qualify, see plan_ring): rows whose lane groups fill a
+// whole warp, where the register kernels hold a row's chunks in registers
+// and their prefetch queue in shared memory per thread.
+bool ring_preferred(const SegPlan* plans, int nseg) {
+  for (int i = 0; i < nseg; ++i)
+    if (plans[i].lanes != 32) return false;
+  return true;
+}
+
+// Plans a ring launch for RMSNorm / LayerNorm segments of the lane-group
+// family in EXACT layouts: by default where ring_preferred says so, everywhere
+// it qualifies with rn_set_path_override(2), never with 1 or 3. Returns
+// false (the register-kernel plan stays in charge) otherwise.
+bool plan_ring(int dtype, int op, const SegPlan* plans, const rn_view* const* xs, int nseg,
+               int chunks, int slots, int dev, int sms, Launch* out) {
+  const int path = g_path_override.load(std::memory_order_relaxed);
+  if (path == 1 || path == 3) return false;
+  if (op != rn::kOpRms && op != rn::kOpLn && op != rn::kOpRmsRopeLocal) return false;
+  for (int i = 0; i < nseg; ++i)
+    if (plans[i].family != 0 || !plans[i].exact) return false;
+  if (path == 0 && !ring_preferred(plans, nseg)) return false;
+  const void* fn = dtype == RN_F32 ? rn::ring_kernel_f32(op, slots, chunks)
+                                   : rn::ring_kernel_bf16(op, slots, chunks);
   if (!fn) return false;
   Launch l{};
-  l.staged = 1;
-  int64_t stage_bytes = 0;
+  l.ring = 1;
+  const int es = elem_size(dtype);
+  int64_t stage_bytes = 16;
+  int64_t tiles_max = 1;
   for (int i = 0; i < nseg; ++i) {
     const int64_t row_bytes = xs[i]->dim * es;
-    int64_t tr = 1;
-    if (!wide) {
-      tr = kNarrowTileBytes / row_bytes;
-      if (tr < 1) tr = 1;
-      if (tr > xs[i]->rows) tr = xs[i]->rows > 0 ? xs[i]->rows : 1;
-    }
+    const int64_t per = 32 / plans[i].lanes;  // rows a warp takes at once
+    int64_t rounds = kRingTileBytes / (per * row_bytes);
+    if (rounds < 1) rounds = 1;
+    const int64_t tr = per * rounds;
     l.tile_rows[i] = (int)tr;
-    l.contiguous[i] = xs[i]->rows <= 1 || xs[i]->row_stride == xs[i]->dim;
-    l.tiles[i] = ceil_div(xs[i]->rows, tr);
-    const int64_t b = tr * row_bytes;
-    if (b > stage_bytes) stage_bytes = b;
+    l.contiguous[i] = !two_level(xs[i]) && (xs[i]->rows <= 1 || xs[i]->row_stride == xs[i]->dim);
+    const int64_t tiles = ceil_div(xs[i]->rows, tr);
+    if (tiles > tiles_max) tiles_max = tiles;
+    if (tr * row_bytes > stage_bytes) stage_bytes = tr * row_bytes;
   }
-  l.stage_bytes = round_up(stage_bytes, 128);
-  const int affine = exact ? 0 : rn::affine_cache_smem_bytes(op, threads, chunks);
+  l.stage_bytes = round_up(stage_bytes, 16);
   const DeviceInfo di = device_info(dev);
-  // blocks per SM: as many as leave each block its weight cache and four
-  // stages, at most 1024 threads per SM
-  const int64_t want = affine + 4LL * l.stage_bytes + 1024 + 512;
-  int blocks_target = (int)(di.smem_per_sm / want);
-  if (blocks_target > (threads >= 1024 ? 1 : 1024 / threads))
-    blocks_target = threads >= 1024 ? 1 : 1024 / threads;
-  if (blocks_target < 1) blocks_target = 1;
-  // per block: the SM's shared memory split over the target block count, less
-  // the 1 KB the hardware reserves per block and the kernel's static arrays
-  int64_t budget = di.smem_per_sm / blocks_target - 1024 - 512;
-  if (budget > di.smem_per_block - 512) budget = di.smem_per_block - 512;
-  int64_t stages = (budget - affine) / l.stage_bytes;
-  if (stages > kMaxStages) stages = kMaxStages;
-  if (stages < 2) return false;
-  l.stages = (int)stages;
-  l.cache_offset = (int)(stages * l.stage_bytes);
+  int stages = kRingStages;
+  while (stages > 2 && rn::ring_smem_bytes(stages, l.stage_bytes) > di.smem_per_block - 1024)
+    --stages;
+  if (rn::ring_smem_bytes(stages, l.stage_bytes) > di.smem_per_block - 1024) return false;
+  l.stages = stages;
   l.fn = fn;
-  l.smem = l.cache_offset + affine;
+  l.smem = rn::ring_smem_bytes(stages, l.stage_bytes);
   int bps = 0;
-  if (blocks_per_sm(dev, fn, threads, l.smem, &bps)) return false;
-  int64_t needed = 1;
-  for (int i = 0; i < nseg; ++i) needed = l.tiles[i] > needed ? l.tiles[i] : needed;
+  if (blocks_per_sm(dev, fn, rn::kRingWarps * 32, l.smem, &bps)) return false;
   int64_t grid = (int64_t)sms * bps;
-  if (wide && grid >= plans[0].phase_period) grid -= grid % plans[0].phase_period;
+  const int64_t needed = ceil_div(tiles_max, rn::kRingWarps);
   if (needed < grid) grid = needed;
   if (const int go = g_grid_override.load(std::memory_order_relaxed)) grid = go;
   rn_launch_info& in = l.info;
-  in.family = plans[0].family;
+  in.family = 0;
   in.threads_per_row = plans[0].lanes;
   in.chunks_per_thread = chunks;
   in.smem_bytes = l.smem;
-  in.block_threads = threads;
+  in.block_threads = rn::kRingWarps * 32;
   in.grid_blocks = (int32_t)grid;
   in.blocks_per_sm = bps;
   in.vector_y = plans[0].vector_y;
   in.phase_period = plans[0].phase_period;
-  in.exact = exact;
+  in.exact = slots == rn::kSlotsFull ? 2 : 1;
+  in.staged = 1;
+  in.stages = l.stages;
+  in.stage_bytes = l.stage_bytes;
+  *out = l;
+  return true;
+}
+
+// Whether the planner uses the block rings by default for this block-family
+// segment (it must qualify, see plan_cta_ring).
+bool cta_ring_preferred(const SegPlan& p) {
+  (void)p;
+  return false;
+}
+
+// Plans a block-ring launch for one RMSNorm / LayerNorm segment of the block
+// family (any layout): by default where cta_ring_preferred says so,
+// everywhere with rn_set_path_override(2), never with 1 or 3. Returns false
+// (the register-kernel plan stays in charge) otherwise.
+bool plan_cta_ring(int dtype, int op, const SegPlan* plans, const rn_view* const* xs, int nseg,
+                   int slots, int dev, int sms, Launch* out) {
+  const int path = g_path_override.load(std::memory_order_relaxed);
+  if (path == 1 || path == 3 || nseg != 1) return false;
+  if (op != rn::kOpRms && op != rn::kOpLn) return false;
+  const SegPlan& p = plans[0];
+  if (p.family != 1) return false;
+  if (path == 0 && !cta_ring_preferred(p)) return false;
+  const bool ex = p.exact != 0;
+  const void* fn = dtype == RN_F32 ? rn::cta_ring_kernel_f32(op, ex, slots, p.lanes, p.chunks)
+                                   : rn::cta_ring_kernel_bf16(op, ex, slots, p.lanes, p.chunks);
+  if (!fn) return false;
+  Launch l{};
+  l.ring = 2;
+  l.stages = rn::cta_ring_stages(p.lanes);
+  l.stage_bytes = round_up(p.nfull_max * 16 > 16 ? p.nfull_max * 16 : 16, 16);
+  const int cache = ex ? 0 : rn::affine_cache_smem_bytes(op, p.lanes, p.chunks);
+  l.smem = l.stages * l.stage_bytes + cache;
+  if (l.smem > device_info(dev).smem_per_block - 1024) return false;
+  l.fn = fn;
+  int bps = 0;
+  if (blocks_per_sm(dev, fn, p.lanes, l.smem, &bps)) return false;
+  int64_t grid = (int64_t)sms * bps;
+  if (grid >= p.phase_period) grid -= grid % p.phase_period;
+  if (xs[0]->rows < grid) grid = xs[0]->rows > 0 ? xs[0]->rows : 1;
+  if (const int go = g_grid_override.load(std::memory_order_relaxed)) grid = go;
+  rn_launch_info& in = l.info;
+  in.family = 1;
+  in.threads_per_row = p.lanes;
+  in.chunks_per_thread = p.chunks;
+  in.smem_bytes = l.smem;
+  in.block_threads = p.lanes;
+  in.grid_blocks = (int32_t)grid;
+  in.blocks_per_sm = bps;
+  in.vector_y = p.vector_y;
+  in.phase_period = p.phase_period;
+  in.exact = ex ? (slots == rn::kSlotsFull ? 2 : 1) : 0;
   in.staged = 1;
   in.stages = l.stages;
   in.stage_bytes = l.stage_bytes;
@@ -488,7 +525,8 @@ bool plan_staged(int dtype, int op, const SegPlan* plans, const rn_view* const* 
 }
 
 // Plans the launch for one or two segments that share one kernel: the
-// bulk-copy staged kernel where it applies, else the register kernels.
+// per-warp bulk-copy rings where they apply and are chosen, else the register
+// kernels.
 int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* xs,
                 const void* const* ws, const void* const* bs, int nseg, Launch* out) {
   int64_t rows[2] = {xs[0]->rows, nseg > 1 ? xs[1]->rows : 0};
@@ -512,7 +550,8 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
   int sms = 0, bps = 0;
   int st = device_sms(dev, &sms);
   if (st) return st;
-  if (plan_staged(dtype, op, plans, xs, ws, bs, nseg, dev, sms, out)) return RN_OK;
+  if (plan_ring(dtype, op, plans, xs, nseg, merged.chunks, slots, dev, sms, out)) return RN_OK;
+  if (plan_cta_ring(dtype, op, plans, xs, nseg, slots, dev, sms, out)) return RN_OK;
   const int threads = merged.family == 0 ? rn::kWarpBlock : merged.lanes;
   // the streaming kernels keep no weight cache and prefetch nothing
   const bool stream = merged.family == 2;
@@ -570,7 +609,7 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
   out->fn = fn;
   out->smem = smem;
   out->prefetch = prefetch;
-  out->staged = 0;
+  out->ring = 0;
   rn_launch_info& in = out->info;
   in.family = merged.family;
   in.threads_per_row = plans[0].lanes;
@@ -609,20 +648,22 @@ rn::Segment make_segment(const rn_view* x, const rn_view* y, const void* w, cons
 
 int launch(const Launch& l, const rn::Params& params, void* stream) {
   cudaError_t e;
-  if (l.staged) {
-    rn::StagedParams sp{};
+  if (l.ring) {
+    rn::RingParams rp{};
     for (int i = 0; i < 2; ++i) {
-      sp.seg[i] = params.seg[i];
-      sp.tile_rows[i] = l.tile_rows[i];
-      sp.contiguous[i] = l.contiguous[i];
-      sp.tiles[i] = i < params.nseg ? l.tiles[i] : 0;
+      rp.seg[i] = params.seg[i];
+      rp.tile_rows[i] = i < params.nseg ? l.tile_rows[i] : 1;
+      rp.contiguous[i] = l.contiguous[i];
     }
-    sp.nseg = params.nseg;
-    sp.eps = params.eps;
-    sp.stages = l.stages;
-    sp.stage_bytes = l.stage_bytes;
-    sp.cache_offset = l.cache_offset;
-    void* args[] = {&sp};
+    rp.nseg = params.nseg;
+    rp.eps = params.eps;
+    rp.stages = l.stages;
+    rp.stage_bytes = l.stage_bytes;
+    const bool wait_test = g_ring_wait_test.load(std::memory_order_relaxed) != 0;
+    rp.wait_ns = wait_test ? 1000000ull : rn::kRingWaitLimitNs;
+    rp.drain_ns = wait_test ? 2000000ull : rn::kRingDrainLimitNs;
+    rp.tx_extra = wait_test ? 16 : 0;
+    void* args[] = {&rp};
     e = cudaLaunchKernel(l.fn, dim3((unsigned)l.info.grid_blocks),
                          dim3((unsigned)l.info.block_threads), args, (size_t)l.smem,
                          static_cast<cudaStream_t>(stream));
@@ -987,14 +1028,23 @@ RN_API int rn_set_path_override(int path) {
   return RN_OK;
 }
 
+RN_API int rn_set_ring_wait_test(int on) {
+  if (on != 0 && on != 1) return fail(RN_ERR_SHAPE, "ring wait test must be 0 or 1");
+  g_ring_wait_test.store(on, std::memory_order_relaxed);
+  return RN_OK;
+}
+
 RN_API int rn_device_error_count(unsigned int* count, int reset) {
   if (!count) return fail(RN_ERR_NULL, "count is NULL");
   unsigned int a = 0, b = 0;
-  int e = rn::staged_timeouts_f32(&a, reset != 0);
-  if (e == 0) e = rn::staged_timeouts_bf16(&b, reset != 0);
+  unsigned int c = 0, d = 0;
+  int e = rn::ring_timeouts_f32(&a, reset != 0);
+  if (e == 0) e = rn::ring_timeouts_bf16(&b, reset != 0);
+  if (e == 0) e = rn::cta_ring_timeouts_f32(&c, reset != 0);
+  if (e == 0) e = rn::cta_ring_timeouts_bf16(&d, reset != 0);
   if (e != 0)
     return fail(RN_ERR_CUDA, "device error counter: %s", cudaGetErrorString((cudaError_t)e));
-  *count = a + b;
+  *count = a + b + c + d;
   return RN_OK;
 }
 

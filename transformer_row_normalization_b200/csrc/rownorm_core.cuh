@@ -408,9 +408,11 @@ __device__ __forceinline__ float shift_and_sum(F2 (&v)[NSLOT][Elem<T>::P], float
   return s;
 }
 
-// LayerNorm pass 2: the thread's sum of (d - mean)^2.
+// LayerNorm pass 2: replaces d by the centred c = d - mean (slots and edge
+// element; the normalization uses c as it is) and returns the thread's sum
+// of c^2.
 template <typename T, bool EXACT, int SLOTS, int NSLOT>
-__device__ __forceinline__ float sum_dev_squares(const F2 (&v)[NSLOT][Elem<T>::P], float xe,
+__device__ __forceinline__ float sum_dev_squares(F2 (&v)[NSLOT][Elem<T>::P], float& xe,
                                                  const Row<T>& g, int k0, int step, float mean,
                                                  bool has_edge) {
   constexpr int P = Elem<T>::P;
@@ -421,15 +423,15 @@ __device__ __forceinline__ float sum_dev_squares(const F2 (&v)[NSLOT][Elem<T>::P
     if (slot_present<SLOTS, NSLOT>(p, k0 + step * p, g.nfull)) {
 #pragma unroll
       for (int j = 0; j < P; ++j) {
-        const F2 t = sub2(v[p][j], M2);
-        acc = fma2(t, t, acc);
+        v[p][j] = sub2(v[p][j], M2);
+        acc = fma2(v[p][j], v[p][j], acc);
       }
     }
   }
   float s = hsum2(acc);
   if (!EXACT && has_edge) {
-    const float t = __fsub_rn(xe, mean);
-    s = __fmaf_rn(t, t, s);
+    xe = __fsub_rn(xe, mean);
+    s = __fmaf_rn(xe, xe, s);
   }
   return s;
 }
@@ -437,9 +439,12 @@ __device__ __forceinline__ float sum_dev_squares(const F2 (&v)[NSLOT][Elem<T>::P
 // ---------------------------------------------------------------------------
 // reductions across the threads of a row
 
-// xor butterfly over the G lanes of `mask` (G a power of two <= 32).
+// xor butterfly over the G lanes of `mask` (G a power of two <= 32): offsets
+// G/2, ..., 1, unrolled (G is uniform across the warp).
 __device__ __forceinline__ float group_sum(float x, int G, unsigned mask) {
-  for (int off = G >> 1; off > 0; off >>= 1) x = __fadd_rn(x, __shfl_xor_sync(mask, x, off));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1)
+    if (off < G) x = __fadd_rn(x, __shfl_xor_sync(mask, x, off));
   return x;
 }
 
@@ -596,7 +601,7 @@ __device__ __forceinline__ void normalize_store(const Segment& s, const Row<T>& 
   constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
   const F2 R2 = splat(rstd);
-  const F2 M2 = splat(mean);
+  (void)mean;  // LayerNorm rows arrive centred (row_stats)
 #pragma unroll
   for (int p = 0; p < NSLOT; ++p) {
     const int f = k0 + step * p;
@@ -605,8 +610,8 @@ __device__ __forceinline__ void normalize_store(const Segment& s, const Row<T>& 
     src.get(p, f, wf, bf);
 #pragma unroll
     for (int j = 0; j < P; ++j) {
-      if constexpr (OP == kOpLn)
-        o[j] = fma2(mul2(sub2(v[p][j], M2), R2), wf[j], bf[j]);
+      if constexpr (OP == kOpLn)  // v holds the centred c = d - mean
+        o[j] = fma2(mul2(v[p][j], R2), wf[j], bf[j]);
       else
         o[j] = mul2(mul2(v[p][j], R2), wf[j]);
     }
@@ -632,7 +637,7 @@ __device__ __forceinline__ void normalize_store(const Segment& s, const Row<T>& 
   if (!EXACT && has_edge) {
     float we, be;
     src.edge(we, be);
-    float o = OP == kOpLn ? __fmaf_rn(__fmul_rn(__fsub_rn(xe, mean), rstd), we, be)
+    float o = OP == kOpLn ? __fmaf_rn(__fmul_rn(xe, rstd), we, be)  // xe centred
                           : __fmul_rn(__fmul_rn(xe, rstd), we);
     if constexpr (OP == kOpGatedRms) o = __fmul_rn(o, silu(gate.edge()));
     Elem<T>::put(g.y_row + edge_column(g, s.dim, k0), o);
@@ -734,11 +739,12 @@ __device__ __forceinline__ void normalize_rope_store(const Segment& s, const Row
         F2 ya[P], yb[P];
 #pragma unroll
         for (int j = 0; j < P; ++j) {
+          // packed pairs of planes: y_a = fma(a, cos, -(b sin)), y_b = fma(b, cos, a sin)
           const F2 a = v[p][j], b = v[p + NSLOT / 2][j];
-          ya[j] = make2(__fmaf_rn(a.x, cs[2 * j], -__fmul_rn(b.x, sn[2 * j])),
-                        __fmaf_rn(a.y, cs[2 * j + 1], -__fmul_rn(b.y, sn[2 * j + 1])));
-          yb[j] = make2(__fmaf_rn(b.x, cs[2 * j], __fmul_rn(a.x, sn[2 * j])),
-                        __fmaf_rn(b.y, cs[2 * j + 1], __fmul_rn(a.y, sn[2 * j + 1])));
+          const F2 c = make2(cs[2 * j], cs[2 * j + 1]), sn2 = make2(sn[2 * j], sn[2 * j + 1]);
+          const F2 bs = mul2(b, sn2), as = mul2(a, sn2);
+          ya[j] = fma2(a, c, make2(-bs.x, -bs.y));
+          yb[j] = fma2(b, c, as);
         }
         store_chunk<T>(s, g.y_row + c0, ya, vstore);
         store_chunk<T>(s, g.y_row + c0 + half, yb, vstore);
@@ -772,9 +778,10 @@ __device__ __forceinline__ void normalize_rope_store(const Segment& s, const Row
         }
 #pragma unroll
         for (int j = 0; j < P; ++j) {
-          const float a = o[j].x, b = o[j].y;
-          o[j] = make2(__fmaf_rn(a, cs[j], -__fmul_rn(b, sn[j])),
-                       __fmaf_rn(b, cs[j], __fmul_rn(a, sn[j])));
+          // plane (a, b) = o[j]: (a cos - b sin, b cos + a sin) as one packed
+          // multiply of the swapped pair and one packed fused multiply-add
+          const F2 t = mul2(make2(o[j].y, o[j].x), splat(sn[j]));
+          o[j] = fma2(o[j], splat(cs[j]), make2(-t.x, t.y));
         }
       }
       store_chunk<T>(s, g.y_row + c0, o, vstore);
@@ -861,16 +868,19 @@ __device__ __forceinline__ void normalize_rope_store(const Segment& s, const Row
   __syncwarp(mask);
 }
 
+// Means are sums times 1/D rounded to binary32 (one multiply instead of a
+// divide per row; exact for power-of-two D, within 2 ulps otherwise).
+__device__ __forceinline__ float inv_dim(int D) { return __frcp_rn((float)D); }
+
 // rstd (and mean) of one row from the thread's slots and edge element, with
-// `reduce` summing a per-thread partial over the threads of the row.
+// `reduce` summing a per-thread partial over the threads of the row. For
+// LayerNorm the slots and edge element leave centred (x - K - mean).
+// inv_d is inv_dim(D), computed once per row space by the caller.
 template <typename T, int OP, bool EXACT, int SLOTS, int NSLOT, typename Reduce>
 __device__ __forceinline__ void row_stats(F2 (&v)[NSLOT][Elem<T>::P], float& xe,
-                                          const Row<T>& g, int D, int k0, int step, float K,
+                                          const Row<T>& g, float inv_d, int k0, int step, float K,
                                           float eps, bool has_edge, Reduce reduce, float& rstd,
                                           float& mean) {
-  // Means are sums times 1/D rounded to binary32 (one multiply instead of a
-  // divide per row; exact for power-of-two D, within 2 ulps otherwise).
-  const float inv_d = __frcp_rn((float)D);
   if (OP != kOpLn) {
     const float ss = reduce(sum_squares<T, EXACT, NSLOT>(v, xe, has_edge));
     mean = 0.f;

@@ -23,8 +23,8 @@
 // barrier. The shift K of each row ahead (LayerNorm) and the thread's edge
 // element of it are loaded into registers when its copies are issued.
 //
-// The bulk-copy staged kernels (rownorm_staged.cuh) run the same per-row
-// code; which kernel the planner picks never changes a bit.
+// The bulk-copy ring kernels (rownorm_ring.cuh) run the same per-row code;
+// which kernel the planner picks never changes a bit.
 #pragma once
 
 #include "rownorm_core.cuh"
@@ -199,6 +199,7 @@ __device__ __forceinline__ void segment_rows(const Segment& s, const Prefetch<T,
   constexpr bool SECOND = op_has_second(OP);
   constexpr bool LATE_REFILL = OP == kOpGatedRms;
   const int D = s.dim;
+  const float inv_d = inv_dim(D);
   float Kq[NST], Eq[NST], E2q[NST];
   // queue the loads of row ra into stage `stage`, its scalars at queue entry j
   auto ahead = [&](long long ra, int stage, int j) {
@@ -275,8 +276,8 @@ __device__ __forceinline__ void segment_rows(const Segment& s, const Prefetch<T,
       if constexpr (!LATE_REFILL) refill(r, st);
     }
     float rstd, mean;
-    row_stats<T, OP, EXACT, SLOTS, NSLOT>(v, xe, g, D, k0, step, K, eps, has_edge, reduce, rstd,
-                                          mean);
+    row_stats<T, OP, EXACT, SLOTS, NSLOT>(v, xe, g, inv_d, k0, step, K, eps, has_edge, reduce,
+                                          rstd, mean);
     if constexpr (!EXACT) {
       if (g.phase != src.phase) src.fill(s, g, k0, step);
     }

@@ -33,9 +33,7 @@ constexpr int cta_key(int op, bool exact, int slots, int threads, int chunks) {
   return (((op * 2 + (exact ? 1 : 0)) * 3 + slots) * 2048 + threads) * 8 + chunks;
 }
 
-constexpr int staged_key(int op, bool wide, bool exact, int threads, int chunks) {
-  return (((op * 2 + (wide ? 1 : 0)) * 2 + (exact ? 1 : 0)) * 2048 + threads) * 16 + chunks;
-}
+constexpr int ring_key(int op, int slots, int chunks) { return (op * 3 + slots) * 16 + chunks; }
 
 // Kernel entry for (op, exact, chunks per lane) in the warp family; nullptr
 // if that configuration is not compiled. op: 0 RMSNorm, 1 LayerNorm. exact:
@@ -47,8 +45,6 @@ const void* warp_kernel_bf16(int op, bool exact, int slots, int chunks);
 // block family; nullptr if not compiled.
 const void* cta_kernel_f32(int op, bool exact, int slots, int threads, int chunks);
 const void* cta_kernel_bf16(int op, bool exact, int slots, int threads, int chunks);
-// Bulk-copy staged kernels: wide (one block per row) or narrow (lane groups,
-// rows 16-byte aligned); nullptr if not compiled.
 // Streaming kernels (rows wider than the register kernels hold): RMSNorm
 // and LayerNorm, any layout.
 const void* stream_kernel(int dtype_f32, int op, bool exact, int threads);
@@ -58,11 +54,22 @@ constexpr int kStreamBlockThreads = 1024;
 constexpr int kStreamPairThreads = 512;
 constexpr long long kStreamPairMaxRowBytes = 192 * 1024;
 
-const void* staged_kernel_f32(int op, bool wide, bool exact, int threads, int chunks);
-const void* staged_kernel_bf16(int op, bool wide, bool exact, int threads, int chunks);
-// Timed-out stage waits recorded by the staged kernels of each element type
+// Per-warp bulk-copy ring kernels (lane-group rows, 16-byte aligned
+// layouts) for (op, slot policy, chunks per lane); op 0 RMSNorm, 1
+// LayerNorm, 5 RMSNorm + RoPE with in-thread planes; nullptr if not compiled.
+const void* ring_kernel_f32(int op, int slots, int chunks);
+const void* ring_kernel_bf16(int op, int slots, int chunks);
+// Block bulk-copy ring kernels (the block family's rows, any layout) for
+// (op, exact, slot policy, threads per block, chunks per thread), keyed like
+// the register block kernels; op 0 RMSNorm, 1 LayerNorm; nullptr if not
+// compiled.
+const void* cta_ring_kernel_f32(int op, bool exact, int slots, int threads, int chunks);
+const void* cta_ring_kernel_bf16(int op, bool exact, int slots, int threads, int chunks);
+// Timed-out stage waits recorded by the ring kernels of each table
 // (optionally resetting the counter); returns a cudaError_t value.
-int staged_timeouts_f32(unsigned int* count, bool reset);
-int staged_timeouts_bf16(unsigned int* count, bool reset);
+int ring_timeouts_f32(unsigned int* count, bool reset);
+int ring_timeouts_bf16(unsigned int* count, bool reset);
+int cta_ring_timeouts_f32(unsigned int* count, bool reset);
+int cta_ring_timeouts_bf16(unsigned int* count, bool reset);
 
 }  // namespace rn

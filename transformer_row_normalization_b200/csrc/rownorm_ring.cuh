@@ -1,0 +1,491 @@
+// Per-warp bulk-copy row rings (sm_100a), for rows whose lane groups fit in
+// one warp (dim <= 1024) in 16-byte aligned layouts: RMSNorm, LayerNorm, and
+// the q/k head RMSNorm + RoPE whose plane partners are the same thread's.
+//
+// Every warp of a block runs its own pipeline, with no block barrier: a ring
+// of S stages in shared memory, each holding one tile of R consecutive rows
+// of the warp's static share of the row space (tiles w, w + W, w + 2W, ...
+// for warp w of W). Lane 0 fills a stage with the bulk-copy engine
+// (cp.async.bulk global -> shared, completion counted in bytes on the
+// stage's mbarrier): one copy for a tile whose rows are adjacent in memory,
+// else one copy per row. The warp waits for the stage, its lane groups
+// normalize the tile's rows from shared memory and store them to global
+// memory, and lane 0 refills the stage with the tile S ahead. So S tiles of
+// every warp are in flight while it computes, independently of its register
+// budget, and a tile costs one copy instruction instead of one per 16-byte
+// chunk and lane.
+//
+// The per-row arithmetic is that of the register kernels (rownorm_core.cuh):
+// the same lanes per row, chunk-to-lane mapping, shift K = x_0, summation
+// order and operation order. Which kernel the planner picks never changes a
+// bit.
+//
+// Waits are bounded. A warp whose stage wait gives up after kRingWaitLimitNs
+// stops issuing, then waits for every copy it still has in flight (bounded
+// by kRingDrainLimitNs; the copies read valid memory and always complete),
+// records the timeout in the device counter (rn_device_error_count) and
+// returns. No warp leaves with a copy into its shared memory outstanding.
+// The wait test (rn_set_ring_wait_test) makes every stage announce 16 bytes
+// more than its copies bring, so that no stage completes: every first wait
+// runs out after a millisecond and the timeout path runs, with all copies
+// landed and nothing faulted.
+#pragma once
+
+#include <type_traits>
+
+#include "rownorm_kernels.cuh"
+
+namespace rn {
+
+// Timed-out stage waits. Each translation unit that instantiates the ring
+// kernels has its own counter (internal linkage) and a host accessor beside
+// its table.
+static __device__ unsigned int g_ring_timeouts;
+
+constexpr int kRingWarps = 4;        // warps (independent rings) per block
+constexpr int kRingMaxStages = 8;    // barrier slots reserved per warp
+constexpr unsigned long long kRingWaitLimitNs = 2000000000ull;    // 2 s
+constexpr unsigned long long kRingDrainLimitNs = 30000000000ull;  // 30 s
+
+struct RingParams {
+  Segment seg[2];
+  int nseg;
+  float eps;
+  int stages;          // S, 2 .. kRingMaxStages
+  int stage_bytes;     // bytes of one stage (the widest tile), a multiple of 16
+  int tile_rows[2];    // R per segment: a multiple of the rows a warp takes at once
+  int contiguous[2];   // 1: a tile's rows are adjacent in memory (one copy)
+  unsigned long long wait_ns;   // stage wait limit (normally kRingWaitLimitNs)
+  unsigned long long drain_ns;  // limit of the wait for copies in flight after a timeout
+  int tx_extra;        // bytes announced beyond the copies' (0; > 0 only under the
+                       // wait test, so that no stage completes and every wait runs out)
+};
+
+// Shared memory of a block: the warps' rings, then their barrier slots.
+__host__ __device__ constexpr int ring_smem_bytes(int stages, int stage_bytes) {
+  return kRingWarps * stages * stage_bytes + kRingWarps * kRingMaxStages * 8;
+}
+
+__device__ __forceinline__ unsigned long long global_timer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+
+// Makes the initialized barriers visible to the bulk-copy (async) proxy.
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Orders this thread's earlier shared-memory reads before bulk copies it
+// issues next into the same bytes.
+__device__ __forceinline__ void fence_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// The one arrival of a stage's phase, announcing the bytes its copies bring.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Wait for the phase of `bar` with the given parity to complete; false after
+// `limit_ns` without completion.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          unsigned long long limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_timer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer() - t0 > limit_ns) return false;
+  }
+  return true;
+}
+
+// Global -> shared bulk copy of `bytes` (both addresses 16-byte aligned, a
+// multiple of 16 bytes), completion counted on `bar`. No multicast.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Weight and bias of a lane's chunk slots held in registers as their packed
+// 16-byte words (loaded once per row space: in an aligned layout a lane owns
+// the same chunks of every row), unpacked at each use. NULL weight = ones,
+// NULL bias = zeros, as AffineDirect; the values, and so the bits, are the
+// same.
+template <typename T, bool BIAS, int NSLOT>
+struct AffineRegs {
+  uint4 w[NSLOT];
+  uint4 b[BIAS ? NSLOT : 1];
+  __device__ __forceinline__ void load(const Segment& s, int k0, int step) {
+    constexpr int V = Elem<T>::V;
+    const T* wv = static_cast<const T*>(s.w);
+    const T* bv = static_cast<const T*>(s.b);
+    const uint32_t one = Elem<T>::kOneBits | (sizeof(T) == 2 ? Elem<T>::kOneBits << 16 : 0u);
+    const int nfull = s.dim / V;
+#pragma unroll
+    for (int p = 0; p < NSLOT; ++p) {
+      const int f = k0 + step * p;
+      const bool in = f < nfull;
+      w[p] = (wv && in) ? load_cached(wv + f * V) : make_uint4(one, one, one, one);
+      if constexpr (BIAS) b[p] = (bv && in) ? load_cached(bv + f * V) : make_uint4(0, 0, 0, 0);
+    }
+  }
+  __device__ __forceinline__ void get(int p, int /*f*/, F2 (&wf)[Elem<T>::P],
+                                      F2 (&bf)[Elem<T>::P]) const {
+    Elem<T>::unpack(w[p], wf);
+    if constexpr (BIAS) Elem<T>::unpack(b[p], bf);
+  }
+  __device__ __forceinline__ void edge(float& w_, float& b_) const {
+    w_ = 1.f;
+    b_ = 0.f;
+  }
+};
+
+// Lane 0: start the copies of tile `tile` of row space s (R rows per tile)
+// into `dst`, counted on `bar`.
+template <typename T>
+__device__ __forceinline__ void ring_issue(const Segment& s, long long tile, int R,
+                                           bool contiguous, int tx_extra, unsigned char* dst,
+                                           uint64_t* bar) {
+  const long long r0 = tile * R;
+  const long long nr = s.rows - r0 < R ? s.rows - r0 : R;
+  const uint32_t row_bytes = (uint32_t)s.dim * (uint32_t)sizeof(T);
+  const T* x = static_cast<const T*>(s.x);
+  mbar_expect_tx(bar, (uint32_t)nr * row_bytes + (uint32_t)tx_extra);
+  if (contiguous) {
+    bulk_load(dst, x + row_off(r0, s.x_stride, s.x_inner, s.x_outer), (uint32_t)nr * row_bytes,
+              bar);
+  } else {
+    for (long long rr = 0; rr < nr; ++rr)
+      bulk_load(dst + rr * row_bytes, x + row_off(r0 + rr, s.x_stride, s.x_inner, s.x_outer),
+                row_bytes, bar);
+  }
+}
+
+// The rows of one staged tile (rows r0 .. r0 + nr - 1), normalized by the
+// warp's lane groups: lane group gi takes rows gi, gi + 32/G, ...
+template <typename T, int OP, int SLOTS, int VPL, typename Src>
+__device__ __forceinline__ void ring_tile_rows(const Segment& s, const unsigned char* stage,
+                                               long long r0, int nr, float eps, float inv_d,
+                                               int gl, int gi, unsigned mask, const Src& src) {
+  constexpr int P = Elem<T>::P;
+  const int G = s.lanes;
+  auto reduce = [&](float t) { return group_sum(t, G, mask); };
+  const int row_bytes = s.dim * (int)sizeof(T);
+#pragma unroll 1
+  for (int rr = gi; rr < nr; rr += 32 / G) {
+    const Row<T> g = row_geometry<T, true>(s, r0 + rr);
+    const uint4* row = reinterpret_cast<const uint4*>(stage + rr * row_bytes);
+    F2 v[VPL][P];
+#pragma unroll
+    for (int q = 0; q < VPL; ++q) {
+      if (slot_present<SLOTS, VPL>(q, gl + G * q, g.nfull)) {
+        Elem<T>::unpack(row[gl + G * q], v[q]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < P; ++j) v[q][j] = zero2();
+      }
+    }
+    const float K = OP == kOpLn ? Elem<T>::get(reinterpret_cast<const T*>(row)) : 0.f;
+    float xe = 0.f, rstd, mean;
+    row_stats<T, OP, true, SLOTS, VPL>(v, xe, g, inv_d, gl, G, K, eps, false, reduce, rstd,
+                                       mean);
+    if constexpr (OP == kOpRmsRopeLocal)
+      normalize_rope_store<T, true, true, SLOTS, VPL>(s, g, v, xe, src, gl, G, rstd, false,
+                                                      r0 + rr, nullptr, mask);
+    else
+      normalize_store<T, OP, true, SLOTS, VPL>(s, g, v, xe, src, gl, G, rstd, mean, false);
+  }
+}
+
+// Weight and bias in registers (AffineRegs) for lanes of up to 3 chunks when
+// the op needs no other per-element tables; otherwise read from L1 per row
+// (AffineDirect). Beyond that, the values held across the row spill under
+// the 128-register budget (ptxas).
+template <int OP, int VPL>
+__host__ __device__ constexpr bool ring_weights_in_regs() {
+  return OP != kOpRmsRopeLocal && VPL <= 3;
+}
+
+// Register budget: 4 blocks of kRingWarps warps per SM (16 warps, up to 128
+// registers). The rows in flight sit in the rings, not in registers, so more
+// warps buy nothing; measured on B200 (LayerNorm bf16 65536 x 768), a budget
+// of 80 registers spilled and ran 10 % slower.
+constexpr int kRingBlocksPerSm = 4;
+
+template <typename T, int OP, int SLOTS, int VPL>
+__global__ void __launch_bounds__(kRingWarps * 32, kRingBlocksPerSm)
+rows_ring_kernel(const RingParams p) {
+  static_assert(OP == kOpRms || OP == kOpLn || OP == kOpRmsRopeLocal,
+                "rings carry RMSNorm and LayerNorm rows, and head rows rotated in-thread");
+  constexpr bool BIAS = OP == kOpLn;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int S = p.stages;
+  unsigned char* const smem = reinterpret_cast<unsigned char*>(dyn_smem);
+  unsigned char* const ring = smem + warp * S * p.stage_bytes;
+  uint64_t* const bars =
+      reinterpret_cast<uint64_t*>(smem + kRingWarps * S * p.stage_bytes) + warp * kRingMaxStages;
+  const long long w = (long long)blockIdx.x * kRingWarps + warp;
+  const long long W = (long long)gridDim.x * kRingWarps;
+  if (lane == 0) {
+    for (int k = 0; k < S; ++k) mbar_init(&bars[k], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  // The stages are used round robin across the row spaces; bit k of
+  // `parity` is the phase parity with which stage k completes next.
+  uint32_t parity = 0;
+  int st = 0;
+  bool ok = true;
+#pragma unroll 1
+  for (int si = 0; si < p.nseg && ok; ++si) {
+    const Segment s = pick_segment(p.seg, si);
+    const int R = si ? p.tile_rows[1] : p.tile_rows[0];
+    const bool contiguous = (si ? p.contiguous[1] : p.contiguous[0]) != 0;
+    const long long ntiles = (s.rows + R - 1) / R;
+    const long long n = ntiles > w ? (ntiles - w + W - 1) / W : 0;  // this warp's tiles
+    if (n == 0) continue;
+    const int G = s.lanes;
+    const int gl = lane & (G - 1);
+    const int gi = lane / G;
+    const unsigned mask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << (gi * G));
+    const float inv_d = inv_dim(s.dim);
+    using Regs = AffineRegs<T, BIAS, VPL>;
+    using Direct = AffineDirect<T, BIAS, false>;
+    std::conditional_t<ring_weights_in_regs<OP, VPL>(), Regs, Direct> src;
+    if constexpr (ring_weights_in_regs<OP, VPL>())
+      src.load(s, gl, G);
+    else
+      src = Direct{static_cast<const T*>(s.w), static_cast<const T*>(s.b)};
+    // every stage is free here: the previous row space's tiles are consumed
+    if (lane == 0) {
+      int k = st;
+      for (long long i = 0; i < n && i < S; ++i) {
+        ring_issue<T>(s, w + i * W, R, contiguous, p.tx_extra, ring + k * p.stage_bytes,
+                      &bars[k]);
+        k = k + 1 == S ? 0 : k + 1;
+      }
+    }
+    __syncwarp();
+    long long i = 0;
+#pragma unroll 1
+    for (; i < n; ++i) {
+      ok = mbar_wait(&bars[st], (parity >> st) & 1u, p.wait_ns);
+      if (__any_sync(0xffffffffu, !ok)) {
+        ok = false;
+        break;
+      }
+      parity ^= 1u << st;
+      const long long r0 = (w + i * W) * R;
+      const int nr = (int)(s.rows - r0 < R ? s.rows - r0 : R);
+      ring_tile_rows<T, OP, SLOTS, VPL>(s, ring + st * p.stage_bytes, r0, nr, p.eps, inv_d, gl,
+                                        gi, mask, src);
+      // every lane has read the stage: refill it with the tile S ahead
+      __syncwarp();
+      if (lane == 0 && i + S < n) {
+        fence_async_shared();
+        ring_issue<T>(s, w + (i + S) * W, R, contiguous, p.tx_extra, ring + st * p.stage_bytes,
+                      &bars[st]);
+      }
+      st = st + 1 == S ? 0 : st + 1;
+    }
+    if (!ok && lane == 0) {
+      // tiles i .. min(n, i + S) - 1 are issued and not yet consumed, in
+      // stages st, st + 1, ... (mod S)
+      int k = st;
+      for (long long j = i; j < n && j < i + S; ++j) {
+        mbar_wait(&bars[k], (parity >> k) & 1u, p.drain_ns);
+        k = k + 1 == S ? 0 : k + 1;
+      }
+      atomicAdd(&g_ring_timeouts, 1u);
+    }
+  }
+}
+
+}  // namespace rn
+
+namespace rn {
+
+// ---------------------------------------------------------------------------
+// Block rings: rows wider than one warp's lane groups hold (the block
+// family, one block of NT threads per row). Thread 0 fills a ring of NST
+// stages, each holding the full 16-byte chunks of one row (one bulk copy:
+// they are contiguous and 16-byte aligned whatever the row's phase); every
+// thread waits for the stage of its current row, reads its chunks from it,
+// and the row is reduced and stored as in rows_cta_kernel (same threads per
+// row, chunk ownership, edge elements, shift, summation and operation
+// order: the same bits). The stage of row i is refilled with row i + NST at
+// the start of row i + 1, when every thread has passed row i's reduction
+// barriers and so has read it; NST - 1 rows are in flight while one is
+// normalized. Each thread's edge element and the shift K of the rows ahead
+// are loaded into register queues when their copies are issued.
+
+template <typename T, bool EXACT>
+__device__ __forceinline__ void cta_ring_issue(const Segment& s, long long r, unsigned char* dst,
+                                               uint64_t* bar, int tx_extra) {
+  const Row<T> g = row_geometry<T, EXACT>(s, r);
+  const uint32_t bytes = (uint32_t)g.nfull * 16u;
+  mbar_expect_tx(bar, bytes + (uint32_t)tx_extra);
+  if (bytes) bulk_load(dst, g.x_full, bytes, bar);
+}
+
+template <typename T, int OP, bool EXACT, int SLOTS, int NT, int VPT, int NST, typename Src>
+__device__ __forceinline__ void cta_ring_rows(const RingParams& p, const Segment& s,
+                                              unsigned char* ring, uint64_t* bars, Src& src,
+                                              float (*red)[NT / 32], bool& ok) {
+  constexpr int P = Elem<T>::P;
+  const int tid = threadIdx.x;
+  const int D = s.dim;
+  const float inv_d = inv_dim(D);
+  const long long stride = gridDim.x;
+  const long long r0 = blockIdx.x;
+  int slot = 0;
+  auto reduce = [&](float t) {
+    const float v = block_sum<NT>(t, red[slot]);
+    slot ^= 1;
+    return v;
+  };
+  float Kq[NST], Eq[NST];
+  // thread 0 starts the copies; every thread queues its scalars of the row
+  auto ahead = [&](long long ra, int st, int j) {
+    const Row<T> ga = row_geometry<T, EXACT>(s, ra);
+    if (tid == 0)
+      cta_ring_issue<T, EXACT>(s, ra, ring + (long long)st * p.stage_bytes, &bars[st], p.tx_extra);
+    Kq[j] = OP == kOpLn ? Elem<T>::get(ga.x_row) : 0.f;
+    Eq[j] = load_edge<T, EXACT>(ga, D, tid);
+  };
+#pragma unroll
+  for (int j = 0; j < NST; ++j) {
+    Kq[j] = 0.f;
+    Eq[j] = 0.f;
+    const long long rj = r0 + j * stride;
+    if (rj < s.rows) ahead(rj, j, j);
+  }
+  long long i = 0;
+  int st = 0;           // stage of row i: i % NST
+  uint32_t parity = 0;  // phase parity of row i: (i / NST) & 1
+#pragma unroll 1
+  for (long long r = r0; r < s.rows; r += stride, ++i) {
+    if (i > 0) {
+      // every thread has passed row i - 1's reduction barriers: its stage
+      // is free for row i - 1 + NST
+      const long long ra = r + (NST - 1) * stride;
+      const int rs = st == 0 ? NST - 1 : st - 1;
+      if (tid == 0) fence_async_shared();
+      if (ra < s.rows) ahead(ra, rs, NST - 1);
+    }
+    const float K = Kq[0];
+    float xe = Eq[0];
+#pragma unroll
+    for (int j = 0; j + 1 < NST; ++j) {
+      Kq[j] = Kq[j + 1];
+      Eq[j] = Eq[j + 1];
+    }
+    const bool done = mbar_wait(&bars[st], parity, p.wait_ns);
+    if (__syncthreads_or(!done)) {
+      ok = false;
+      if (tid == 0) {
+        // rows i .. i + NST - 1 are issued and not yet consumed; row j sits
+        // in stage (st + j - i) mod NST, one phase later once it wraps
+        for (int j = 0; j < NST && r + j * stride < s.rows; ++j) {
+          const int k = st + j;
+          mbar_wait(&bars[k < NST ? k : k - NST], k < NST ? parity : parity ^ 1u, p.drain_ns);
+        }
+        atomicAdd(&g_ring_timeouts, 1u);
+      }
+      return;
+    }
+    const Row<T> g = row_geometry<T, EXACT>(s, r);
+    const bool has_edge = !EXACT && tid < g.nedge;
+    const uint4* stage = reinterpret_cast<const uint4*>(ring + (long long)st * p.stage_bytes);
+    F2 v[VPT][P];
+#pragma unroll
+    for (int q = 0; q < VPT; ++q) {
+      if (slot_present<SLOTS, VPT>(q, tid + NT * q, g.nfull)) {
+        Elem<T>::unpack(stage[tid + NT * q], v[q]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < P; ++j) v[q][j] = zero2();
+      }
+    }
+    float rstd, mean;
+    row_stats<T, OP, EXACT, SLOTS, VPT>(v, xe, g, inv_d, tid, NT, K, p.eps, has_edge, reduce,
+                                        rstd, mean);
+    if constexpr (!EXACT) {
+      if (g.phase != src.phase) src.fill(s, g, tid, NT);
+    }
+    normalize_store<T, OP, EXACT, SLOTS, VPT>(s, g, v, xe, src, tid, NT, rstd, mean, has_edge);
+    if (++st == NST) {
+      st = 0;
+      parity ^= 1u;
+    }
+  }
+}
+
+// Rows in flight per block ring: NST - 1 while one is normalized.
+__host__ __device__ constexpr int cta_ring_stages(int threads) { return threads >= 512 ? 2 : 3; }
+
+// Register budget: the rows ahead wait in the ring, not in registers, so
+// blocks of up to 256 threads take 80 registers (768 threads per SM) rather
+// than spill at 64; wider blocks keep 1024 threads per SM.
+__host__ __device__ constexpr int cta_ring_min_blocks(int threads) {
+  return threads >= 512 ? kMinThreadsPerSm / threads : 768 / threads;
+}
+
+template <typename T, int OP, bool EXACT, int SLOTS, int NT, int VPT>
+__global__ void __launch_bounds__(NT, cta_ring_min_blocks(NT))
+rows_cta_ring_kernel(const RingParams p) {
+  static_assert(OP == kOpRms || OP == kOpLn, "block rings carry RMSNorm and LayerNorm rows");
+  static_assert(NT >= 2 * (Elem<T>::V - 1), "every edge element needs its own thread");
+  constexpr int NST = cta_ring_stages(NT);
+  constexpr bool BIAS = OP == kOpLn;
+  __shared__ float red[2][NT / 32];
+  __shared__ __align__(8) uint64_t bars[NST];
+  unsigned char* const ring = reinterpret_cast<unsigned char*>(dyn_smem);
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < NST; ++st) mbar_init(&bars[st], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const Segment& s = p.seg[0];
+  bool ok = true;
+  const T* w = static_cast<const T*>(s.w);
+  const T* b = static_cast<const T*>(s.b);
+  if constexpr (EXACT) {
+    if (w && (!BIAS || b)) {
+      AffineDirect<T, BIAS, true> src{w, b};
+      cta_ring_rows<T, OP, true, SLOTS, NT, VPT, NST>(p, s, ring, bars, src, red, ok);
+    } else {
+      AffineDirect<T, BIAS, false> src{w, b};
+      cta_ring_rows<T, OP, true, SLOTS, NT, VPT, NST>(p, s, ring, bars, src, red, ok);
+    }
+  } else {
+    AffineCache<T, VPT, BIAS> src;
+    src.init(NST * p.stage_bytes / 16);
+    cta_ring_rows<T, OP, false, SLOTS, NT, VPT, NST>(p, s, ring, bars, src, red, ok);
+  }
+}
+
+}  // namespace rn
