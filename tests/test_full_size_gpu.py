@@ -31,7 +31,9 @@ def test_full_size_single(name):
     # the default plan: the kernel bench.py times
     plan = rn.plan(rn.RN_OP_LN if w.op == "ln" else rn.RN_OP_RMS, x, weight=a["w"],
                    bias=a.get("b"))
-    assert plan["staged"] == (1 if w.dim in (768, 1000) else 0), plan
+    # rings by default: warp rings for rows one warp's lanes share (768,
+    # 1000), block rings for blocks of 512+ threads (16384)
+    assert plan["staged"] == (1 if w.dim in (768, 1000, 16384) else 0), plan
     if w.op == "ln":
         y = rn.layer_norm(a["x"], a["w"], a["b"], w.eps).reshape(-1, w.dim)
     else:

@@ -389,19 +389,28 @@ struct Launch {
 
 // Ring tiles: R rows of a lane-group segment per stage, about this many
 // bytes (at least one round of the warp's lane groups); S stages per warp.
-constexpr int kRingTileBytes = 2048;
+#ifndef RN_RING_TILE_BYTES
+#define RN_RING_TILE_BYTES 2048
+#endif
+constexpr int kRingTileBytes = RN_RING_TILE_BYTES;
 constexpr int kRingStages = 4;
 
 int round_up(int64_t v, int64_t m) { return (int)((v + m - 1) / m * m); }
 
 // Whether the planner uses the per-warp bulk-copy rings by default for these
-// segments (they must qualify, see plan_ring): rows whose lane groups fill a
-// whole warp, where the register kernels hold a row's chunks in registers
-// and their prefetch queue in shared memory per thread.
-bool ring_preferred(const SegPlan* plans, int nseg) {
-  for (int i = 0; i < nseg; ++i)
-    if (plans[i].lanes != 32) return false;
-  return true;
+// segments (they must qualify, see plan_ring). Measured on B200 against the
+// register lane-group kernels (65536 rows, cold L2, medians):
+//   bf16 rows whose lane groups fill a warp: LayerNorm 768 47.9 -> 38.9 us,
+//     1000 73.8 -> 53.3 us, RMSNorm 1024 51.1 -> 45.0 us;
+//   the bf16 dual head norm (q [8192, 32, 128] and k [8192, 8, 128], 4 lanes
+//     per row): 32.8 -> 30.7 us;
+//   but bf16 LayerNorm 512 (16 lanes per row) 31.8 -> 34.7 us and binary32
+//   LayerNorm 1024 88.1 -> 94.1 us ran slower, and stay on the register
+//   kernels.
+bool ring_preferred(int dtype, const SegPlan* plans, int nseg) {
+  if (dtype != RN_BF16) return false;
+  if (nseg == 2) return true;
+  return plans[0].lanes == 32;
 }
 
 // Plans a ring launch for RMSNorm / LayerNorm segments of the lane-group
@@ -415,7 +424,7 @@ bool plan_ring(int dtype, int op, const SegPlan* plans, const rn_view* const* xs
   if (op != rn::kOpRms && op != rn::kOpLn && op != rn::kOpRmsRopeLocal) return false;
   for (int i = 0; i < nseg; ++i)
     if (plans[i].family != 0 || !plans[i].exact) return false;
-  if (path == 0 && !ring_preferred(plans, nseg)) return false;
+  if (path == 0 && !ring_preferred(dtype, plans, nseg)) return false;
   const void* fn = dtype == RN_F32 ? rn::ring_kernel_f32(op, slots, chunks)
                                    : rn::ring_kernel_bf16(op, slots, chunks);
   if (!fn) return false;
@@ -470,11 +479,15 @@ bool plan_ring(int dtype, int op, const SegPlan* plans, const rn_view* const* xs
 }
 
 // Whether the planner uses the block rings by default for this block-family
-// segment (it must qualify, see plan_cta_ring).
-bool cta_ring_preferred(const SegPlan& p) {
-  (void)p;
-  return false;
-}
+// segment (it must qualify, see plan_cta_ring): blocks of 512 or more
+// threads, which run two or fewer rows per SM at a time. Measured on B200
+// (bf16 LayerNorm, 65536 rows, cold): D = 16384 (512 threads) 760.6 ->
+// 722.9 us; at D = 8192 (256 threads) the register kernel with per-thread
+// prefetch stayed ahead (352.5 against 374.8 us), and at 4097 (128 threads)
+// too (204.9 against 222.2 us).
+bool cta_ring_preferred(const SegPlan& p) { return p.lanes >= 512; }
+// (Measured again after the rings' register trim: D = 16384 768.9 -> 698.2 us,
+// the same before and after a full bench run.)
 
 // Plans a block-ring launch for one RMSNorm / LayerNorm segment of the block
 // family (any layout): by default where cta_ring_preferred says so,

@@ -45,10 +45,11 @@
 //
 // Summation order (fixed; it depends only on D, the element type, the
 // threads per row and the row's 16-byte phase):
-//   1. each thread keeps two partial sums, one over the elements at even
-//      positions of its chunks and one over the odd positions, each added in
-//      slot order then position order; its partial is even + odd, plus the
-//      term of its edge element if it owns one;
+//   1. each thread keeps four partial sums: binary32 pairs (columns 2j,
+//      2j + 1 of a chunk) go to one of two packed accumulators by the parity
+//      of j, each added in slot order then pair order; the two accumulators
+//      are added, then the two lanes of the result (the even and the odd
+//      columns), plus the term of its edge element if it owns one;
 //   2. an xor butterfly over the G lanes sharing the row (offsets G/2 .. 1);
 //   3. for rows owned by a whole block of NW warps, the per-warp sums are
 //      combined by the same xor butterfly over lanes 0 .. NW-1 (warp w's sum
@@ -204,6 +205,8 @@ struct Elem<float> {
     return __float_as_uint(*p);
   }
   static __device__ __forceinline__ void put(float* p, float v) { *p = v; }
+  // the element in the low bytes of a little-endian 32-bit word
+  static __device__ __forceinline__ float low(uint32_t w) { return __uint_as_float(w); }
   // v as stored: binary32 already is
   static __device__ __forceinline__ float stored(float v) { return v; }
   static __device__ __forceinline__ void unpack(const uint4& u, F2 (&f)[2]) {
@@ -233,6 +236,8 @@ struct Elem<__nv_bfloat16> {
   static __device__ __forceinline__ void put(__nv_bfloat16* p, float v) {
     *p = __float2bfloat16_rn(v);
   }
+  // the element in the low bytes of a little-endian 32-bit word, widened
+  static __device__ __forceinline__ float low(uint32_t w) { return __uint_as_float(w << 16); }
   // v rounded to bfloat16 (nearest, ties to even), widened back exactly
   static __device__ __forceinline__ float stored(float v) {
     return __bfloat162float(__float2bfloat16_rn(v));
@@ -366,17 +371,22 @@ __device__ __forceinline__ float load_edge(const Row<T>& g, int D, int k0) {
 // the thread's slots, then, for a thread that owns an edge element, that
 // element's term added (a square by one fused multiply-add).
 
+// Two packed accumulators per pass: pair j of every chunk goes to
+// acc[j & 1], so the dependent chains are half as long; the thread's partial
+// is (acc[0] + acc[1]), then its two lanes added.
+__device__ __forceinline__ float hsum_acc(const F2 (&acc)[2]) { return hsum2(add2(acc[0], acc[1])); }
+
 // RMSNorm: sum of squares (absent slots hold zeros, which add nothing).
 template <typename T, bool EXACT, int NSLOT>
 __device__ __forceinline__ float sum_squares(const F2 (&v)[NSLOT][Elem<T>::P], float xe,
                                              bool has_edge) {
   constexpr int P = Elem<T>::P;
-  F2 acc = zero2();
+  F2 acc[2] = {zero2(), zero2()};
 #pragma unroll
   for (int p = 0; p < NSLOT; ++p)
 #pragma unroll
-    for (int j = 0; j < P; ++j) acc = fma2(v[p][j], v[p][j], acc);
-  float s = hsum2(acc);
+    for (int j = 0; j < P; ++j) acc[j & 1] = fma2(v[p][j], v[p][j], acc[j & 1]);
+  float s = hsum_acc(acc);
   if (!EXACT && has_edge) s = __fmaf_rn(xe, xe, s);
   return s;
 }
@@ -389,18 +399,18 @@ __device__ __forceinline__ float shift_and_sum(F2 (&v)[NSLOT][Elem<T>::P], float
                                                bool has_edge) {
   constexpr int P = Elem<T>::P;
   const F2 K2 = splat(K);
-  F2 acc = zero2();
+  F2 acc[2] = {zero2(), zero2()};
 #pragma unroll
   for (int p = 0; p < NSLOT; ++p) {
     if (slot_present<SLOTS, NSLOT>(p, k0 + step * p, g.nfull)) {
 #pragma unroll
       for (int j = 0; j < P; ++j) {
         v[p][j] = sub2(v[p][j], K2);
-        acc = add2(acc, v[p][j]);
+        acc[j & 1] = add2(acc[j & 1], v[p][j]);
       }
     }
   }
-  float s = hsum2(acc);
+  float s = hsum_acc(acc);
   if (!EXACT && has_edge) {
     xe = __fsub_rn(xe, K);
     s = __fadd_rn(s, xe);
@@ -417,18 +427,18 @@ __device__ __forceinline__ float sum_dev_squares(F2 (&v)[NSLOT][Elem<T>::P], flo
                                                  bool has_edge) {
   constexpr int P = Elem<T>::P;
   const F2 M2 = splat(mean);
-  F2 acc = zero2();
+  F2 acc[2] = {zero2(), zero2()};
 #pragma unroll
   for (int p = 0; p < NSLOT; ++p) {
     if (slot_present<SLOTS, NSLOT>(p, k0 + step * p, g.nfull)) {
 #pragma unroll
       for (int j = 0; j < P; ++j) {
         v[p][j] = sub2(v[p][j], M2);
-        acc = fma2(v[p][j], v[p][j], acc);
+        acc[j & 1] = fma2(v[p][j], v[p][j], acc[j & 1]);
       }
     }
   }
-  float s = hsum2(acc);
+  float s = hsum_acc(acc);
   if (!EXACT && has_edge) {
     xe = __fsub_rn(xe, mean);
     s = __fmaf_rn(xe, xe, s);

@@ -39,10 +39,6 @@ struct Params {
   int stage_word;  // kOpRmsRope: first 16-byte word of the lane groups' staging rows
 };
 
-__device__ __forceinline__ Segment pick_segment(const Segment (&seg)[2], int i) {
-  return i == 0 ? seg[0] : seg[1];
-}
-
 constexpr int kWarpBlock = 256;
 // Block-family register budget: at least 1024 threads resident per SM (64
 // registers).
@@ -330,6 +326,27 @@ __device__ __forceinline__ void run_segment(const Segment& s, const Prefetch<T, 
   }
 }
 
+// One row space of the lane-group kernel.
+template <typename T, int OP, bool EXACT, int SLOTS, int VPL>
+__device__ __forceinline__ void warp_segment(const Params& p, const Segment& s,
+                                             const Prefetch<T, VPL>& pf,
+                                             const Prefetch<T, VPL>& pf2, int lane,
+                                             long long warp, long long nwarps, int cache_word) {
+  const int G = s.lanes;
+  const int per_warp = 32 / G;
+  const int gl = lane & (G - 1);
+  const int gi = lane / G;
+  const unsigned mask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << (gi * G));
+  auto reduce = [&](float t) { return group_sum(t, G, mask); };
+  float* stage = nullptr;
+  if constexpr (OP == kOpRmsRope)  // the in-thread variant stages nothing
+    stage = reinterpret_cast<float*>(dyn_smem + p.stage_word) +
+            ((threadIdx.x >> 5) * per_warp + gi) * s.dim;
+  run_segment<T, OP, EXACT, SLOTS, VPL, kWarpPrefetchStages>(
+      s, pf, pf2, warp * per_warp + gi, nwarps * per_warp, gl, G, p.eps, reduce, cache_word,
+      stage, mask);
+}
+
 template <typename T, int OP, bool EXACT, int SLOTS, int VPL>
 __global__ void __launch_bounds__(kWarpBlock, (warp_blocks_per_sm<T, OP, SLOTS, VPL>()))
 rows_warp_kernel(const Params p) {
@@ -340,23 +357,11 @@ rows_warp_kernel(const Params p) {
   const long long warp = (long long)blockIdx.x * (kWarpBlock / 32) + (threadIdx.x >> 5);
   const long long nwarps = (long long)gridDim.x * (kWarpBlock / 32);
   const int cache_word = p.prefetch ? BANK * (op_has_second(OP) ? 2 : 1) : 0;
-#pragma unroll 1
-  for (int si = 0; si < p.nseg; ++si) {
-    const Segment s = pick_segment(p.seg, si);
-    const int G = s.lanes;
-    const int per_warp = 32 / G;
-    const int gl = lane & (G - 1);
-    const int gi = lane / G;
-    const unsigned mask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << (gi * G));
-    auto reduce = [&](float t) { return group_sum(t, G, mask); };
-    float* stage = nullptr;
-    if constexpr (OP == kOpRmsRope)  // the in-thread variant stages nothing
-      stage = reinterpret_cast<float*>(dyn_smem + p.stage_word) +
-              ((threadIdx.x >> 5) * per_warp + gi) * s.dim;
-    run_segment<T, OP, EXACT, SLOTS, VPL, kWarpPrefetchStages>(
-        s, pf, pf2, warp * per_warp + gi, nwarps * per_warp, gl, G, p.eps, reduce, cache_word,
-        stage, mask);
-  }
+  // each row space by a reference fixed at compile time (p.seg[0], p.seg[1]),
+  // so that its fields stay kernel-parameter operands rather than registers
+  warp_segment<T, OP, EXACT, SLOTS, VPL>(p, p.seg[0], pf, pf2, lane, warp, nwarps, cache_word);
+  if (p.nseg > 1)
+    warp_segment<T, OP, EXACT, SLOTS, VPL>(p, p.seg[1], pf, pf2, lane, warp, nwarps, cache_word);
 }
 
 template <typename T, int OP, bool EXACT, int SLOTS, int NT, int VPT>
@@ -377,13 +382,15 @@ rows_cta_kernel(const Params p) {
     return r;
   };
   const int cache_word = p.prefetch ? BANK * (op_has_second(OP) ? 2 : 1) : 0;
-#pragma unroll 1
-  for (int si = 0; si < p.nseg; ++si) {
-    const Segment s = pick_segment(p.seg, si);
+  // block rows come one row space at a time (the dual op runs head rows in
+  // lane groups), by a reference fixed at compile time
+  run_segment<T, OP, EXACT, SLOTS, VPT, cta_prefetch_stages(NT, OP)>(
+      p.seg[0], pf, pf2, blockIdx.x, gridDim.x, threadIdx.x, NT, p.eps, reduce, cache_word,
+      nullptr, 0u);
+  if (p.nseg > 1)
     run_segment<T, OP, EXACT, SLOTS, VPT, cta_prefetch_stages(NT, OP)>(
-        s, pf, pf2, blockIdx.x, gridDim.x, threadIdx.x, NT, p.eps, reduce, cache_word, nullptr,
-        0u);
-  }
+        p.seg[1], pf, pf2, blockIdx.x, gridDim.x, threadIdx.x, NT, p.eps, reduce, cache_word,
+        nullptr, 0u);
 }
 
 }  // namespace rn

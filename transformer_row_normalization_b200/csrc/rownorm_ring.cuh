@@ -133,28 +133,58 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 // the same chunks of every row), unpacked at each use. NULL weight = ones,
 // NULL bias = zeros, as AffineDirect; the values, and so the bits, are the
 // same.
-template <typename T, bool BIAS, int NSLOT>
+// Weight and bias of a lane's chunk slots: the packed 16-byte words of the
+// first NREG slots held in registers (loaded once per row space: in an
+// aligned layout a lane owns the same chunks of every row), the others read
+// from L1 at each use; unpacked at each use. NULL weight = ones, NULL bias =
+// zeros, as AffineDirect; the values, and so the bits, are the same.
+template <typename T, bool BIAS, int NSLOT, int NREG>
 struct AffineRegs {
-  uint4 w[NSLOT];
-  uint4 b[BIAS ? NSLOT : 1];
-  __device__ __forceinline__ void load(const Segment& s, int k0, int step) {
+  static_assert(NREG >= 1 && NREG <= NSLOT, "slots in registers");
+  uint4 w[NREG];
+  uint4 b[BIAS ? NREG : 1];
+  const T* wv;
+  const T* bv;
+  int k0, step;
+  __device__ __forceinline__ void load(const Segment& s, int k0_, int step_) {
     constexpr int V = Elem<T>::V;
-    const T* wv = static_cast<const T*>(s.w);
-    const T* bv = static_cast<const T*>(s.b);
+    wv = static_cast<const T*>(s.w);
+    bv = static_cast<const T*>(s.b);
+    k0 = k0_;
+    step = step_;
     const uint32_t one = Elem<T>::kOneBits | (sizeof(T) == 2 ? Elem<T>::kOneBits << 16 : 0u);
     const int nfull = s.dim / V;
 #pragma unroll
-    for (int p = 0; p < NSLOT; ++p) {
+    for (int p = 0; p < NREG; ++p) {
       const int f = k0 + step * p;
       const bool in = f < nfull;
       w[p] = (wv && in) ? load_cached(wv + f * V) : make_uint4(one, one, one, one);
       if constexpr (BIAS) b[p] = (bv && in) ? load_cached(bv + f * V) : make_uint4(0, 0, 0, 0);
     }
   }
-  __device__ __forceinline__ void get(int p, int /*f*/, F2 (&wf)[Elem<T>::P],
+  __device__ __forceinline__ void get(int p, int f, F2 (&wf)[Elem<T>::P],
                                       F2 (&bf)[Elem<T>::P]) const {
-    Elem<T>::unpack(w[p], wf);
-    if constexpr (BIAS) Elem<T>::unpack(b[p], bf);
+    constexpr int V = Elem<T>::V;
+    constexpr int P = Elem<T>::P;
+    if (p < NREG) {
+      Elem<T>::unpack(w[p < NREG ? p : 0], wf);
+      if constexpr (BIAS) Elem<T>::unpack(b[p < NREG ? p : 0], bf);
+      return;
+    }
+    if (wv) {
+      Elem<T>::unpack(load_cached(wv + f * V), wf);
+    } else {
+#pragma unroll
+      for (int j = 0; j < P; ++j) wf[j] = splat(1.f);
+    }
+    if constexpr (BIAS) {
+      if (bv) {
+        Elem<T>::unpack(load_cached(bv + f * V), bf);
+      } else {
+#pragma unroll
+        for (int j = 0; j < P; ++j) bf[j] = zero2();
+      }
+    }
   }
   __device__ __forceinline__ void edge(float& w_, float& b_) const {
     w_ = 1.f;
@@ -166,7 +196,7 @@ struct AffineRegs {
 // into `dst`, counted on `bar`.
 template <typename T>
 __device__ __forceinline__ void ring_issue(const Segment& s, long long tile, int R,
-                                           bool contiguous, int tx_extra, unsigned char* dst,
+                                           bool contiguous, int tx_extra, uint4* dst,
                                            uint64_t* bar) {
   const long long r0 = tile * R;
   const long long nr = s.rows - r0 < R ? s.rows - r0 : R;
@@ -178,36 +208,52 @@ __device__ __forceinline__ void ring_issue(const Segment& s, long long tile, int
               bar);
   } else {
     for (long long rr = 0; rr < nr; ++rr)
-      bulk_load(dst + rr * row_bytes, x + row_off(r0 + rr, s.x_stride, s.x_inner, s.x_outer),
-                row_bytes, bar);
+      bulk_load(dst + rr * (row_bytes / 16),
+                x + row_off(r0 + rr, s.x_stride, s.x_inner, s.x_outer), row_bytes, bar);
   }
 }
 
 // The rows of one staged tile (rows r0 .. r0 + nr - 1), normalized by the
-// warp's lane groups: lane group gi takes rows gi, gi + 32/G, ...
-template <typename T, int OP, int SLOTS, int VPL, typename Src>
-__device__ __forceinline__ void ring_tile_rows(const Segment& s, const unsigned char* stage,
-                                               long long r0, int nr, float eps, float inv_d,
-                                               int gl, int gi, unsigned mask, const Src& src) {
+// warp's lane groups: lane group gi takes rows gi, gi + 32/G, ... GC = 32
+// compiles the whole-warp case (one row at a time, a fixed butterfly); GC =
+// 0 takes G from the row space. Both add in the same order.
+// The stage starts at 16-byte word `stage_word` of the dynamic shared memory
+// (indexed from the shared array itself, so that the loads use 32-bit
+// shared-window addresses).
+template <typename T, int OP, int SLOTS, int VPL, int GC, typename Src>
+__device__ __forceinline__ void ring_tile_rows(const Segment& s, int stage_word, long long r0,
+                                               int nr, float eps, float inv_d, int gl, int gi,
+                                               unsigned mask, const Src& src) {
   constexpr int P = Elem<T>::P;
-  const int G = s.lanes;
-  auto reduce = [&](float t) { return group_sum(t, G, mask); };
-  const int row_bytes = s.dim * (int)sizeof(T);
+  const int G = GC ? GC : s.lanes;
+  auto reduce = [&](float t) {
+    if constexpr (GC == 32) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+        t = __fadd_rn(t, __shfl_xor_sync(0xffffffffu, t, off));
+      return t;
+    } else {
+      return group_sum(t, G, mask);
+    }
+  };
+  const int row_words = s.dim * (int)sizeof(T) / 16;
 #pragma unroll 1
   for (int rr = gi; rr < nr; rr += 32 / G) {
     const Row<T> g = row_geometry<T, true>(s, r0 + rr);
-    const uint4* row = reinterpret_cast<const uint4*>(stage + rr * row_bytes);
+    const int row = stage_word + rr * row_words;
     F2 v[VPL][P];
 #pragma unroll
     for (int q = 0; q < VPL; ++q) {
       if (slot_present<SLOTS, VPL>(q, gl + G * q, g.nfull)) {
-        Elem<T>::unpack(row[gl + G * q], v[q]);
+        Elem<T>::unpack(dyn_smem[row + gl + G * q], v[q]);
       } else {
 #pragma unroll
         for (int j = 0; j < P; ++j) v[q][j] = zero2();
       }
     }
-    const float K = OP == kOpLn ? Elem<T>::get(reinterpret_cast<const T*>(row)) : 0.f;
+    // the row's first element, from the first 4 bytes of its first chunk
+    const float K =
+        OP == kOpLn ? Elem<T>::low(reinterpret_cast<const uint32_t*>(dyn_smem)[4 * row]) : 0.f;
     float xe = 0.f, rstd, mean;
     row_stats<T, OP, true, SLOTS, VPL>(v, xe, g, inv_d, gl, G, K, eps, false, reduce, rstd,
                                        mean);
@@ -223,9 +269,16 @@ __device__ __forceinline__ void ring_tile_rows(const Segment& s, const unsigned 
 // the op needs no other per-element tables; otherwise read from L1 per row
 // (AffineDirect). Beyond that, the values held across the row spill under
 // the 128-register budget (ptxas).
-template <int OP, int VPL>
-__host__ __device__ constexpr bool ring_weights_in_regs() {
-  return OP != kOpRmsRopeLocal && VPL <= 3;
+// Slots whose weight (and bias) words stay in registers: as many as keep a
+// lane's row values (VPL chunks as binary32) plus those words within 48
+// registers, so that the kernel fits the 128-register budget without
+// spilling (ptxas, both element types); none for RoPE rows, which also hold
+// their cos / sin values.
+template <typename T, int OP, int VPL>
+__host__ __device__ constexpr int ring_weight_slots_in_regs() {
+  if (OP == kOpRmsRopeLocal) return 0;
+  const int room = (48 - VPL * Elem<T>::V) / (4 * (OP == kOpLn ? 2 : 1));
+  return room < 0 ? 0 : (room > VPL ? VPL : room);
 }
 
 // Register budget: 4 blocks of kRingWarps warps per SM (16 warps, up to 128
@@ -234,19 +287,110 @@ __host__ __device__ constexpr bool ring_weights_in_regs() {
 // of 80 registers spilled and ran 10 % slower.
 constexpr int kRingBlocksPerSm = 4;
 
+// The state of one warp's ring between row spaces: the stage to use next,
+// bit k of `parity` the phase parity with which stage k completes next (the
+// stages run round robin across the row spaces).
+struct RingState {
+  int st;
+  uint32_t parity;
+  bool ok;
+};
+
+// One row space (segment SI, a compile-time index, so that its fields stay
+// kernel-parameter operands rather than registers) through this warp's ring.
+template <typename T, int OP, int SLOTS, int VPL, int SI>
+__device__ __forceinline__ void ring_segment(const RingParams& p, RingState& rs, int ring_word,
+                                             int stage_words, uint64_t* bars, long long w,
+                                             long long W) {
+  constexpr bool BIAS = OP == kOpLn;
+  const Segment& s = p.seg[SI];
+  const int lane = threadIdx.x & 31;
+  const int S = p.stages;
+  const int R = p.tile_rows[SI];
+  const bool contiguous = p.contiguous[SI] != 0;
+  const long long ntiles = (s.rows + R - 1) / R;
+  const long long n = ntiles > w ? (ntiles - w + W - 1) / W : 0;  // this warp's tiles
+  if (n == 0) return;
+  const int G = s.lanes;
+  const int gl = lane & (G - 1);
+  const int gi = lane / G;
+  const unsigned mask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << (gi * G));
+  const float inv_d = inv_dim(s.dim);
+  constexpr int NREG = ring_weight_slots_in_regs<T, OP, VPL>();
+  using Regs = AffineRegs<T, BIAS, VPL, NREG ? NREG : 1>;
+  using Direct = AffineDirect<T, BIAS, false>;
+  std::conditional_t<(NREG > 0), Regs, Direct> src;
+  if constexpr (NREG > 0)
+    src.load(s, gl, G);
+  else
+    src = Direct{static_cast<const T*>(s.w), static_cast<const T*>(s.b)};
+  int st = rs.st;
+  uint32_t parity = rs.parity;
+  // every stage is free here: the previous row space's tiles are consumed
+  if (lane == 0) {
+    int k = st;
+    for (long long i = 0; i < n && i < S; ++i) {
+      ring_issue<T>(s, w + i * W, R, contiguous, p.tx_extra,
+                    dyn_smem + ring_word + k * stage_words, &bars[k]);
+      k = k + 1 == S ? 0 : k + 1;
+    }
+  }
+  __syncwarp();
+  long long i = 0;
+  bool ok = true;
+#pragma unroll 1
+  for (; i < n; ++i) {
+    ok = mbar_wait(&bars[st], (parity >> st) & 1u, p.wait_ns);
+    if (__any_sync(0xffffffffu, !ok)) {
+      ok = false;
+      break;
+    }
+    parity ^= 1u << st;
+    const long long r0 = (w + i * W) * R;
+    const int nr = (int)(s.rows - r0 < R ? s.rows - r0 : R);
+    const int stage_word = ring_word + st * stage_words;
+    if (G == 32)
+      ring_tile_rows<T, OP, SLOTS, VPL, 32>(s, stage_word, r0, nr, p.eps, inv_d, gl, gi, mask,
+                                            src);
+    else
+      ring_tile_rows<T, OP, SLOTS, VPL, 0>(s, stage_word, r0, nr, p.eps, inv_d, gl, gi, mask,
+                                           src);
+    // every lane has read the stage: refill it with the tile S ahead
+    __syncwarp();
+    if (lane == 0 && i + S < n) {
+      fence_async_shared();
+      ring_issue<T>(s, w + (i + S) * W, R, contiguous, p.tx_extra,
+                    dyn_smem + ring_word + st * stage_words, &bars[st]);
+    }
+    st = st + 1 == S ? 0 : st + 1;
+  }
+  if (!ok && lane == 0) {
+    // tiles i .. min(n, i + S) - 1 are issued and not yet consumed, in
+    // stages st, st + 1, ... (mod S)
+    int k = st;
+    for (long long j = i; j < n && j < i + S; ++j) {
+      mbar_wait(&bars[k], (parity >> k) & 1u, p.drain_ns);
+      k = k + 1 == S ? 0 : k + 1;
+    }
+    atomicAdd(&g_ring_timeouts, 1u);
+  }
+  rs.st = st;
+  rs.parity = parity;
+  rs.ok = ok;
+}
+
 template <typename T, int OP, int SLOTS, int VPL>
 __global__ void __launch_bounds__(kRingWarps * 32, kRingBlocksPerSm)
 rows_ring_kernel(const RingParams p) {
   static_assert(OP == kOpRms || OP == kOpLn || OP == kOpRmsRopeLocal,
                 "rings carry RMSNorm and LayerNorm rows, and head rows rotated in-thread");
-  constexpr bool BIAS = OP == kOpLn;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int S = p.stages;
-  unsigned char* const smem = reinterpret_cast<unsigned char*>(dyn_smem);
-  unsigned char* const ring = smem + warp * S * p.stage_bytes;
+  const int stage_words = p.stage_bytes / 16;
+  const int ring_word = warp * S * stage_words;  // this warp's stages, in 16-byte words
   uint64_t* const bars =
-      reinterpret_cast<uint64_t*>(smem + kRingWarps * S * p.stage_bytes) + warp * kRingMaxStages;
+      reinterpret_cast<uint64_t*>(dyn_smem + kRingWarps * S * stage_words) + warp * kRingMaxStages;
   const long long w = (long long)blockIdx.x * kRingWarps + warp;
   const long long W = (long long)gridDim.x * kRingWarps;
   if (lane == 0) {
@@ -254,74 +398,10 @@ rows_ring_kernel(const RingParams p) {
     fence_mbar_init();
   }
   __syncwarp();
-  // The stages are used round robin across the row spaces; bit k of
-  // `parity` is the phase parity with which stage k completes next.
-  uint32_t parity = 0;
-  int st = 0;
-  bool ok = true;
-#pragma unroll 1
-  for (int si = 0; si < p.nseg && ok; ++si) {
-    const Segment s = pick_segment(p.seg, si);
-    const int R = si ? p.tile_rows[1] : p.tile_rows[0];
-    const bool contiguous = (si ? p.contiguous[1] : p.contiguous[0]) != 0;
-    const long long ntiles = (s.rows + R - 1) / R;
-    const long long n = ntiles > w ? (ntiles - w + W - 1) / W : 0;  // this warp's tiles
-    if (n == 0) continue;
-    const int G = s.lanes;
-    const int gl = lane & (G - 1);
-    const int gi = lane / G;
-    const unsigned mask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << (gi * G));
-    const float inv_d = inv_dim(s.dim);
-    using Regs = AffineRegs<T, BIAS, VPL>;
-    using Direct = AffineDirect<T, BIAS, false>;
-    std::conditional_t<ring_weights_in_regs<OP, VPL>(), Regs, Direct> src;
-    if constexpr (ring_weights_in_regs<OP, VPL>())
-      src.load(s, gl, G);
-    else
-      src = Direct{static_cast<const T*>(s.w), static_cast<const T*>(s.b)};
-    // every stage is free here: the previous row space's tiles are consumed
-    if (lane == 0) {
-      int k = st;
-      for (long long i = 0; i < n && i < S; ++i) {
-        ring_issue<T>(s, w + i * W, R, contiguous, p.tx_extra, ring + k * p.stage_bytes,
-                      &bars[k]);
-        k = k + 1 == S ? 0 : k + 1;
-      }
-    }
-    __syncwarp();
-    long long i = 0;
-#pragma unroll 1
-    for (; i < n; ++i) {
-      ok = mbar_wait(&bars[st], (parity >> st) & 1u, p.wait_ns);
-      if (__any_sync(0xffffffffu, !ok)) {
-        ok = false;
-        break;
-      }
-      parity ^= 1u << st;
-      const long long r0 = (w + i * W) * R;
-      const int nr = (int)(s.rows - r0 < R ? s.rows - r0 : R);
-      ring_tile_rows<T, OP, SLOTS, VPL>(s, ring + st * p.stage_bytes, r0, nr, p.eps, inv_d, gl,
-                                        gi, mask, src);
-      // every lane has read the stage: refill it with the tile S ahead
-      __syncwarp();
-      if (lane == 0 && i + S < n) {
-        fence_async_shared();
-        ring_issue<T>(s, w + (i + S) * W, R, contiguous, p.tx_extra, ring + st * p.stage_bytes,
-                      &bars[st]);
-      }
-      st = st + 1 == S ? 0 : st + 1;
-    }
-    if (!ok && lane == 0) {
-      // tiles i .. min(n, i + S) - 1 are issued and not yet consumed, in
-      // stages st, st + 1, ... (mod S)
-      int k = st;
-      for (long long j = i; j < n && j < i + S; ++j) {
-        mbar_wait(&bars[k], (parity >> k) & 1u, p.drain_ns);
-        k = k + 1 == S ? 0 : k + 1;
-      }
-      atomicAdd(&g_ring_timeouts, 1u);
-    }
-  }
+  RingState rs{0, 0u, true};
+  ring_segment<T, OP, SLOTS, VPL, 0>(p, rs, ring_word, stage_words, bars, w, W);
+  if (p.nseg > 1 && rs.ok)
+    ring_segment<T, OP, SLOTS, VPL, 1>(p, rs, ring_word, stage_words, bars, w, W);
 }
 
 }  // namespace rn
@@ -343,7 +423,7 @@ namespace rn {
 // are loaded into register queues when their copies are issued.
 
 template <typename T, bool EXACT>
-__device__ __forceinline__ void cta_ring_issue(const Segment& s, long long r, unsigned char* dst,
+__device__ __forceinline__ void cta_ring_issue(const Segment& s, long long r, uint4* dst,
                                                uint64_t* bar, int tx_extra) {
   const Row<T> g = row_geometry<T, EXACT>(s, r);
   const uint32_t bytes = (uint32_t)g.nfull * 16u;
@@ -353,7 +433,7 @@ __device__ __forceinline__ void cta_ring_issue(const Segment& s, long long r, un
 
 template <typename T, int OP, bool EXACT, int SLOTS, int NT, int VPT, int NST, typename Src>
 __device__ __forceinline__ void cta_ring_rows(const RingParams& p, const Segment& s,
-                                              unsigned char* ring, uint64_t* bars, Src& src,
+                                              uint64_t* bars, Src& src,
                                               float (*red)[NT / 32], bool& ok) {
   constexpr int P = Elem<T>::P;
   const int tid = threadIdx.x;
@@ -372,7 +452,7 @@ __device__ __forceinline__ void cta_ring_rows(const RingParams& p, const Segment
   auto ahead = [&](long long ra, int st, int j) {
     const Row<T> ga = row_geometry<T, EXACT>(s, ra);
     if (tid == 0)
-      cta_ring_issue<T, EXACT>(s, ra, ring + (long long)st * p.stage_bytes, &bars[st], p.tx_extra);
+      cta_ring_issue<T, EXACT>(s, ra, dyn_smem + st * (p.stage_bytes / 16), &bars[st], p.tx_extra);
     Kq[j] = OP == kOpLn ? Elem<T>::get(ga.x_row) : 0.f;
     Eq[j] = load_edge<T, EXACT>(ga, D, tid);
   };
@@ -419,12 +499,12 @@ __device__ __forceinline__ void cta_ring_rows(const RingParams& p, const Segment
     }
     const Row<T> g = row_geometry<T, EXACT>(s, r);
     const bool has_edge = !EXACT && tid < g.nedge;
-    const uint4* stage = reinterpret_cast<const uint4*>(ring + (long long)st * p.stage_bytes);
+    const int stage = st * (p.stage_bytes / 16);  // 16-byte words
     F2 v[VPT][P];
 #pragma unroll
     for (int q = 0; q < VPT; ++q) {
       if (slot_present<SLOTS, VPT>(q, tid + NT * q, g.nfull)) {
-        Elem<T>::unpack(stage[tid + NT * q], v[q]);
+        Elem<T>::unpack(dyn_smem[stage + tid + NT * q], v[q]);
       } else {
 #pragma unroll
         for (int j = 0; j < P; ++j) v[q][j] = zero2();
@@ -463,7 +543,6 @@ rows_cta_ring_kernel(const RingParams p) {
   constexpr bool BIAS = OP == kOpLn;
   __shared__ float red[2][NT / 32];
   __shared__ __align__(8) uint64_t bars[NST];
-  unsigned char* const ring = reinterpret_cast<unsigned char*>(dyn_smem);
   if (threadIdx.x == 0) {
     for (int st = 0; st < NST; ++st) mbar_init(&bars[st], 1);
     fence_mbar_init();
@@ -476,15 +555,15 @@ rows_cta_ring_kernel(const RingParams p) {
   if constexpr (EXACT) {
     if (w && (!BIAS || b)) {
       AffineDirect<T, BIAS, true> src{w, b};
-      cta_ring_rows<T, OP, true, SLOTS, NT, VPT, NST>(p, s, ring, bars, src, red, ok);
+      cta_ring_rows<T, OP, true, SLOTS, NT, VPT, NST>(p, s, bars, src, red, ok);
     } else {
       AffineDirect<T, BIAS, false> src{w, b};
-      cta_ring_rows<T, OP, true, SLOTS, NT, VPT, NST>(p, s, ring, bars, src, red, ok);
+      cta_ring_rows<T, OP, true, SLOTS, NT, VPT, NST>(p, s, bars, src, red, ok);
     }
   } else {
     AffineCache<T, VPT, BIAS> src;
     src.init(NST * p.stage_bytes / 16);
-    cta_ring_rows<T, OP, false, SLOTS, NT, VPT, NST>(p, s, ring, bars, src, red, ok);
+    cta_ring_rows<T, OP, false, SLOTS, NT, VPT, NST>(p, s, bars, src, red, ok);
   }
 }
 
