@@ -407,8 +407,10 @@ int round_up(int64_t v, int64_t m) { return (int)((v + m - 1) / m * m); }
 //   but bf16 LayerNorm 512 (16 lanes per row) 31.8 -> 34.7 us and binary32
 //   LayerNorm 1024 88.1 -> 94.1 us ran slower, and stay on the register
 //   kernels.
-bool ring_preferred(int dtype, const SegPlan* plans, int nseg) {
-  if (dtype != RN_BF16) return false;
+//   The dual head norm + RoPE also ran slower in rings (47.1 -> 53.2 us), so
+//   the rings take it only when forced.
+bool ring_preferred(int dtype, int op, const SegPlan* plans, int nseg) {
+  if (dtype != RN_BF16 || (op != rn::kOpRms && op != rn::kOpLn)) return false;
   if (nseg == 2) return true;
   return plans[0].lanes == 32;
 }
@@ -424,7 +426,7 @@ bool plan_ring(int dtype, int op, const SegPlan* plans, const rn_view* const* xs
   if (op != rn::kOpRms && op != rn::kOpLn && op != rn::kOpRmsRopeLocal) return false;
   for (int i = 0; i < nseg; ++i)
     if (plans[i].family != 0 || !plans[i].exact) return false;
-  if (path == 0 && !ring_preferred(dtype, plans, nseg)) return false;
+  if (path == 0 && !ring_preferred(dtype, op, plans, nseg)) return false;
   const void* fn = dtype == RN_F32 ? rn::ring_kernel_f32(op, slots, chunks)
                                    : rn::ring_kernel_bf16(op, slots, chunks);
   if (!fn) return false;

@@ -184,12 +184,13 @@ struct GateSrc {
 // rows ahead wait in register queues. `src` supplies weight and bias.
 template <typename T, int OP, bool EXACT, int SLOTS, int NSLOT, int NST, typename Src,
           typename Reduce>
-__device__ __forceinline__ void segment_rows(const Segment& s, const Prefetch<T, NSLOT>& pf,
+__device__ __forceinline__ void segment_rows(const Segment& seg, const Prefetch<T, NSLOT>& pf,
                                              const Prefetch<T, NSLOT>& pf2, long long r0,
                                              long long stride, int k0, int step, float eps,
                                              Reduce reduce, Src& src, float* stage,
                                              unsigned mask) {
   static_assert(NST >= 1, "at least one row ahead");
+  const Segment& s = seg;
   constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
   constexpr bool SECOND = op_has_second(OP);
@@ -382,15 +383,30 @@ rows_cta_kernel(const Params p) {
     return r;
   };
   const int cache_word = p.prefetch ? BANK * (op_has_second(OP) ? 2 : 1) : 0;
-  // block rows come one row space at a time (the dual op runs head rows in
-  // lane groups), by a reference fixed at compile time
-  run_segment<T, OP, EXACT, SLOTS, VPT, cta_prefetch_stages(NT, OP)>(
-      p.seg[0], pf, pf2, blockIdx.x, gridDim.x, threadIdx.x, NT, p.eps, reduce, cache_word,
-      nullptr, 0u);
-  if (p.nseg > 1)
+  if constexpr (EXACT) {
+    // the row space by a compile-time reference to the kernel parameters, as
+    // the lane-group and ring kernels take it (LayerNorm 65536 x 8192: 345.0
+    // -> 338.9 us on B200)
     run_segment<T, OP, EXACT, SLOTS, VPT, cta_prefetch_stages(NT, OP)>(
-        p.seg[1], pf, pf2, blockIdx.x, gridDim.x, threadIdx.x, NT, p.eps, reduce, cache_word,
+        p.seg[0], pf, pf2, blockIdx.x, gridDim.x, threadIdx.x, NT, p.eps, reduce, cache_word,
         nullptr, 0u);
+    if (p.nseg > 1)
+      run_segment<T, OP, EXACT, SLOTS, VPT, cta_prefetch_stages(NT, OP)>(
+          p.seg[1], pf, pf2, blockIdx.x, gridDim.x, threadIdx.x, NT, p.eps, reduce, cache_word,
+          nullptr, 0u);
+  } else {
+    // rows off the 16-byte grid take a copy picked at run time: with the
+    // compile-time reference the off-grid LayerNorm kernel spilled 12 bytes
+    // in its row loop at 64 registers (LayerNorm 65536 x 4097: 303 against
+    // 204 us)
+#pragma unroll 1
+    for (int si = 0; si < p.nseg; ++si) {
+      const Segment s = si == 0 ? p.seg[0] : p.seg[1];
+      run_segment<T, OP, EXACT, SLOTS, VPT, cta_prefetch_stages(NT, OP)>(
+          s, pf, pf2, blockIdx.x, gridDim.x, threadIdx.x, NT, p.eps, reduce, cache_word, nullptr,
+          0u);
+    }
+  }
 }
 
 }  // namespace rn

@@ -432,10 +432,11 @@ __device__ __forceinline__ void cta_ring_issue(const Segment& s, long long r, ui
 }
 
 template <typename T, int OP, bool EXACT, int SLOTS, int NT, int VPT, int NST, typename Src>
-__device__ __forceinline__ void cta_ring_rows(const RingParams& p, const Segment& s,
+__device__ __forceinline__ void cta_ring_rows(const RingParams& p, const Segment& seg,
                                               uint64_t* bars, Src& src,
                                               float (*red)[NT / 32], bool& ok) {
   constexpr int P = Elem<T>::P;
+  const Segment& s = seg;
   const int tid = threadIdx.x;
   const int D = s.dim;
   const float inv_d = inv_dim(D);
