@@ -291,11 +291,13 @@ typedef struct rn_launch_info {
                             /* aligned and dim fills whole 16-byte chunks;  */
                             /* 2 as 1, and those chunks divide evenly over  */
                             /* the row's threads (no slot is ever empty)    */
-    int32_t staged;         /* 1: rows come through per-warp rings in      */
-                            /* shared memory filled by bulk copies (S      */
-                            /* stages per warp); 0: per-thread loads       */
-    int32_t stages;         /* staged: stages per warp                      */
-    int32_t stage_bytes;    /* staged: bytes per stage (a tile of rows)     */
+    int32_t staged;         /* 1: rows come through rings of shared-memory */
+                            /* stages filled by bulk copies, one ring per  */
+                            /* warp (family 0) or per block (family 1);    */
+                            /* 0: per-thread loads                         */
+    int32_t stages;         /* staged: stages per ring                      */
+    int32_t stage_bytes;    /* staged: bytes per stage (a tile of rows, or  */
+                            /* one row's full 16-byte chunks)              */
 } rn_launch_info;
 
 enum { RN_OP_RMS = 0, RN_OP_LN = 1, RN_OP_DUAL = 2, RN_OP_ADD_RMS = 3, RN_OP_GATED_RMS = 4 };
@@ -319,12 +321,14 @@ RN_API int rn_plan(int op, const rn_view *x, const rn_view *y,
 RN_API int rn_set_grid_override(int blocks);
 
 /* Kernel choice: 0 automatic; 1 register-resident kernels loading rows
- * directly; 2 the per-warp bulk-copy rings (rows of up to 1024 columns in
- * 16-byte aligned layouts come through a ring of shared-memory stages per
- * warp, filled with cp.async.bulk) wherever the shape allows, the register
- * kernels elsewhere; 3 register-resident kernels with a per-thread prefetch
- * of the rows ahead through shared memory (cp.async), also where the planner
- * would not prefetch. The per-row arithmetic is identical in every kind of
+ * directly; 2 the bulk-copy rings wherever the shape allows (RMSNorm and
+ * LayerNorm rows, and the dual head norm with or without in-thread RoPE:
+ * rows of up to 1024 columns in 16-byte aligned layouts through a ring of
+ * shared-memory stages per warp, wider rows through a ring per block; all
+ * filled with cp.async.bulk), the register kernels elsewhere; 3
+ * register-resident kernels with a per-thread prefetch of the rows ahead
+ * through shared memory (cp.async), also where the planner would not
+ * prefetch. The per-row arithmetic is identical in every kind of
  * kernel, so results do not depend on it. A test hook for tests and
  * measurements: it applies to every thread of the process (an atomic
  * setting). */

@@ -383,7 +383,7 @@ struct Launch {
   int ring;         // 1: rows_ring_kernel, 2: rows_cta_ring_kernel (RingParams)
   rn_launch_info info;
   // ring kernels only
-  int stages, stage_bytes, tile_rows[2], contiguous[2];
+  int stages, stage_bytes, tile_rows[2], contiguous[2], table_bytes;
   int stage_word;   // kOpRmsRope: staging rows after the slots and the cache
 };
 
@@ -393,7 +393,10 @@ struct Launch {
 #define RN_RING_TILE_BYTES 2048
 #endif
 constexpr int kRingTileBytes = RN_RING_TILE_BYTES;
-constexpr int kRingStages = 4;
+#ifndef RN_RING_STAGES
+#define RN_RING_STAGES 4
+#endif
+constexpr int kRingStages = RN_RING_STAGES;
 
 int round_up(int64_t v, int64_t m) { return (int)((v + m - 1) / m * m); }
 
@@ -420,7 +423,7 @@ bool ring_preferred(int dtype, int op, const SegPlan* plans, int nseg) {
 // it qualifies with rn_set_path_override(2), never with 1 or 3. Returns
 // false (the register-kernel plan stays in charge) otherwise.
 bool plan_ring(int dtype, int op, const SegPlan* plans, const rn_view* const* xs, int nseg,
-               int chunks, int slots, int dev, int sms, Launch* out) {
+               int chunks, int slots, int dev, int sms, const rn_rope* rope, Launch* out) {
   const int path = g_path_override.load(std::memory_order_relaxed);
   if (path == 1 || path == 3) return false;
   if (op != rn::kOpRms && op != rn::kOpLn && op != rn::kOpRmsRopeLocal) return false;
@@ -446,6 +449,24 @@ bool plan_ring(int dtype, int op, const SegPlan* plans, const rn_view* const* xs
     const int64_t tiles = ceil_div(xs[i]->rows, tr);
     if (tiles > tiles_max) tiles_max = tiles;
     if (tr * row_bytes > stage_bytes) stage_bytes = tr * row_bytes;
+  }
+  // RoPE rows: stage each tile's token's table row beside its rows when
+  // every tile lies in one token (tile rows divide both head counts) and the
+  // table rows start on the 16-byte grid
+  l.table_bytes = 0;
+  if (op == rn::kOpRmsRopeLocal && rope && rope->table && nseg == 2) {
+    const int64_t tb = (int64_t)rope->dims * 4;
+    const bool one_token = rope->heads_q % l.tile_rows[0] == 0 &&
+                           rope->heads_k % l.tile_rows[1] == 0;
+    if (one_token && tb % 16 == 0 && reinterpret_cast<uintptr_t>(rope->table) % 16 == 0) {
+      l.table_bytes = (int)tb;
+      int64_t sb = 16;
+      for (int i = 0; i < nseg; ++i) {
+        const int64_t b = (int64_t)l.tile_rows[i] * xs[i]->dim * es + tb;
+        if (b > sb) sb = b;
+      }
+      stage_bytes = sb;
+    }
   }
   l.stage_bytes = round_up(stage_bytes, 16);
   const DeviceInfo di = device_info(dev);
@@ -543,7 +564,8 @@ bool plan_cta_ring(int dtype, int op, const SegPlan* plans, const rn_view* const
 // per-warp bulk-copy rings where they apply and are chosen, else the register
 // kernels.
 int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* xs,
-                const void* const* ws, const void* const* bs, int nseg, Launch* out) {
+                const void* const* ws, const void* const* bs, int nseg, Launch* out,
+                const rn_rope* rope = nullptr) {
   int64_t rows[2] = {xs[0]->rows, nseg > 1 ? xs[1]->rows : 0};
   SegPlan merged = plans[0];
   for (int i = 1; i < nseg; ++i) {
@@ -565,7 +587,8 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
   int sms = 0, bps = 0;
   int st = device_sms(dev, &sms);
   if (st) return st;
-  if (plan_ring(dtype, op, plans, xs, nseg, merged.chunks, slots, dev, sms, out)) return RN_OK;
+  if (plan_ring(dtype, op, plans, xs, nseg, merged.chunks, slots, dev, sms, rope, out))
+    return RN_OK;
   if (plan_cta_ring(dtype, op, plans, xs, nseg, slots, dev, sms, out)) return RN_OK;
   const int threads = merged.family == 0 ? rn::kWarpBlock : merged.lanes;
   // the streaming kernels keep no weight cache and prefetch nothing
@@ -678,6 +701,7 @@ int launch(const Launch& l, const rn::Params& params, void* stream) {
     rp.wait_ns = wait_test ? 1000000ull : rn::kRingWaitLimitNs;
     rp.drain_ns = wait_test ? 2000000ull : rn::kRingDrainLimitNs;
     rp.tx_extra = wait_test ? 16 : 0;
+    rp.table_bytes = l.table_bytes;
     void* args[] = {&rp};
     e = cudaLaunchKernel(l.fn, dim3((unsigned)l.info.grid_blocks),
                          dim3((unsigned)l.info.block_threads), args, (size_t)l.smem,
@@ -923,7 +947,7 @@ int run_dual_rope(const rn_view* q, const rn_view* k, const void* wq, const void
   }
   Launch l{};
   if ((st = plan_launch(q->dtype, local ? rn::kOpRmsRopeLocal : rn::kOpRmsRope, plans, xs, ws,
-                        bs, 2, &l)))
+                        bs, 2, &l, rope)))
     return st;
   rn::Params params{};
   params.seg[0] = make_segment(q, yq, wq, nullptr, plans[0]);

@@ -706,12 +706,26 @@ __device__ __forceinline__ void store_chunk(const Segment& s, T* yc, const F2 (&
   }
 }
 
-template <typename T, bool LOCAL, bool EXACT, int SLOTS, int NSLOT, typename Src>
+// The row's cos / sin come from the table in global memory, or (TAB_SHARED,
+// in-thread planes only) from `tab_shared`: a copy of the row's table row
+// that the caller staged in shared memory.
+template <bool TAB_SHARED, int N>
+__device__ __forceinline__ void table_floats(const float* p, float (&d)[N]) {
+  if constexpr (TAB_SHARED)
+    load_floats<N>(p, d);
+  else
+    ldg_floats<N>(p, d);
+}
+
+template <typename T, bool LOCAL, bool EXACT, int SLOTS, int NSLOT, typename Src,
+          bool TAB_SHARED = false>
 __device__ __forceinline__ void normalize_rope_store(const Segment& s, const Row<T>& g,
                                                      F2 (&v)[NSLOT][Elem<T>::P], float xe,
                                                      const Src& src, int k0, int step,
                                                      float rstd, bool has_edge, long long r,
-                                                     float* stage, unsigned mask) {
+                                                     float* stage, unsigned mask,
+                                                     const float* tab_shared = nullptr) {
+  static_assert(!TAB_SHARED || LOCAL, "a staged table row serves in-thread planes");
   constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
   const int dims = s.rope_dims;
@@ -726,7 +740,7 @@ __device__ __forceinline__ void normalize_rope_store(const Segment& s, const Row
   // token = r / heads (32-bit division: head rows never reach 2^31)
   const long long token = r < 0x7fffffffLL ? (long long)((unsigned)r / (unsigned)s.rope_heads)
                                            : r / s.rope_heads;
-  const float* tab = s.rope_table + (s.rope_offset + token) * dims;
+  const float* tab = TAB_SHARED ? tab_shared : s.rope_table + (s.rope_offset + token) * dims;
   if constexpr (LOCAL && NSLOT % 2 == 0) {
     if (!trad) {
       // full split-half rotary whose chunks divide evenly: slot p < NSLOT/2
@@ -744,8 +758,8 @@ __device__ __forceinline__ void normalize_rope_store(const Segment& s, const Row
       for (int p = 0; p < NSLOT / 2; ++p) {
         const int c0 = (k0 + step * p) * V;
         float cs[V], sn[V];
-        ldg_floats<V>(tab + c0, cs);
-        ldg_floats<V>(tab + half + c0, sn);
+        table_floats<TAB_SHARED, V>(tab + c0, cs);
+        table_floats<TAB_SHARED, V>(tab + half + c0, sn);
         F2 ya[P], yb[P];
 #pragma unroll
         for (int j = 0; j < P; ++j) {
@@ -777,13 +791,13 @@ __device__ __forceinline__ void normalize_rope_store(const Segment& s, const Row
       if (c0 < dims) {
         float cs[P], sn[P];
         if constexpr (P % 4 == 0) {
-          ldg_floats<P>(tab + (c0 >> 1), cs);
-          ldg_floats<P>(tab + half + (c0 >> 1), sn);
+          table_floats<TAB_SHARED, P>(tab + (c0 >> 1), cs);
+          table_floats<TAB_SHARED, P>(tab + half + (c0 >> 1), sn);
         } else {
 #pragma unroll
           for (int j = 0; j < P; ++j) {
-            cs[j] = __ldg(tab + (c0 >> 1) + j);
-            sn[j] = __ldg(tab + half + (c0 >> 1) + j);
+            cs[j] = TAB_SHARED ? tab[(c0 >> 1) + j] : __ldg(tab + (c0 >> 1) + j);
+            sn[j] = TAB_SHARED ? tab[half + (c0 >> 1) + j] : __ldg(tab + half + (c0 >> 1) + j);
           }
         }
 #pragma unroll

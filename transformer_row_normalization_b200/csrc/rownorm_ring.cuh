@@ -1,14 +1,16 @@
 // Per-warp bulk-copy row rings (sm_100a), for rows whose lane groups fit in
 // one warp (dim <= 1024) in 16-byte aligned layouts: RMSNorm, LayerNorm, and
-// the q/k head RMSNorm + RoPE whose plane partners are the same thread's.
+// the q/k head RMSNorm + RoPE whose plane partners are the same thread's
+// (with each tile's token's cos / sin row staged beside the tile's rows).
 //
 // Every warp of a block runs its own pipeline, with no block barrier: a ring
 // of S stages in shared memory, each holding one tile of R consecutive rows
 // of the warp's static share of the row space (tiles w, w + W, w + 2W, ...
-// for warp w of W). Lane 0 fills a stage with the bulk-copy engine
+// for warp w of W). The warp fills a stage with the bulk-copy engine
 // (cp.async.bulk global -> shared, completion counted in bytes on the
-// stage's mbarrier): one copy for a tile whose rows are adjacent in memory,
-// else one copy per row. The warp waits for the stage, its lane groups
+// stage's mbarrier, announced by lane 0): one copy for a tile whose rows are
+// adjacent in memory, else one copy per row, lane i copying row i. The warp
+// waits for the stage, its lane groups
 // normalize the tile's rows from shared memory and store them to global
 // memory, and lane 0 refills the stage with the tile S ahead. So S tiles of
 // every warp are in flight while it computes, independently of its register
@@ -59,6 +61,8 @@ struct RingParams {
   unsigned long long drain_ns;  // limit of the wait for copies in flight after a timeout
   int tx_extra;        // bytes announced beyond the copies' (0; > 0 only under the
                        // wait test, so that no stage completes and every wait runs out)
+  int table_bytes;     // RoPE rows: bytes of the token's table row staged after a
+                       // tile's rows (every tile lies in one token); 0: not staged
 };
 
 // Shared memory of a block: the warps' rings, then their barrier slots.
@@ -194,22 +198,40 @@ struct AffineRegs {
 
 // Lane 0: start the copies of tile `tile` of row space s (R rows per tile)
 // into `dst`, counted on `bar`.
+// The warp starts the copies of tile `tile` of row space s (R rows per tile)
+// into `dst`, counted on `bar`: lane 0 announces the bytes, then one copy for
+// adjacent rows, else lane i copies row i (rows i + 32, ... too). Rows sit
+// `pitch` 16-byte words apart in the stage: their own size. (Padding rows of
+// under 8 lanes against shared-memory bank conflicts, which then takes a
+// copy per row, measured slower on B200: dual head norm prefill 30.7 ->
+// 33.5 us.)
 template <typename T>
 __device__ __forceinline__ void ring_issue(const Segment& s, long long tile, int R,
-                                           bool contiguous, int tx_extra, uint4* dst,
-                                           uint64_t* bar) {
+                                           bool contiguous, int pitch, int tx_extra,
+                                           int table_bytes, uint4* dst, uint64_t* bar) {
+  const int lane = threadIdx.x & 31;
   const long long r0 = tile * R;
-  const long long nr = s.rows - r0 < R ? s.rows - r0 : R;
+  const int nr = (int)(s.rows - r0 < R ? s.rows - r0 : R);
   const uint32_t row_bytes = (uint32_t)s.dim * (uint32_t)sizeof(T);
   const T* x = static_cast<const T*>(s.x);
-  mbar_expect_tx(bar, (uint32_t)nr * row_bytes + (uint32_t)tx_extra);
+  if (lane == 0) {
+    mbar_expect_tx(bar, (uint32_t)nr * row_bytes + (uint32_t)table_bytes + (uint32_t)tx_extra);
+    if (table_bytes) {
+      // the tile's token's cos / sin row, after the tile's R row slots
+      const long long token = r0 / s.rope_heads;
+      bulk_load(dst + R * pitch, s.rope_table + (s.rope_offset + token) * s.rope_dims,
+                (uint32_t)table_bytes, bar);
+    }
+  }
   if (contiguous) {
-    bulk_load(dst, x + row_off(r0, s.x_stride, s.x_inner, s.x_outer), (uint32_t)nr * row_bytes,
-              bar);
+    if (lane == 0)
+      bulk_load(dst, x + row_off(r0, s.x_stride, s.x_inner, s.x_outer),
+                (uint32_t)nr * row_bytes, bar);
   } else {
-    for (long long rr = 0; rr < nr; ++rr)
-      bulk_load(dst + rr * (row_bytes / 16),
-                x + row_off(r0 + rr, s.x_stride, s.x_inner, s.x_outer), row_bytes, bar);
+    __syncwarp();  // the bytes are announced before any of these copies starts
+    for (int rr = lane; rr < nr; rr += 32)
+      bulk_load(dst + rr * pitch, x + row_off(r0 + rr, s.x_stride, s.x_inner, s.x_outer),
+                row_bytes, bar);
   }
 }
 
@@ -221,9 +243,10 @@ __device__ __forceinline__ void ring_issue(const Segment& s, long long tile, int
 // (indexed from the shared array itself, so that the loads use 32-bit
 // shared-window addresses).
 template <typename T, int OP, int SLOTS, int VPL, int GC, typename Src>
-__device__ __forceinline__ void ring_tile_rows(const Segment& s, int stage_word, long long r0,
-                                               int nr, float eps, float inv_d, int gl, int gi,
-                                               unsigned mask, const Src& src) {
+__device__ __forceinline__ void ring_tile_rows(const Segment& s, int stage_word, int pitch,
+                                               long long r0, int nr, float eps, float inv_d,
+                                               int gl, int gi, unsigned mask, const Src& src,
+                                               int table_word) {
   constexpr int P = Elem<T>::P;
   const int G = GC ? GC : s.lanes;
   auto reduce = [&](float t) {
@@ -236,11 +259,10 @@ __device__ __forceinline__ void ring_tile_rows(const Segment& s, int stage_word,
       return group_sum(t, G, mask);
     }
   };
-  const int row_words = s.dim * (int)sizeof(T) / 16;
 #pragma unroll 1
   for (int rr = gi; rr < nr; rr += 32 / G) {
     const Row<T> g = row_geometry<T, true>(s, r0 + rr);
-    const int row = stage_word + rr * row_words;
+    const int row = stage_word + rr * pitch;
     F2 v[VPL][P];
 #pragma unroll
     for (int q = 0; q < VPL; ++q) {
@@ -257,10 +279,16 @@ __device__ __forceinline__ void ring_tile_rows(const Segment& s, int stage_word,
     float xe = 0.f, rstd, mean;
     row_stats<T, OP, true, SLOTS, VPL>(v, xe, g, inv_d, gl, G, K, eps, false, reduce, rstd,
                                        mean);
-    if constexpr (OP == kOpRmsRopeLocal)
-      normalize_rope_store<T, true, true, SLOTS, VPL>(s, g, v, xe, src, gl, G, rstd, false,
-                                                      r0 + rr, nullptr, mask);
-    else
+    if constexpr (OP == kOpRmsRopeLocal) {
+      if (table_word >= 0)
+        normalize_rope_store<T, true, true, SLOTS, VPL, Src, true>(
+            s, g, v, xe, src, gl, G, rstd, false, r0 + rr, nullptr, mask,
+            reinterpret_cast<const float*>(dyn_smem + table_word));
+      else
+        normalize_rope_store<T, true, true, SLOTS, VPL>(s, g, v, xe, src, gl, G, rstd, false,
+                                                        r0 + rr, nullptr, mask);
+    } else
+
       normalize_store<T, OP, true, SLOTS, VPL>(s, g, v, xe, src, gl, G, rstd, mean, false);
   }
 }
@@ -277,7 +305,10 @@ __device__ __forceinline__ void ring_tile_rows(const Segment& s, int stage_word,
 template <typename T, int OP, int VPL>
 __host__ __device__ constexpr int ring_weight_slots_in_regs() {
   if (OP == kOpRmsRopeLocal) return 0;
-  const int room = (48 - VPL * Elem<T>::V) / (4 * (OP == kOpLn ? 2 : 1));
+#ifndef RN_RING_WB_BUDGET
+#define RN_RING_WB_BUDGET 48
+#endif
+  const int room = (RN_RING_WB_BUDGET - VPL * Elem<T>::V) / (4 * (OP == kOpLn ? 2 : 1));
   return room < 0 ? 0 : (room > VPL ? VPL : room);
 }
 
@@ -326,11 +357,12 @@ __device__ __forceinline__ void ring_segment(const RingParams& p, RingState& rs,
     src = Direct{static_cast<const T*>(s.w), static_cast<const T*>(s.b)};
   int st = rs.st;
   uint32_t parity = rs.parity;
+  const int pitch = s.dim * (int)sizeof(T) / 16;  // a row's 16-byte words
   // every stage is free here: the previous row space's tiles are consumed
-  if (lane == 0) {
+  {
     int k = st;
     for (long long i = 0; i < n && i < S; ++i) {
-      ring_issue<T>(s, w + i * W, R, contiguous, p.tx_extra,
+      ring_issue<T>(s, w + i * W, R, contiguous, pitch, p.tx_extra, p.table_bytes,
                     dyn_smem + ring_word + k * stage_words, &bars[k]);
       k = k + 1 == S ? 0 : k + 1;
     }
@@ -349,17 +381,18 @@ __device__ __forceinline__ void ring_segment(const RingParams& p, RingState& rs,
     const long long r0 = (w + i * W) * R;
     const int nr = (int)(s.rows - r0 < R ? s.rows - r0 : R);
     const int stage_word = ring_word + st * stage_words;
+    const int table_word = p.table_bytes ? stage_word + R * pitch : -1;
     if (G == 32)
-      ring_tile_rows<T, OP, SLOTS, VPL, 32>(s, stage_word, r0, nr, p.eps, inv_d, gl, gi, mask,
-                                            src);
+      ring_tile_rows<T, OP, SLOTS, VPL, 32>(s, stage_word, pitch, r0, nr, p.eps, inv_d, gl, gi,
+                                            mask, src, table_word);
     else
-      ring_tile_rows<T, OP, SLOTS, VPL, 0>(s, stage_word, r0, nr, p.eps, inv_d, gl, gi, mask,
-                                           src);
+      ring_tile_rows<T, OP, SLOTS, VPL, 0>(s, stage_word, pitch, r0, nr, p.eps, inv_d, gl, gi,
+                                           mask, src, table_word);
     // every lane has read the stage: refill it with the tile S ahead
     __syncwarp();
-    if (lane == 0 && i + S < n) {
+    if (i + S < n) {
       fence_async_shared();
-      ring_issue<T>(s, w + (i + S) * W, R, contiguous, p.tx_extra,
+      ring_issue<T>(s, w + (i + S) * W, R, contiguous, pitch, p.tx_extra, p.table_bytes,
                     dyn_smem + ring_word + st * stage_words, &bars[st]);
     }
     st = st + 1 == S ? 0 : st + 1;
