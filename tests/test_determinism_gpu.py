@@ -162,10 +162,12 @@ def test_ring_strided_and_block_views():
         for path in (1, 2):
             rn.set_path_override(path)
             assert rn.plan(rn.RN_OP_RMS, x, weight=w)["staged"] == path - 1
-            res[path] = (rn.rms_norm(x, w, 1e-6), rn.rms_norm(heads, wh, 1e-6))
+            res[path] = (rn.rms_norm(x, w, 1e-6), rn.rms_norm(heads, wh, 1e-6),
+                         rn.layer_norm(x, w, None, 1e-5))
     finally:
         rn.set_path_override(0)
-    assert torch.equal(res[1][0], res[2][0]) and torch.equal(res[1][1], res[2][1])
+    for a, b in zip(res[1], res[2]):
+        assert torch.equal(a, b)
     assert rn.device_error_count(reset=True) == 0
 
 
@@ -209,7 +211,8 @@ def test_ring_waits_run_out_and_the_context_survives(dim):
 
 def test_ring_plans_for_the_large_workloads():
     """By default warp rings carry aligned bf16 lane-group rows that fill a
-    warp (the narrow LayerNorm widths) and the bf16 dual head norm; block
+    warp (the narrow LayerNorm widths, two rows to a tile) and the bf16 dual
+    head norm; block
     rings carry blocks of 512+ threads (D = 16384); the rest keep the
     register kernels unless the rings are forced."""
     for dim, ring in ((768, 1), (1000, 1), (4096, 0), (8192, 0), (16384, 1), (4097, 0)):
@@ -218,6 +221,8 @@ def test_ring_plans_for_the_large_workloads():
         assert p["staged"] == ring, (dim, p)
         if ring:
             assert p["stages"] >= 2 and p["stage_bytes"] >= 2 * dim, p
+        if dim in (768, 1000):  # whole-warp LayerNorm rows: two to a tile, 3 stages
+            assert p["stage_bytes"] == 2 * 2 * dim and p["stages"] == 3, p
     q = torch.empty(8192 * 32, 128, dtype=torch.bfloat16, device="cuda")
     k = torch.empty(8192 * 8, 128, dtype=torch.bfloat16, device="cuda")
     w = torch.ones(128, dtype=torch.bfloat16, device="cuda")

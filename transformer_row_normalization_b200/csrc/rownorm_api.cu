@@ -397,6 +397,16 @@ constexpr int kRingTileBytes = RN_RING_TILE_BYTES;
 #define RN_RING_STAGES 4
 #endif
 constexpr int kRingStages = RN_RING_STAGES;
+// LayerNorm rows of a whole warp go two to a tile when two fit in
+// rn::kRingPairTileBytes (ring_ln_pair normalizes them together), with this
+// many stages.
+// Measured on B200 (bf16, 65536 rows, cold / back to back, us): D = 768
+// 40.9 / 37.0 -> 37.0 / 38.5, D = 1000 55.4 / 53.3 -> 48.0 / 50.2, D = 1024
+// 51.2 / 49.3 -> 49.2 / 50.0; two stages ran faster cold still (768: 36.9)
+// but slower back to back (1000: 51.7), four slower back to back at 768
+// (39.6). RMSNorm rows measured mixed in pairs (1024: 41.0 -> 44.9 cold,
+// 51.6 -> 50.3 back to back) and stay one to a tile.
+constexpr int kRingPairStages = 3;
 
 int round_up(int64_t v, int64_t m) { return (int)((v + m - 1) / m * m); }
 
@@ -438,11 +448,16 @@ bool plan_ring(int dtype, int op, const SegPlan* plans, const rn_view* const* xs
   const int es = elem_size(dtype);
   int64_t stage_bytes = 16;
   int64_t tiles_max = 1;
+  bool paired = false;
   for (int i = 0; i < nseg; ++i) {
     const int64_t row_bytes = xs[i]->dim * es;
     const int64_t per = 32 / plans[i].lanes;  // rows a warp takes at once
     int64_t rounds = kRingTileBytes / (per * row_bytes);
     if (rounds < 1) rounds = 1;
+    if (op == rn::kOpLn && per == 1 && rounds < 2 && rn::ring_pairs_fit(chunks)) {
+      rounds = 2;
+      paired = true;
+    }
     const int64_t tr = per * rounds;
     l.tile_rows[i] = (int)tr;
     l.contiguous[i] = !two_level(xs[i]) && (xs[i]->rows <= 1 || xs[i]->row_stride == xs[i]->dim);
@@ -470,8 +485,12 @@ bool plan_ring(int dtype, int op, const SegPlan* plans, const rn_view* const* xs
   }
   l.stage_bytes = round_up(stage_bytes, 16);
   const DeviceInfo di = device_info(dev);
-  int stages = kRingStages;
-  while (stages > 2 && rn::ring_smem_bytes(stages, l.stage_bytes) > di.smem_per_block - 1024)
+  int stages = paired ? kRingPairStages : kRingStages;
+  // as many stages as keep kRingBlocksPerSm blocks on an SM (1 KB of each
+  // block's shared memory is the system's)
+  while (stages > 2 && (rn::ring_smem_bytes(stages, l.stage_bytes) > di.smem_per_block - 1024 ||
+                        rn::kRingBlocksPerSm * (rn::ring_smem_bytes(stages, l.stage_bytes) + 1024) >
+                            di.smem_per_sm))
     --stages;
   if (rn::ring_smem_bytes(stages, l.stage_bytes) > di.smem_per_block - 1024) return false;
   l.stages = stages;

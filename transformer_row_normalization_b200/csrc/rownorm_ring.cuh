@@ -132,11 +132,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-// Weight and bias of a lane's chunk slots held in registers as their packed
-// 16-byte words (loaded once per row space: in an aligned layout a lane owns
-// the same chunks of every row), unpacked at each use. NULL weight = ones,
-// NULL bias = zeros, as AffineDirect; the values, and so the bits, are the
-// same.
 // Weight and bias of a lane's chunk slots: the packed 16-byte words of the
 // first NREG slots held in registers (loaded once per row space: in an
 // aligned layout a lane owns the same chunks of every row), the others read
@@ -196,8 +191,6 @@ struct AffineRegs {
   }
 };
 
-// Lane 0: start the copies of tile `tile` of row space s (R rows per tile)
-// into `dst`, counted on `bar`.
 // The warp starts the copies of tile `tile` of row space s (R rows per tile)
 // into `dst`, counted on `bar`: lane 0 announces the bytes, then one copy for
 // adjacent rows, else lane i copies row i (rows i + 32, ... too). Rows sit
@@ -235,6 +228,83 @@ __device__ __forceinline__ void ring_issue(const Segment& s, long long tile, int
   }
 }
 
+// LayerNorm rows of a whole warp go two to a ring tile when two rows fit in
+// kRingPairTileBytes (the planner decides; ring_ln_pair normalizes them
+// together). Lanes of more chunks never pair, and their kernels carry no
+// pair code (it would only add to their register pressure).
+constexpr int kRingPairTileBytes = 4096;
+__host__ __device__ constexpr bool ring_pairs_fit(int vpl) {
+  return 2 * 32 * 16 * vpl <= kRingPairTileBytes;
+}
+
+// The xor butterfly of two rows' partial sums at once over the whole warp:
+// each step adds the partner lane's pair with one packed add, which rounds
+// each half as the scalar add of the one-row butterfly does.
+__device__ __forceinline__ F2 warp_sum_pair(F2 t) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    F2 u;
+    u.x = __shfl_xor_sync(0xffffffffu, t.x, off);
+    u.y = __shfl_xor_sync(0xffffffffu, t.y, off);
+    t = add2(t, u);
+  }
+  return t;
+}
+
+// Two whole-warp LayerNorm rows of a stage at once: rows r and r + 1, at
+// 16-byte words `row` and `row + pitch`. Each row takes the operations of
+// one row, in the same order (row_stats, normalize_store), so its bits are
+// those of the one-row path; the two rows' independent chains interleave,
+// their butterflies share each step's add, and each weight / bias word is
+// read and unpacked once for both rows.
+template <typename T, int SLOTS, int VPL, typename Src>
+__device__ __forceinline__ void ring_ln_pair(const Segment& s, int row, int pitch, long long r,
+                                             float eps, float inv_d, int gl, const Src& src) {
+  constexpr int P = Elem<T>::P;
+  constexpr int V = Elem<T>::V;
+  const Row<T> ga = row_geometry<T, true>(s, r);
+  const Row<T> gb = row_geometry<T, true>(s, r + 1);
+  F2 va[VPL][P], vb[VPL][P];
+#pragma unroll
+  for (int q = 0; q < VPL; ++q) {
+    if (slot_present<SLOTS, VPL>(q, gl + 32 * q, ga.nfull)) {
+      Elem<T>::unpack(dyn_smem[row + gl + 32 * q], va[q]);
+      Elem<T>::unpack(dyn_smem[row + pitch + gl + 32 * q], vb[q]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < P; ++j) va[q][j] = vb[q][j] = zero2();
+    }
+  }
+  // each row's first element, from the first 4 bytes of its first chunk
+  const uint32_t* words = reinterpret_cast<const uint32_t*>(dyn_smem);
+  const float Ka = Elem<T>::low(words[4 * row]);
+  const float Kb = Elem<T>::low(words[4 * (row + pitch)]);
+  float xe = 0.f;  // no edge elements in these layouts
+  F2 s1 = make_float2(shift_and_sum<T, true, SLOTS, VPL>(va, xe, ga, gl, 32, Ka, false),
+                      shift_and_sum<T, true, SLOTS, VPL>(vb, xe, gb, gl, 32, Kb, false));
+  s1 = warp_sum_pair(s1);
+  const float ma = __fmul_rn(s1.x, inv_d), mb = __fmul_rn(s1.y, inv_d);
+  F2 s2 = make_float2(sum_dev_squares<T, true, SLOTS, VPL>(va, xe, ga, gl, 32, ma, false),
+                      sum_dev_squares<T, true, SLOTS, VPL>(vb, xe, gb, gl, 32, mb, false));
+  s2 = warp_sum_pair(s2);
+  const F2 Ra = splat(rsqrtf(__fadd_rn(__fmul_rn(s2.x, inv_d), eps)));
+  const F2 Rb = splat(rsqrtf(__fadd_rn(__fmul_rn(s2.y, inv_d), eps)));
+#pragma unroll
+  for (int q = 0; q < VPL; ++q) {
+    const int f = gl + 32 * q;
+    if (!slot_present<SLOTS, VPL>(q, f, ga.nfull)) continue;
+    F2 wf[P], bf[P], oa[P], ob[P];
+    src.get(q, f, wf, bf);
+#pragma unroll
+    for (int j = 0; j < P; ++j) {  // the rows are centred
+      oa[j] = fma2(mul2(va[q][j], Ra), wf[j], bf[j]);
+      ob[j] = fma2(mul2(vb[q][j], Rb), wf[j], bf[j]);
+    }
+    store_stream(ga.y_row + (long long)f * V, Elem<T>::pack(oa));
+    store_stream(gb.y_row + (long long)f * V, Elem<T>::pack(ob));
+  }
+}
+
 // The rows of one staged tile (rows r0 .. r0 + nr - 1), normalized by the
 // warp's lane groups: lane group gi takes rows gi, gi + 32/G, ... GC = 32
 // compiles the whole-warp case (one row at a time, a fixed butterfly); GC =
@@ -259,8 +329,14 @@ __device__ __forceinline__ void ring_tile_rows(const Segment& s, int stage_word,
       return group_sum(t, G, mask);
     }
   };
+  int rr = gi;
+  if constexpr (GC == 32 && OP == kOpLn && ring_pairs_fit(VPL)) {
 #pragma unroll 1
-  for (int rr = gi; rr < nr; rr += 32 / G) {
+    for (; rr + 1 < nr; rr += 2)
+      ring_ln_pair<T, SLOTS, VPL>(s, stage_word + rr * pitch, pitch, r0 + rr, eps, inv_d, gl, src);
+  }
+#pragma unroll 1
+  for (; rr < nr; rr += 32 / G) {
     const Row<T> g = row_geometry<T, true>(s, r0 + rr);
     const int row = stage_word + rr * pitch;
     F2 v[VPL][P];
@@ -287,24 +363,25 @@ __device__ __forceinline__ void ring_tile_rows(const Segment& s, int stage_word,
       else
         normalize_rope_store<T, true, true, SLOTS, VPL>(s, g, v, xe, src, gl, G, rstd, false,
                                                         r0 + rr, nullptr, mask);
-    } else
-
+    } else {
       normalize_store<T, OP, true, SLOTS, VPL>(s, g, v, xe, src, gl, G, rstd, mean, false);
+    }
   }
 }
 
-// Weight and bias in registers (AffineRegs) for lanes of up to 3 chunks when
-// the op needs no other per-element tables; otherwise read from L1 per row
-// (AffineDirect). Beyond that, the values held across the row spill under
-// the 128-register budget (ptxas).
-// Slots whose weight (and bias) words stay in registers: as many as keep a
-// lane's row values (VPL chunks as binary32) plus those words within 48
-// registers, so that the kernel fits the 128-register budget without
-// spilling (ptxas, both element types); none for RoPE rows, which also hold
-// their cos / sin values.
+// Slots whose weight (and bias) words stay in registers (AffineRegs; the
+// others are read from L1 at each use): as many as keep a lane's row values
+// (VPL chunks as binary32) plus those words within 48 registers, so that the
+// kernel fits the 128-register budget without spilling (ptxas, both element
+// types); none for RoPE rows, which also hold their cos / sin values, nor for
+// LayerNorm rows.
 template <typename T, int OP, int VPL>
 __host__ __device__ constexpr int ring_weight_slots_in_regs() {
   if (OP == kOpRmsRopeLocal) return 0;
+  // LayerNorm rows of a whole warp run in pairs (ring_ln_pair): two rows'
+  // values leave no room (ptxas spilled), and each weight / bias word read
+  // from L1 serves both rows
+  if (OP == kOpLn) return 0;
 #ifndef RN_RING_WB_BUDGET
 #define RN_RING_WB_BUDGET 48
 #endif
