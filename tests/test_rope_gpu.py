@@ -139,3 +139,25 @@ def test_bitwise_repeatable_across_grids():
             assert torch.equal(y[0], base[0]) and torch.equal(y[1], base[1]), grid
     finally:
         rn.set_grid_override(0)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("trad", [False, True], ids=["split", "interleaved"])
+@pytest.mark.parametrize("tokens,hq,hk,offset", [(1, 32, 8, 0), (3, 32, 8, 7), (301, 32, 8, 100),
+                                                 (64, 8, 2, 5), (17, 16, 4, 0)])
+def test_ring_and_register_rope_agree_bitwise(dtype, trad, tokens, hq, hk, offset):
+    """The bulk-copy rings (table row staged with tiles of whole lane-group
+    rounds inside one token where the head counts allow it, else read from
+    global memory) give the register kernels' bits."""
+    q, k, wq, wk = inputs(tokens, hq, hk, 128, dtype, seed=tokens + hq)
+    table = rn.rope_table(128, offset + tokens + 1, device="cuda")
+    res = {}
+    try:
+        for path in (1, 2):
+            rn.set_path_override(path)
+            res[path] = rn.dual_head_rms_norm_rope(q, k, wq, wk, 1e-6, table, offset, 128,
+                                                   heads_q=hq, heads_k=hk, traditional=trad)
+    finally:
+        rn.set_path_override(0)
+    assert torch.equal(res[1][0], res[2][0]) and torch.equal(res[1][1], res[2][1])
+    assert rn.device_error_count(reset=True) == 0

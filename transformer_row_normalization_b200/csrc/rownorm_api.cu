@@ -407,6 +407,14 @@ constexpr int kRingStages = RN_RING_STAGES;
 // (39.6). RMSNorm rows measured mixed in pairs (1024: 41.0 -> 44.9 cold,
 // 51.6 -> 50.3 back to back) and stay one to a tile.
 constexpr int kRingPairStages = 3;
+// RoPE tiles (table row staged): whole lane-group rounds of one token, up
+// to this many bytes of rows. Measured on B200 (bf16 dual head norm + RoPE,
+// 8192 tokens of 32 + 8 heads of 128, cold / back to back, us): tiles of 8 q
+// rows 45.9 / 41.0, 16 rows 43.0 / 37.6, 32 rows 43.0 / 40.3.
+#ifndef RN_RING_ROPE_TILE_BYTES
+#define RN_RING_ROPE_TILE_BYTES 4096
+#endif
+constexpr int kRingRopeTileBytes = RN_RING_ROPE_TILE_BYTES;
 
 int round_up(int64_t v, int64_t m) { return (int)((v + m - 1) / m * m); }
 
@@ -420,10 +428,17 @@ int round_up(int64_t v, int64_t m) { return (int)((v + m - 1) / m * m); }
 //   but bf16 LayerNorm 512 (16 lanes per row) 31.8 -> 34.7 us and binary32
 //   LayerNorm 1024 88.1 -> 94.1 us ran slower, and stay on the register
 //   kernels.
-//   The dual head norm + RoPE also ran slower in rings (47.1 -> 53.2 us), so
-//   the rings take it only when forced.
-bool ring_preferred(int dtype, int op, const SegPlan* plans, int nseg) {
-  if (dtype != RN_BF16 || (op != rn::kOpRms && op != rn::kOpLn)) return false;
+//   The bf16 dual head norm + split-half RoPE (same shapes) runs in rings
+//   when each tile's token's table row can be staged with the tile (tiles of
+//   16 q rows: 43.0 -> 39.1 us cold, 41.0 -> 37.0 back to back); with the
+//   table read from global memory per row the rings ran slower (47.1 ->
+//   53.2 us), and interleaved planes are not measured: both stay on the
+//   register kernels unless the rings are forced (plan_ring checks the
+//   staging).
+bool ring_preferred(int dtype, int op, const SegPlan* plans, int nseg, const rn_rope* rope) {
+  if (dtype != RN_BF16) return false;
+  if (op == rn::kOpRmsRopeLocal) return nseg == 2 && rope && !rope->traditional;
+  if (op != rn::kOpRms && op != rn::kOpLn) return false;
   if (nseg == 2) return true;
   return plans[0].lanes == 32;
 }
@@ -439,7 +454,7 @@ bool plan_ring(int dtype, int op, const SegPlan* plans, const rn_view* const* xs
   if (op != rn::kOpRms && op != rn::kOpLn && op != rn::kOpRmsRopeLocal) return false;
   for (int i = 0; i < nseg; ++i)
     if (plans[i].family != 0 || !plans[i].exact) return false;
-  if (path == 0 && !ring_preferred(dtype, op, plans, nseg)) return false;
+  if (path == 0 && !ring_preferred(dtype, op, plans, nseg, rope)) return false;
   const void* fn = dtype == RN_F32 ? rn::ring_kernel_f32(op, slots, chunks)
                                    : rn::ring_kernel_bf16(op, slots, chunks);
   if (!fn) return false;
@@ -457,6 +472,16 @@ bool plan_ring(int dtype, int op, const SegPlan* plans, const rn_view* const* xs
     if (op == rn::kOpLn && per == 1 && rounds < 2 && rn::ring_pairs_fit(chunks)) {
       rounds = 2;
       paired = true;
+    }
+    if (op == rn::kOpRmsRopeLocal && rope && rope->table && nseg == 2) {
+      // tiles of whole lane-group rounds inside one token, as large as fit
+      // kRingRopeTileBytes: the table row staged with the tile serves every
+      // row a lane takes from it
+      const int64_t heads = i == 0 ? rope->heads_q : rope->heads_k;
+      int64_t best = 0;
+      for (int64_t rd = 1; per * rd * row_bytes <= kRingRopeTileBytes; ++rd)
+        if (heads % (per * rd) == 0) best = rd;
+      if (best) rounds = best;
     }
     const int64_t tr = per * rounds;
     l.tile_rows[i] = (int)tr;
@@ -483,6 +508,7 @@ bool plan_ring(int dtype, int op, const SegPlan* plans, const rn_view* const* xs
       stage_bytes = sb;
     }
   }
+  if (path == 0 && op == rn::kOpRmsRopeLocal && l.table_bytes == 0) return false;
   l.stage_bytes = round_up(stage_bytes, 16);
   const DeviceInfo di = device_info(dev);
   int stages = paired ? kRingPairStages : kRingStages;

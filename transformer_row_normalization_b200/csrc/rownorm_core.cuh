@@ -706,6 +706,57 @@ __device__ __forceinline__ void store_chunk(const Segment& s, T* yc, const F2 (&
   }
 }
 
+// Split-half planes of one chunk pair held by the thread: a (columns c0 ..
+// c0 + V - 1 of the first half) and b (its partner chunk, `half` columns
+// on), rotated by their columns' cos / sin and stored: packed pairs of
+// planes, y_a = fma(a, cos, -(b sin)), y_b = fma(b, cos, a sin).
+template <typename T>
+__device__ __forceinline__ void rotate_split_store(const Segment& s, T* yc, int half,
+                                                   const F2 (&a)[Elem<T>::P],
+                                                   const F2 (&b)[Elem<T>::P],
+                                                   const float (&cs)[Elem<T>::V],
+                                                   const float (&sn)[Elem<T>::V], bool vstore) {
+  constexpr int P = Elem<T>::P;
+  F2 ya[P], yb[P];
+#pragma unroll
+  for (int j = 0; j < P; ++j) {
+    const F2 c = make2(cs[2 * j], cs[2 * j + 1]), sn2 = make2(sn[2 * j], sn[2 * j + 1]);
+    const F2 bs = mul2(b[j], sn2), as = mul2(a[j], sn2);
+    ya[j] = fma2(a[j], c, make2(-bs.x, -bs.y));
+    yb[j] = fma2(b[j], c, as);
+  }
+  store_chunk<T>(s, yc, ya, vstore);
+  store_chunk<T>(s, yc + half, yb, vstore);
+}
+
+// The split-half in-thread RoPE path of normalize_rope_store (full rotary,
+// every slot present, EXACT rows) with the thread's cos / sin already in
+// registers: cs[p] / sn[p] for its first-half slot p. For several rows of
+// one token whose angles the caller loaded once; the operations are those
+// of normalize_rope_store, so the bits are too.
+template <typename T, int NSLOT, typename Src>
+__device__ __forceinline__ void normalize_rope_split_pre(
+    const Segment& s, const Row<T>& g, F2 (&v)[NSLOT][Elem<T>::P], const Src& src, int k0,
+    int step, float rstd, const float (&cs)[NSLOT / 2][Elem<T>::V],
+    const float (&sn)[NSLOT / 2][Elem<T>::V]) {
+  static_assert(NSLOT % 2 == 0, "chunk pairs");
+  constexpr int V = Elem<T>::V;
+  constexpr int P = Elem<T>::P;
+  const int half = s.rope_dims >> 1;
+  const F2 R2 = splat(rstd);
+#pragma unroll
+  for (int p = 0; p < NSLOT; ++p) {
+    F2 wf[P], bf[P];
+    src.get(p, k0 + step * p, wf, bf);
+#pragma unroll
+    for (int j = 0; j < P; ++j) v[p][j] = mul2(mul2(v[p][j], R2), wf[j]);
+  }
+#pragma unroll
+  for (int p = 0; p < NSLOT / 2; ++p)
+    rotate_split_store<T>(s, g.y_row + (k0 + step * p) * V, half, v[p], v[p + NSLOT / 2], cs[p],
+                          sn[p], true);
+}
+
 // The row's cos / sin come from the table in global memory, or (TAB_SHARED,
 // in-thread planes only) from `tab_shared`: a copy of the row's table row
 // that the caller staged in shared memory.
@@ -760,18 +811,7 @@ __device__ __forceinline__ void normalize_rope_store(const Segment& s, const Row
         float cs[V], sn[V];
         table_floats<TAB_SHARED, V>(tab + c0, cs);
         table_floats<TAB_SHARED, V>(tab + half + c0, sn);
-        F2 ya[P], yb[P];
-#pragma unroll
-        for (int j = 0; j < P; ++j) {
-          // packed pairs of planes: y_a = fma(a, cos, -(b sin)), y_b = fma(b, cos, a sin)
-          const F2 a = v[p][j], b = v[p + NSLOT / 2][j];
-          const F2 c = make2(cs[2 * j], cs[2 * j + 1]), sn2 = make2(sn[2 * j], sn[2 * j + 1]);
-          const F2 bs = mul2(b, sn2), as = mul2(a, sn2);
-          ya[j] = fma2(a, c, make2(-bs.x, -bs.y));
-          yb[j] = fma2(b, c, as);
-        }
-        store_chunk<T>(s, g.y_row + c0, ya, vstore);
-        store_chunk<T>(s, g.y_row + c0 + half, yb, vstore);
+        rotate_split_store<T>(s, g.y_row + c0, half, v[p], v[p + NSLOT / 2], cs, sn, vstore);
       }
       return;
     }

@@ -330,6 +330,35 @@ __device__ __forceinline__ void ring_tile_rows(const Segment& s, int stage_word,
     }
   };
   int rr = gi;
+  if constexpr (OP == kOpRmsRopeLocal && VPL % 2 == 0) {
+    if (table_word >= 0 && !s.rope_trad) {
+      // full split-half rotary, the tile's token's table row staged beside
+      // its rows: the lane's cos / sin, the same for every row it takes
+      // here, are read once per tile
+      constexpr int V = Elem<T>::V;
+      const float* tab = reinterpret_cast<const float*>(dyn_smem + table_word);
+      const int half = s.rope_dims >> 1;
+      float cs[VPL / 2][V], sn[VPL / 2][V];
+#pragma unroll
+      for (int q = 0; q < VPL / 2; ++q) {
+        load_floats<V>(tab + (gl + G * q) * V, cs[q]);
+        load_floats<V>(tab + half + (gl + G * q) * V, sn[q]);
+      }
+#pragma unroll 1
+      for (; rr < nr; rr += 32 / G) {
+        const Row<T> g = row_geometry<T, true>(s, r0 + rr);
+        const int row = stage_word + rr * pitch;
+        F2 v[VPL][P];
+#pragma unroll
+        for (int q = 0; q < VPL; ++q) Elem<T>::unpack(dyn_smem[row + gl + G * q], v[q]);
+        float xe = 0.f, rstd, mean;
+        row_stats<T, OP, true, SLOTS, VPL>(v, xe, g, inv_d, gl, G, 0.f, eps, false, reduce, rstd,
+                                           mean);
+        normalize_rope_split_pre<T, VPL>(s, g, v, src, gl, G, rstd, cs, sn);
+      }
+      return;
+    }
+  }
   if constexpr (GC == 32 && OP == kOpLn && ring_pairs_fit(VPL)) {
 #pragma unroll 1
     for (; rr + 1 < nr; rr += 2)
@@ -459,7 +488,12 @@ __device__ __forceinline__ void ring_segment(const RingParams& p, RingState& rs,
     const int nr = (int)(s.rows - r0 < R ? s.rows - r0 : R);
     const int stage_word = ring_word + st * stage_words;
     const int table_word = p.table_bytes ? stage_word + R * pitch : -1;
-    if (G == 32)
+    // (head rows with RoPE keep one copy of the row code, with the lane
+    // count read at run time: without the second, whole-warp copy the dual
+    // head norm + RoPE prefill ran 43.0 -> 39.1 us cold, 37.6 -> 37.0 back to
+    // back on B200, where ncu had counted 1.45 cycles per issue stalled on
+    // instruction fetch)
+    if (OP != kOpRmsRopeLocal && G == 32)
       ring_tile_rows<T, OP, SLOTS, VPL, 32>(s, stage_word, pitch, r0, nr, p.eps, inv_d, gl, gi,
                                             mask, src, table_word);
     else
