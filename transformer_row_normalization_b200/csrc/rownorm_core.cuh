@@ -729,16 +729,40 @@ __device__ __forceinline__ void rotate_split_store(const Segment& s, T* yc, int 
   store_chunk<T>(s, yc + half, yb, vstore);
 }
 
+// rotate_split_store with the negated sines given (nsn = -sn): b (-s) is
+// -(b s) exactly (rounding to nearest is symmetric), so the bits are the
+// same, without a sign flip per element.
+template <typename T>
+__device__ __forceinline__ void rotate_split_store_ns(const Segment& s, T* yc, int half,
+                                                      const F2 (&a)[Elem<T>::P],
+                                                      const F2 (&b)[Elem<T>::P],
+                                                      const float (&cs)[Elem<T>::V],
+                                                      const float (&sn)[Elem<T>::V],
+                                                      const float (&nsn)[Elem<T>::V],
+                                                      bool vstore) {
+  constexpr int P = Elem<T>::P;
+  F2 ya[P], yb[P];
+#pragma unroll
+  for (int j = 0; j < P; ++j) {
+    const F2 c = make2(cs[2 * j], cs[2 * j + 1]);
+    const F2 sn2 = make2(sn[2 * j], sn[2 * j + 1]), nsn2 = make2(nsn[2 * j], nsn[2 * j + 1]);
+    ya[j] = fma2(a[j], c, mul2(b[j], nsn2));
+    yb[j] = fma2(b[j], c, mul2(a[j], sn2));
+  }
+  store_chunk<T>(s, yc, ya, vstore);
+  store_chunk<T>(s, yc + half, yb, vstore);
+}
+
 // The split-half in-thread RoPE path of normalize_rope_store (full rotary,
 // every slot present, EXACT rows) with the thread's cos / sin already in
-// registers: cs[p] / sn[p] for its first-half slot p. For several rows of
-// one token whose angles the caller loaded once; the operations are those
-// of normalize_rope_store, so the bits are too.
+// registers: cs[p] / sn[p] for its first-half slot p, nsn[p] = -sn[p]. For
+// several rows of one token whose angles the caller loaded once; the
+// operations are those of normalize_rope_store, so the bits are too.
 template <typename T, int NSLOT, typename Src>
 __device__ __forceinline__ void normalize_rope_split_pre(
     const Segment& s, const Row<T>& g, F2 (&v)[NSLOT][Elem<T>::P], const Src& src, int k0,
     int step, float rstd, const float (&cs)[NSLOT / 2][Elem<T>::V],
-    const float (&sn)[NSLOT / 2][Elem<T>::V]) {
+    const float (&sn)[NSLOT / 2][Elem<T>::V], const float (&nsn)[NSLOT / 2][Elem<T>::V]) {
   static_assert(NSLOT % 2 == 0, "chunk pairs");
   constexpr int V = Elem<T>::V;
   constexpr int P = Elem<T>::P;
@@ -753,8 +777,8 @@ __device__ __forceinline__ void normalize_rope_split_pre(
   }
 #pragma unroll
   for (int p = 0; p < NSLOT / 2; ++p)
-    rotate_split_store<T>(s, g.y_row + (k0 + step * p) * V, half, v[p], v[p + NSLOT / 2], cs[p],
-                          sn[p], true);
+    rotate_split_store_ns<T>(s, g.y_row + (k0 + step * p) * V, half, v[p], v[p + NSLOT / 2],
+                             cs[p], sn[p], nsn[p], true);
 }
 
 // The row's cos / sin come from the table in global memory, or (TAB_SHARED,
