@@ -645,14 +645,17 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
       merged.family == 0 ? rn::kWarpPrefetchStages : rn::cta_prefetch_stages(threads, op);
   const int pf_bytes = rn::prefetch_slots_smem_bytes(threads, merged.chunks, stages) *
                        (rn::op_has_second(op) ? 2 : 1);
-  // Prefetch of the rows ahead where it measured faster on B200: lane groups and
+  // Prefetch of the rows ahead where it measured faster on B200: lane groups,
   // blocks of 256 or more threads (few blocks per SM, so few rows in
-  // flight); blocks of 128 threads already keep 8+ rows per SM in flight and
-  // ran slower with it. Only when the slots fit beside the weight cache
-  // (with a margin for the kernel's static shared memory).
+  // flight), and blocks of 128 threads on rows off the 16-byte grid (bf16
+  // LayerNorm 65536 x 4097: 203.6 -> 200.0 us cold); aligned rows in blocks
+  // of 128 threads, which keep 8 rows per SM in flight, ran slower with it
+  // (LayerNorm 4096: 174.1 -> 177.0 us). Only when the slots fit beside the
+  // weight cache (with a margin for the kernel's static shared memory).
   const int path = g_path_override.load(std::memory_order_relaxed);
   const bool want_prefetch =
-      path == 3 || (path == 0 && (merged.family == 0 || merged.lanes >= 256));
+      path == 3 ||
+      (path == 0 && (merged.family == 0 || merged.lanes >= 256 || !merged.exact));
   const int prefetch =
       !stream && want_prefetch && cache + pf_bytes <= device_info(dev).smem_per_block - 1024
           ? 1
