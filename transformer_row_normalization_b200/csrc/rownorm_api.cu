@@ -420,27 +420,28 @@ int round_up(int64_t v, int64_t m) { return (int)((v + m - 1) / m * m); }
 
 // Whether the planner uses the per-warp bulk-copy rings by default for these
 // segments (they must qualify, see plan_ring). Measured on B200 against the
-// register lane-group kernels (65536 rows, cold L2, medians):
-//   bf16 rows whose lane groups fill a warp: LayerNorm 768 47.9 -> 38.9 us,
-//     1000 73.8 -> 53.3 us, RMSNorm 1024 51.1 -> 45.0 us;
-//   the bf16 dual head norm (q [8192, 32, 128] and k [8192, 8, 128], 4 lanes
-//     per row): 32.8 -> 30.7 us;
-//   but bf16 LayerNorm 512 (16 lanes per row) 31.8 -> 34.7 us and binary32
-//   LayerNorm 1024 88.1 -> 94.1 us ran slower, and stay on the register
-//   kernels.
-//   The bf16 dual head norm + split-half RoPE (same shapes) runs in rings
-//   when each tile's token's table row can be staged with the tile (tiles of
-//   16 q rows: 43.0 -> 39.1 us cold, 41.0 -> 37.0 back to back); with the
-//   table read from global memory per row the rings ran slower (47.1 ->
-//   53.2 us), and interleaved planes are not measured: both stay on the
-//   register kernels unless the rings are forced (plan_ring checks the
-//   staging).
+// register lane-group kernels with their per-thread prefetch (bf16, 65536
+// rows, cold / back to back, us):
+//   rows whose lane groups fill a warp: LayerNorm 768 45.1 / 45.1 -> 36.9 /
+//     38.4, 1000 61.5 / 62.7 -> 47.1 / 49.8, 1024 52.1 / 51.8 -> 49.1 / 50.0,
+//     RMSNorm 1024 44.9 / 51.6 -> 41.0 / 50.6;
+//   the dual head norm + split-half RoPE (q [8192, 32, 128], k [8192, 8,
+//     128]) with the token's table row staged with each tile: 43.0 / 41.1 ->
+//     36.9 / 35.2; with the table read from global memory per row the rings
+//     ran slower (47.1 -> 53.2 cold), and interleaved planes are not
+//     measured: both stay on the register kernels unless the rings are
+//     forced (plan_ring checks the staging);
+//   but the plain dual head norm (same shapes, 4 lanes per row) 26.7 / 31.2
+//     -> 30.9 / 31.5, bf16 LayerNorm 512 (16 lanes per row) 31.8 -> 34.7
+//     and binary32 LayerNorm 1024 88.1 -> 94.1 ran slower, and stay on the
+//     register kernels.
 bool ring_preferred(int dtype, int op, const SegPlan* plans, int nseg, const rn_rope* rope) {
   if (dtype != RN_BF16) return false;
   if (op == rn::kOpRmsRopeLocal) return nseg == 2 && rope && !rope->traditional;
   if (op != rn::kOpRms && op != rn::kOpLn) return false;
-  if (nseg == 2) return true;
-  return plans[0].lanes == 32;
+  for (int i = 0; i < nseg; ++i)
+    if (plans[i].lanes != 32) return false;
+  return true;
 }
 
 // Plans a ring launch for RMSNorm / LayerNorm segments of the lane-group
