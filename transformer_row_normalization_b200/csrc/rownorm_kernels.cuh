@@ -398,7 +398,7 @@ rows_cta_kernel(const Params p) {
     // rows off the 16-byte grid take a copy picked at run time: with the
     // compile-time reference the off-grid LayerNorm kernel spilled 12 bytes
     // in its row loop at 64 registers (LayerNorm 65536 x 4097: 303 against
-    // 204 us)
+    // 204 us), and ran 332 us at 80 registers (the copy: 199 us at 64 or 80)
 #pragma unroll 1
     for (int si = 0; si < p.nseg; ++si) {
       const Segment s = si == 0 ? p.seg[0] : p.seg[1];
