@@ -383,7 +383,7 @@ struct Launch {
   int ring;         // 1: rows_ring_kernel, 2: rows_cta_ring_kernel (RingParams)
   rn_launch_info info;
   // ring kernels only
-  int stages, stage_bytes, tile_rows[2], contiguous[2], table_bytes;
+  int stages, stage_bytes, tile_rows[2], contiguous[2], table_bytes, affine_word;
   int stage_word;   // kOpRmsRope: staging rows after the slots and the cache
 };
 
@@ -453,6 +453,7 @@ bool plan_ring(int dtype, int op, const SegPlan* plans, const rn_view* const* xs
   const int path = g_path_override.load(std::memory_order_relaxed);
   if (path == 1 || path == 3) return false;
   if (op != rn::kOpRms && op != rn::kOpLn && op != rn::kOpRmsRopeLocal) return false;
+  if (op == rn::kOpLn && nseg != 1) return false;  // one weight / bias area per block
   for (int i = 0; i < nseg; ++i)
     if (plans[i].family != 0 || !plans[i].exact) return false;
   if (path == 0 && !ring_preferred(dtype, op, plans, nseg, rope)) return false;
@@ -512,17 +513,21 @@ bool plan_ring(int dtype, int op, const SegPlan* plans, const rn_view* const* xs
   if (path == 0 && op == rn::kOpRmsRopeLocal && l.table_bytes == 0) return false;
   l.stage_bytes = round_up(stage_bytes, 16);
   const DeviceInfo di = device_info(dev);
+  // LayerNorm rings keep the block's binary32 weight and bias after the
+  // barriers (ring_affine_bytes)
+  const int affine = op == rn::kOpLn ? rn::ring_affine_bytes((int)xs[0]->dim) : 0;
   int stages = paired ? kRingPairStages : kRingStages;
   // as many stages as keep kRingBlocksPerSm blocks on an SM (1 KB of each
   // block's shared memory is the system's)
-  while (stages > 2 && (rn::ring_smem_bytes(stages, l.stage_bytes) > di.smem_per_block - 1024 ||
-                        rn::kRingBlocksPerSm * (rn::ring_smem_bytes(stages, l.stage_bytes) + 1024) >
-                            di.smem_per_sm))
+  auto smem_of = [&](int k) { return rn::ring_smem_bytes(k, l.stage_bytes) + affine; };
+  while (stages > 2 && (smem_of(stages) > di.smem_per_block - 1024 ||
+                        rn::kRingBlocksPerSm * (smem_of(stages) + 1024) > di.smem_per_sm))
     --stages;
-  if (rn::ring_smem_bytes(stages, l.stage_bytes) > di.smem_per_block - 1024) return false;
+  if (smem_of(stages) > di.smem_per_block - 1024) return false;
   l.stages = stages;
   l.fn = fn;
-  l.smem = rn::ring_smem_bytes(stages, l.stage_bytes);
+  l.smem = smem_of(stages);
+  l.affine_word = affine ? rn::ring_smem_bytes(stages, l.stage_bytes) / 16 : -1;
   int bps = 0;
   if (blocks_per_sm(dev, fn, rn::kRingWarps * 32, l.smem, &bps)) return false;
   int64_t grid = (int64_t)sms * bps;
@@ -751,6 +756,7 @@ int launch(const Launch& l, const rn::Params& params, void* stream) {
     rp.drain_ns = wait_test ? 2000000ull : rn::kRingDrainLimitNs;
     rp.tx_extra = wait_test ? 16 : 0;
     rp.table_bytes = l.table_bytes;
+    rp.affine_word = l.affine_word;
     void* args[] = {&rp};
     e = cudaLaunchKernel(l.fn, dim3((unsigned)l.info.grid_blocks),
                          dim3((unsigned)l.info.block_threads), args, (size_t)l.smem,

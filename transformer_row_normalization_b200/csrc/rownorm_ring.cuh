@@ -63,12 +63,17 @@ struct RingParams {
                        // wait test, so that no stage completes and every wait runs out)
   int table_bytes;     // RoPE rows: bytes of the token's table row staged after a
                        // tile's rows (every tile lies in one token); 0: not staged
+  int affine_word;     // LayerNorm rows: 16-byte word of the block's binary32 copy of
+                       // the weight and bias (ring_affine_bytes), after the barriers
 };
 
-// Shared memory of a block: the warps' rings, then their barrier slots.
+// Shared memory of a block: the warps' rings, then their barrier slots (and,
+// for LayerNorm rows, the block's binary32 weight and bias: ring_affine_bytes).
 __host__ __device__ constexpr int ring_smem_bytes(int stages, int stage_bytes) {
   return kRingWarps * stages * stage_bytes + kRingWarps * kRingMaxStages * 8;
 }
+// The binary32 weight and bias of a LayerNorm row space of `dim` columns.
+__host__ __device__ constexpr int ring_affine_bytes(int dim) { return dim * 4 * 2; }
 
 __device__ __forceinline__ unsigned long long global_timer() {
   unsigned long long t;
@@ -130,6 +135,69 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
       ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
+}
+
+// Weight and bias of a LayerNorm row space as binary32 in shared memory,
+// written once per block (ring_affine_fill) and read as 16-byte vectors at
+// each use: [vector (w, b)][quarter of a chunk][chunk] float4s, so that the
+// lanes' reads of one quarter of their chunks are contiguous. The values are
+// those of the element type's words (widened exactly; NULL weight = ones,
+// NULL bias = zeros), so the bits of the results are those of AffineDirect.
+template <typename T>
+struct AffineSmemF32 {
+  static constexpr int Q = Elem<T>::V / 4;  // float4s per chunk and vector
+  const float4* area;
+  int nchunks;
+  __device__ __forceinline__ void get(int /*p*/, int f, F2 (&wf)[Elem<T>::P],
+                                      F2 (&bf)[Elem<T>::P]) const {
+#pragma unroll
+    for (int h = 0; h < Q; ++h) {
+      const float4 a = area[h * nchunks + f];
+      const float4 b = area[(Q + h) * nchunks + f];
+      wf[2 * h] = make_float2(a.x, a.y);
+      wf[2 * h + 1] = make_float2(a.z, a.w);
+      bf[2 * h] = make_float2(b.x, b.y);
+      bf[2 * h + 1] = make_float2(b.z, b.w);
+    }
+  }
+  __device__ __forceinline__ void edge(float& w_, float& b_) const {
+    w_ = 1.f;
+    b_ = 0.f;
+  }
+};
+
+// Every thread of the block: write segment s's weight and bias into the
+// area at 16-byte word `word` (then the caller syncs the block).
+template <typename T>
+__device__ __forceinline__ void ring_affine_fill(const Segment& s, int word) {
+  constexpr int V = Elem<T>::V;
+  constexpr int P = Elem<T>::P;
+  constexpr int Q = V / 4;
+  float4* area = reinterpret_cast<float4*>(dyn_smem + word);
+  const int n = s.dim / V;
+  const T* w = static_cast<const T*>(s.w);
+  const T* b = static_cast<const T*>(s.b);
+  for (int f = threadIdx.x; f < n; f += blockDim.x) {
+    F2 wf[P], bf[P];
+    if (w) {
+      Elem<T>::unpack(load_cached(w + (long long)f * V), wf);
+    } else {
+#pragma unroll
+      for (int j = 0; j < P; ++j) wf[j] = splat(1.f);
+    }
+    if (b) {
+      Elem<T>::unpack(load_cached(b + (long long)f * V), bf);
+    } else {
+#pragma unroll
+      for (int j = 0; j < P; ++j) bf[j] = zero2();
+    }
+#pragma unroll
+    for (int h = 0; h < Q; ++h) {
+      area[h * n + f] = make_float4(wf[2 * h].x, wf[2 * h].y, wf[2 * h + 1].x, wf[2 * h + 1].y);
+      area[(Q + h) * n + f] =
+          make_float4(bf[2 * h].x, bf[2 * h].y, bf[2 * h + 1].x, bf[2 * h + 1].y);
+    }
+  }
 }
 
 // Weight and bias of a lane's chunk slots: the packed 16-byte words of the
@@ -256,8 +324,8 @@ __device__ __forceinline__ F2 warp_sum_pair(F2 t) {
 // 16-byte words `row` and `row + pitch`. Each row takes the operations of
 // one row, in the same order (row_stats, normalize_store), so its bits are
 // those of the one-row path; the two rows' independent chains interleave,
-// their butterflies share each step's add, and each weight / bias word is
-// read and unpacked once for both rows.
+// their butterflies share each step's add, and each weight / bias value is
+// read once for both rows.
 template <typename T, int SLOTS, int VPL, typename Src>
 __device__ __forceinline__ void ring_ln_pair(const Segment& s, int row, int pitch, long long r,
                                              float eps, float inv_d, int gl, const Src& src) {
@@ -415,9 +483,13 @@ __host__ __device__ constexpr int ring_weight_slots_in_regs() {
   // weight in registers and the negated sines kept per tile 37.8 / 35.3 (the
   // negated sines alone: 40.9 / 38.5).
   if (OP == kOpRmsRopeLocal) return VPL < 4 ? VPL : 4;
-  // LayerNorm rows of a whole warp run in pairs (ring_ln_pair): two rows'
-  // values leave no room (ptxas spilled), and each weight / bias word read
-  // from L1 serves both rows
+  // LayerNorm rows read the block's binary32 copy in shared memory
+  // (AffineSmemF32): two rows' values in pairs (ring_ln_pair) leave no room
+  // for the words (ptxas spilled), and the copy also saves their unpacking.
+  // Measured on B200 (bf16, 65536 rows, cold / back to back, us), against
+  // the words read from L1 and unpacked once per pair: D = 768 37.2 / 38.3 ->
+  // 34.2 / 41.2, D = 1000 47.1 / 49.6 -> 43.0 / 51.9, D = 1024 49.5 / 51.1 ->
+  // 43.2 / 52.0; over the whole bench step the same (444 M rows/s).
   if (OP == kOpLn) return 0;
 #ifndef RN_RING_WB_BUDGET
 #define RN_RING_WB_BUDGET 48
@@ -464,8 +536,12 @@ __device__ __forceinline__ void ring_segment(const RingParams& p, RingState& rs,
   constexpr int NREG = ring_weight_slots_in_regs<T, OP, VPL>();
   using Regs = AffineRegs<T, BIAS, VPL, NREG ? NREG : 1>;
   using Direct = AffineDirect<T, BIAS, false>;
-  std::conditional_t<(NREG > 0), Regs, Direct> src;
-  if constexpr (NREG > 0)
+  // LayerNorm: the block's binary32 copy in shared memory (one row space)
+  using Smem = AffineSmemF32<T>;
+  std::conditional_t<BIAS, Smem, std::conditional_t<(NREG > 0), Regs, Direct>> src;
+  if constexpr (BIAS)
+    src = Smem{reinterpret_cast<const float4*>(dyn_smem + p.affine_word), s.dim / Elem<T>::V};
+  else if constexpr (NREG > 0)
     src.load(s, gl, G);
   else
     src = Direct{static_cast<const T*>(s.w), static_cast<const T*>(s.b)};
@@ -548,6 +624,11 @@ rows_ring_kernel(const RingParams p) {
   if (lane == 0) {
     for (int k = 0; k < S; ++k) mbar_init(&bars[k], 1);
     fence_mbar_init();
+  }
+  if constexpr (OP == kOpLn) {
+    // LayerNorm rings carry one row space (the planner's rule)
+    ring_affine_fill<T>(p.seg[0], p.affine_word);
+    __syncthreads();
   }
   __syncwarp();
   RingState rs{0, 0u, true};
