@@ -128,7 +128,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
 }
 
 // Global -> shared bulk copy of `bytes` (both addresses 16-byte aligned, a
-// multiple of 16 bytes), completion counted on `bar`. No multicast.
+// multiple of 16 bytes), completion counted on `bar`. Into this CTA's shared memory only.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
                                           uint64_t* bar) {
   asm volatile(
