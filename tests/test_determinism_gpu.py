@@ -212,7 +212,7 @@ def test_ring_waits_run_out_and_the_context_survives(dim):
 def test_ring_plans_for_the_large_workloads():
     """By default warp rings carry aligned bf16 lane-group rows that fill a
     warp (the narrow LayerNorm widths, two rows to a tile); block
-    rings carry blocks of 512+ threads (D = 16384); the rest keep the
+    rings carry LayerNorm blocks of 512+ threads (D = 16384); the rest keep the
     register kernels unless the rings are forced."""
     for dim, ring in ((768, 1), (1000, 1), (4096, 0), (8192, 0), (16384, 1), (4097, 0)):
         x = torch.empty(65536, dim, dtype=torch.bfloat16, device="cuda")
@@ -227,6 +227,9 @@ def test_ring_plans_for_the_large_workloads():
     w = torch.ones(128, dtype=torch.bfloat16, device="cuda")
     # the plain dual head norm (4 lanes per row) stays on the register kernels
     assert rn.plan(rn.RN_OP_DUAL, q, weight=w, bias=w, k=k)["staged"] == 0
+    # wide RMSNorm rows stay on the register kernels with their prefetch
+    assert rn.plan(rn.RN_OP_RMS, torch.empty(1024, 16384, dtype=torch.bfloat16,
+                                             device="cuda"))["staged"] == 0
     # binary32 rows and bf16 rows of 16 lanes stay on the register kernels
     assert rn.plan(rn.RN_OP_LN, torch.empty(4096, 1024, device="cuda"))["staged"] == 0
     x = torch.empty(4096, 512, dtype=torch.bfloat16, device="cuda")

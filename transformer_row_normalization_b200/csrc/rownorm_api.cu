@@ -559,9 +559,12 @@ bool plan_ring(int dtype, int op, const SegPlan* plans, const rn_view* const* xs
 // 722.9 us; at D = 8192 (256 threads) the register kernel with per-thread
 // prefetch stayed ahead (352.5 against 374.8 us), and at 4097 (128 threads)
 // too (204.9 against 222.2 us).
-bool cta_ring_preferred(const SegPlan& p) { return p.lanes >= 512; }
 // (Measured again after the rings' register trim: D = 16384 768.9 -> 698.2 us,
-// the same before and after a full bench run.)
+// the same before and after a full bench run.) RMSNorm rows of blocks of 512
+// threads ran faster on the register kernel with its prefetch (bf16, cold:
+// D = 16384, 32768 rows, 356.2 -> 348.3 us; D = 12288, 16384 rows, 129.5 ->
+// 123.0 us), so only LayerNorm takes the block rings by default.
+bool cta_ring_preferred(const SegPlan& p, int op) { return op == rn::kOpLn && p.lanes >= 512; }
 
 // Plans a block-ring launch for one RMSNorm / LayerNorm segment of the block
 // family (any layout): by default where cta_ring_preferred says so,
@@ -574,7 +577,7 @@ bool plan_cta_ring(int dtype, int op, const SegPlan* plans, const rn_view* const
   if (op != rn::kOpRms && op != rn::kOpLn) return false;
   const SegPlan& p = plans[0];
   if (p.family != 1) return false;
-  if (path == 0 && !cta_ring_preferred(p)) return false;
+  if (path == 0 && !cta_ring_preferred(p, op)) return false;
   const bool ex = p.exact != 0;
   const void* fn = dtype == RN_F32 ? rn::cta_ring_kernel_f32(op, ex, slots, p.lanes, p.chunks)
                                    : rn::cta_ring_kernel_bf16(op, ex, slots, p.lanes, p.chunks);
@@ -651,17 +654,20 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
       merged.family == 0 ? rn::kWarpPrefetchStages : rn::cta_prefetch_stages(threads, op);
   const int pf_bytes = rn::prefetch_slots_smem_bytes(threads, merged.chunks, stages) *
                        (rn::op_has_second(op) ? 2 : 1);
-  // Prefetch of the rows ahead where it measured faster on B200: lane groups,
-  // blocks of 256 or more threads (few blocks per SM, so few rows in
-  // flight), and blocks of 128 threads on rows off the 16-byte grid (bf16
-  // LayerNorm 65536 x 4097: 203.6 -> 200.0 us cold); aligned rows in blocks
-  // of 128 threads, which keep 8 rows per SM in flight, ran slower with it
-  // (LayerNorm 4096: 174.1 -> 177.0 us). Only when the slots fit beside the
+  // Prefetch of the rows ahead where it measured faster on B200 (bf16, 65536
+  // rows, cold): lane groups; blocks of 256 or more threads (few blocks per
+  // SM, so few rows in flight); blocks of 128 threads on rows off the
+  // 16-byte grid (LayerNorm 4097: 203.6 -> 200.0 us) and on LayerNorm rows
+  // of at most 3 chunks per thread (D = 2048: 114.8 -> 110.7 us, 3072: 143.4
+  // -> 137.2 us). Aligned rows in blocks of 128 threads otherwise keep 8 rows
+  // per SM in flight and ran slower with it (LayerNorm 4096: 174.1 -> 177.0
+  // us; RMSNorm 3072: 125.0 -> 135.3 us). Only when the slots fit beside the
   // weight cache (with a margin for the kernel's static shared memory).
   const int path = g_path_override.load(std::memory_order_relaxed);
   const bool want_prefetch =
       path == 3 ||
-      (path == 0 && (merged.family == 0 || merged.lanes >= 256 || !merged.exact));
+      (path == 0 && (merged.family == 0 || merged.lanes >= 256 || !merged.exact ||
+                     (op == rn::kOpLn && merged.chunks <= 3)));
   const int prefetch =
       !stream && want_prefetch && cache + pf_bytes <= device_info(dev).smem_per_block - 1024
           ? 1
