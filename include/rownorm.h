@@ -323,8 +323,9 @@ RN_API int rn_set_grid_override(int blocks);
 /* Kernel choice: 0 automatic; 1 register-resident kernels loading rows
  * directly; 2 the bulk-copy rings wherever the shape allows (RMSNorm and
  * LayerNorm rows, and the dual head norm with or without in-thread RoPE:
- * rows of up to 1024 columns in 16-byte aligned layouts through a ring of
- * shared-memory stages per warp, wider rows through a ring per block; all
+ * rows of up to 2048 bf16 or 1024 binary32 columns in 16-byte aligned
+ * layouts through a ring of shared-memory stages per warp, wider rows
+ * through a ring per block; all
  * filled with cp.async.bulk), the register kernels elsewhere; 3
  * register-resident kernels with a per-thread prefetch of the rows ahead
  * through shared memory (cp.async), also where the planner would not

@@ -72,19 +72,22 @@ PATH_CASES = [
     (torch.float32, 1500, 1024, 0), (torch.bfloat16, 700, 4096, 0), (torch.bfloat16, 700, 4097, 0),
     (torch.bfloat16, 600, 8192, 0), (torch.bfloat16, 300, 16384, 0), (torch.bfloat16, 100, 32768, 0),
     (torch.float32, 500, 4099, 0), (torch.float32, 200, 16384, 0), (torch.bfloat16, 900, 2048, 3),
+    (torch.bfloat16, 1100, 1536, 0), (torch.bfloat16, 801, 2048, 0), (torch.bfloat16, 700, 2056, 0),
     (torch.bfloat16, 1200, 64, 0), (torch.float32, 900, 1536, 1),
 ]
 
 
 def ring_applies(dtype, dim, offset):
     """Under rn_set_path_override(2) the rings carry every RMSNorm and
-    LayerNorm row the register kernels hold, except lane-group rows
-    (dim <= 1024) off the 16-byte grid: per-warp rings take lane-group rows
-    whose rows all start on the grid with whole 16-byte chunks, block rings
-    every wider row."""
+    LayerNorm row the register kernels hold, except lane-group rows (dim <=
+    2048 bf16, 1024 binary32: a warp of 32 lanes of at most 8 chunks) off
+    the 16-byte grid: per-warp rings take lane-group rows whose rows all
+    start on the grid with whole 16-byte chunks, block rings every wider
+    row."""
     v = 8 if dtype == torch.bfloat16 else 4
     widest = 32768 if dtype == torch.bfloat16 else 16384
-    if dim > 1024:
+    lane_widest = 2048 if dtype == torch.bfloat16 else 1024
+    if dim > lane_widest:
         return dim <= widest
     return dim % v == 0 and offset == 0
 

@@ -93,7 +93,7 @@ def test_dual_decode():
 # widths: tiny, ragged, around every family / chunk boundary, the maximum
 
 WIDTHS = [1, 2, 3, 7, 8, 9, 31, 33, 64, 100, 127, 128, 129, 255, 256, 257, 768, 1000,
-          1023, 1024, 1025, 2047, 2048, 4095, 4096, 4097, 8191, 8192, 16383, 16384]
+          1023, 1024, 1025, 1536, 2047, 2048, 2049, 4095, 4096, 4097, 8191, 8192, 16383, 16384]
 
 
 @pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])

@@ -198,7 +198,9 @@ bool same_phase(const rn_view* x, const rn_view* v) {
          ((v->outer_stride - x->outer_stride) * es) % 16 == 0;
 }
 
-constexpr int kWarpFamilyMaxDim = 1024;
+// Widest rows of the lane-group family: a warp of 32 lanes of at most 8
+// chunks (binary32 1024 columns, bf16 2048).
+int64_t warp_family_max_dim(int dtype) { return dtype == RN_F32 ? 1024 : 2048; }
 
 int pow2_ceil(int64_t v) {
   int p = 1;
@@ -241,7 +243,7 @@ SegPlan plan_segment(const rn_view* x, const rn_view* y, const void* w, const vo
     p.family = 2;
     p.lanes = rn::kStreamBlockThreads;
     p.chunks = (int)ceil_div(nfull, p.lanes);
-  } else if (D <= kWarpFamilyMaxDim) {
+  } else if (D <= warp_family_max_dim(x->dtype)) {
     p.family = 0;
     int g = pow2_ceil(ceil_div(ceil_div(D, V), per_thread));
     if (!rows_aligned && g < pow2_ceil(2 * (V - 1))) g = pow2_ceil(2 * (V - 1));

@@ -54,7 +54,7 @@ constexpr int kMinThreadsPerSm = 1024;
 template <typename T, int OP, int SLOTS, int VPL>
 __host__ __device__ constexpr int warp_blocks_per_sm() {
   if (OP != kOpLn) return 2;
-  if (Elem<T>::V == 8) return VPL == 4 && SLOTS != kSlotsFull ? 2 : 3;
+  if (Elem<T>::V == 8) return VPL >= 5 || (VPL == 4 && SLOTS != kSlotsFull) ? 2 : 3;
   return VPL >= 6 ? 2 : 3;
 }
 

@@ -4,8 +4,6 @@
 
 namespace rn {
 
-constexpr int kWarpFamilyMaxChunksF32 = 8;   // dim <= 1024: at most dim / V full chunks
-constexpr int kWarpFamilyMaxChunksBf16 = 4;  // over lanes >= dim / (4 V)
 constexpr int kCtaMinChunks = 1;             // chunks per thread, block family
 constexpr int kCtaMaxChunks = 5;
 constexpr int kTargetChunksPerThread = 4;    // 64 bytes of loads in flight per thread
