@@ -5,8 +5,10 @@
 // rownorm_core.cuh. Two families:
 //   rows_warp_kernel  a group of G lanes (a power of two <= 32) of one warp
 //                     owns a row; G is chosen so each lane holds about four
-//                     16-byte chunks. Used for D <= 1024.
-//   rows_cta_kernel   one block of NT threads owns a row. Used for D > 1024.
+//                     16-byte chunks (whole warps of up to 8 chunks per lane
+//                     for the widest rows). Used for D <= 1024 (binary32) or
+//                     2048 (bf16).
+//   rows_cta_kernel   one block of NT threads owns a row. Used above that.
 // Both are persistent: the grid is sized to the SM count times resident
 // blocks per SM, and rows are strided statically over the lane groups /
 // blocks (no atomics, no work queue, no inter-block communication, no waits
@@ -51,6 +53,8 @@ constexpr int kMinThreadsPerSm = 1024;
 // registers (bf16 rows of 4 chunks per lane with a partial last chunk;
 // binary32 rows of 6 or more chunks per lane: 2-8 % faster with 128, 1.6x at
 // D = 1001), and every RMSNorm ran as fast or faster with 128.
+// bf16 rows of 5 to 8 chunks per lane (1025 to 2048 columns) hold up to 64
+// values and take 128.
 template <typename T, int OP, int SLOTS, int VPL>
 __host__ __device__ constexpr int warp_blocks_per_sm() {
   if (OP != kOpLn) return 2;

@@ -1,7 +1,8 @@
 // Per-warp bulk-copy row rings (sm_100a), for rows whose lane groups fit in
-// one warp (dim <= 1024) in 16-byte aligned layouts: RMSNorm, LayerNorm, and
-// the q/k head RMSNorm + RoPE whose plane partners are the same thread's
-// (with each tile's token's cos / sin row staged beside the tile's rows).
+// one warp (dim <= 1024 binary32, 2048 bf16) in 16-byte aligned layouts:
+// RMSNorm, LayerNorm, and the q/k head RMSNorm + RoPE whose plane partners
+// are the same thread's (with each tile's token's cos / sin row staged
+// beside the tile's rows).
 //
 // Every warp of a block runs its own pipeline, with no block barrier: a ring
 // of S stages in shared memory, each holding one tile of R consecutive rows
