@@ -427,19 +427,19 @@ int round_up(int64_t v, int64_t m) { return (int)((v + m - 1) / m * m); }
 //   rows whose lane groups fill a warp: LayerNorm 768 45.1 / 45.1 -> 36.9 /
 //     38.4, 1000 61.5 / 62.7 -> 47.1 / 49.8, 1024 52.1 / 51.8 -> 49.1 / 50.0,
 //     RMSNorm 1024 44.9 / 51.6 -> 41.0 / 50.6;
-//   the dual head norm + split-half RoPE (q [8192, 32, 128], k [8192, 8,
-//     128]) with the token's table row staged with each tile: 43.0 / 41.1 ->
-//     36.9 / 35.2; with the table read from global memory per row the rings
-//     ran slower (47.1 -> 53.2 cold), and interleaved planes are not
-//     measured: both stay on the register kernels unless the rings are
-//     forced (plan_ring checks the staging);
+//   the dual head norm + RoPE (q [8192, 32, 128], k [8192, 8, 128]) with
+//     the token's table row staged with each tile: split-half planes 43.0 /
+//     41.1 -> 36.9 / 35.2, interleaved planes 52.2 / 49.1 -> 38.9 / 37.0;
+//     with the table read from global memory per row the rings ran slower
+//     (47.1 -> 53.2 cold), so that stays on the register kernels unless the
+//     rings are forced (plan_ring checks the staging);
 //   but the plain dual head norm (same shapes, 4 lanes per row) 26.7 / 31.2
 //     -> 30.9 / 31.5, bf16 LayerNorm 512 (16 lanes per row) 31.8 -> 34.7
 //     and binary32 LayerNorm 1024 88.1 -> 94.1 ran slower, and stay on the
 //     register kernels.
 bool ring_preferred(int dtype, int op, const SegPlan* plans, int nseg, const rn_rope* rope) {
   if (dtype != RN_BF16) return false;
-  if (op == rn::kOpRmsRopeLocal) return nseg == 2 && rope && !rope->traditional;
+  if (op == rn::kOpRmsRopeLocal) return nseg == 2 && rope;
   if (op != rn::kOpRms && op != rn::kOpLn) return false;
   for (int i = 0; i < nseg; ++i)
     if (plans[i].lanes != 32) return false;
