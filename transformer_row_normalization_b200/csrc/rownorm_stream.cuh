@@ -6,7 +6,11 @@
 // pass: RMSNorm makes two passes (sum of squares, then normalize and store),
 // LayerNorm three (sum of d = x - K with K = x_0, then sum of (d - mean)^2,
 // then normalize and store): the same shifted two-pass statistics as the
-// register kernels, so a constant row still gives exactly the bias. Passes
+// register kernels, so a constant row still gives exactly the bias. (One
+// pass of per-chunk (count, mean, squared deviations) merged by Chan et
+// al.'s formula, then the store pass, gave the same results within
+// tolerance but ran slower on B200: bf16 LayerNorm 8192 x 65536 416 -> 477
+// us; each chunk's merge waits on the last, with a division.) Passes
 // after the first find the row in L2 while the rows in flight (one or a few
 // per SM) fit there.
 //
