@@ -482,7 +482,9 @@ __host__ __device__ constexpr int ring_weight_slots_in_regs() {
   // head norm + RoPE prefill, cold / back to back: weight from L1 and sign
   // flips per row 39.7 / 37.1 us; weight in registers 38.8 / 37.0; both the
   // weight in registers and the negated sines kept per tile 37.8 / 35.3 (the
-  // negated sines alone: 40.9 / 38.5).
+  // negated sines alone: 40.9 / 38.5). A block-wide binary32 copy of the
+  // weights in shared memory instead, as for LayerNorm rows, measured the
+  // same (38.9 / 35.3).
   if (OP == kOpRmsRopeLocal) return VPL < 4 ? VPL : 4;
   // LayerNorm rows read the block's binary32 copy in shared memory
   // (AffineSmemF32): two rows' values in pairs (ring_ln_pair) leave no room
