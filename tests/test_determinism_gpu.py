@@ -133,7 +133,8 @@ def test_ring_dual_agrees_with_register_dual():
 
 @pytest.mark.parametrize("rows", [1, 2, 3, 31, 33, 597, 4096 + 3])
 @pytest.mark.parametrize("dtype,dim", [(torch.bfloat16, 768), (torch.bfloat16, 1000),
-                                       (torch.bfloat16, 128), (torch.float32, 1024),
+                                       (torch.bfloat16, 128), (torch.bfloat16, 1536),
+                                       (torch.bfloat16, 2048), (torch.float32, 1024),
                                        (torch.float32, 300)])
 def test_ring_ragged_row_counts(rows, dtype, dim):
     """Row counts that leave partial tiles, warps without tiles and a ragged
