@@ -659,7 +659,8 @@ int plan_launch(int dtype, int op, const SegPlan* plans, const rn_view* const* x
   // Prefetch of the rows ahead where it measured faster on B200 (bf16, 65536
   // rows, cold): lane groups; blocks of 256 or more threads (few blocks per
   // SM, so few rows in flight); blocks of 128 threads on rows off the
-  // 16-byte grid (LayerNorm 4097: 203.6 -> 200.0 us) and on LayerNorm rows
+  // 16-byte grid (LayerNorm 4097: 203.6 -> 200.0 us with two stages, 186.4
+  // us with one) and on LayerNorm rows
   // of at most 3 chunks per thread (D = 2048: 114.8 -> 110.7 us, 3072: 143.4
   // -> 137.2 us). Aligned rows in blocks of 128 threads otherwise keep 8 rows
   // per SM in flight and ran slower with it (LayerNorm 4096: 174.1 -> 177.0

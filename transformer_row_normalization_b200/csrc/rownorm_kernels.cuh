@@ -130,17 +130,18 @@ struct Prefetch {
 // Prefetch stages per thread: rows in flight while one is normalized from
 // registers. Measured on B200 (back-to-back bf16 LayerNorm, D = 768 to
 // 16384): lane groups keep two (a third moved them by no more than noise).
-// Blocks of 256 or more threads, which prefetch, keep one: one row in flight
-// in half the shared memory leaves L1 room for the weight and bias
-// (LayerNorm 16384: 777 -> 746 us, 8192: 357 -> 349 us against two stages;
-// a third stage cost 10-14 %). Blocks of 128 threads prefetch nothing; their
-// two queue entries issue the shift and edge loads two rows ahead (LayerNorm
-// 4097: 224 -> 219 us against one). The gated op reads its gate from the
-// stage until the row is stored, so it refills late and keeps two stages:
-// one row in flight while it normalizes.
+// Blocks keep one: one row in flight in half the shared memory leaves L1
+// room for the weight and bias and more blocks per SM (LayerNorm 16384: 777
+// -> 746 us, 8192: 357 -> 349 us against two stages, a third stage cost
+// 10-14 %; blocks of 128 threads on LayerNorm 4097, which prefetch: 200.7 ->
+// 186.4 us, 8 blocks per SM instead of 6; RMSNorm and LayerNorm 4096, which
+// do not prefetch, unchanged). The gated op reads its gate from the stage
+// until the row is stored, so it refills late and keeps two stages: one row
+// in flight while it normalizes.
 constexpr int kWarpPrefetchStages = 2;
 __host__ __device__ constexpr int cta_prefetch_stages(int threads, int op) {
-  return threads >= 256 && op != kOpGatedRms ? 1 : 2;
+  (void)threads;
+  return op != kOpGatedRms ? 1 : 2;
 }
 
 // 16-byte words of prefetch slots of one bank.
