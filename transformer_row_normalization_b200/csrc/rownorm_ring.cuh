@@ -766,9 +766,11 @@ __device__ __forceinline__ void cta_ring_rows(const RingParams& p, const Segment
 // Rows in flight per block ring: NST - 1 while one is normalized.
 // Stages of a block ring. Measured on B200 (bf16 LayerNorm 65536 x 16384,
 // 512 threads, cold): two stages 699 us, three 774 us (and blocks of 1024
-// threads at two chunks each 1191 us; one block of 512 threads per SM, with
-// 128 registers holding the weight and bias, 3 or 4 stages: 965-975 us, its
-// two reduction barriers per row no longer overlapped by a second block).
+// threads at two chunks each 1191 us; blocks of 256 threads at eight chunks
+// each, 128 registers, 776 us (ptxas spilled 68 bytes); one block of 512
+// threads per SM, with 128 registers holding the weight and bias, 3 or 4
+// stages: 965-975 us, its two reduction barriers per row no longer
+// overlapped by a second block).
 __host__ __device__ constexpr int cta_ring_stages(int threads) { return threads >= 512 ? 2 : 3; }
 
 // Register budget: the rows ahead wait in the ring, not in registers, so
